@@ -1,0 +1,230 @@
+// C-ABI entry points of libfathom: argument checks, pointer classification,
+// kernel launches.  Declarations and contracts: include/fathom.h.
+#include <mutex>
+
+#include "fathom_internal.cuh"
+
+namespace fathom {
+namespace {
+
+// Status word written by kernels (FATHOM_DEV_* bits); one per device.
+__device__ unsigned int g_status;
+
+constexpr int kMaxDevices = 64;
+unsigned int* g_status_ptr[kMaxDevices] = {};
+std::mutex g_status_mu;
+
+// Where a pointer lives.  Returns the device-usable address through `dev`.
+enum class Where { kDevice, kHostPinned, kOther };
+
+Where classify(const void* p, const void** dev) {
+    cudaPointerAttributes a;
+    cudaError_t e = cudaPointerGetAttributes(&a, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return Where::kOther;
+    }
+    if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) {
+        if (dev) *dev = p;
+        return Where::kDevice;
+    }
+    if (a.type == cudaMemoryTypeHost && a.devicePointer != nullptr) {
+        if (dev) *dev = a.devicePointer;
+        return Where::kHostPinned;
+    }
+    return Where::kOther;
+}
+
+bool is_device(const void* p) { return p != nullptr && classify(p, nullptr) == Where::kDevice; }
+
+bool dims_ok(int Hkv, int d) { return Hkv >= 1 && d >= 32 && d <= kMaxD && d % 32 == 0; }
+
+bool heads_ok(int Hq, int Hkv) {
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv) return false;
+    int G = Hq / Hkv;
+    return G == 1 || G == 2 || G == 4 || G == 8;
+}
+
+bool scan_fits(int d, int Hq, int Hkv) { return scan_smem_bytes(d, Hq / Hkv) <= kMaxSmem; }
+
+int to_status(cudaError_t e) { return e == cudaSuccess ? FATHOM_OK : FATHOM_ECUDA; }
+
+// Resolve a store's arrays to device-usable addresses, checking residency.
+int resolve_store(const fathom_store* s, const uint32_t** planes, const uint16_t** scales) {
+    if (!s || !s->planes || !s->scales) return FATHOM_EINVAL;
+    if (!dims_ok(s->n_kv_heads, s->d) || s->n < 1 || s->n_pad != n_pad_of(s->n)) return FATHOM_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(s->planes) & 15) || (reinterpret_cast<uintptr_t>(s->scales) & 1))
+        return FATHOM_EINVAL;
+    const void* dp = nullptr;
+    const void* ds = nullptr;
+    Where wp = classify(s->planes, &dp), ws = classify(s->scales, &ds);
+    Where want = s->host_resident ? Where::kHostPinned : Where::kDevice;
+    if (wp != want || ws != want) return FATHOM_EINVAL;
+    *planes = static_cast<const uint32_t*>(dp);
+    *scales = static_cast<const uint16_t*>(ds);
+    return FATHOM_OK;
+}
+
+}  // namespace
+
+unsigned int* device_status_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_status_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<unsigned int*>(p);
+    }
+    return g_status_ptr[dev];
+}
+
+}  // namespace fathom
+
+using namespace fathom;
+
+extern "C" {
+
+int64_t fathom_n_pad(int64_t n) { return n < 0 ? 0 : n_pad_of(n); }
+
+size_t fathom_planes_bytes(int n_kv_heads, int d, int64_t n) {
+    if (!dims_ok(n_kv_heads, d) || n < 1) return 0;
+    return (size_t)n_kv_heads * d * 4 * (size_t)(n_pad_of(n) / 8);
+}
+
+size_t fathom_scales_bytes(int n_kv_heads, int d, int64_t n) {
+    if (!dims_ok(n_kv_heads, d) || n < 1) return 0;
+    return (size_t)n_kv_heads * d * (size_t)(n_pad_of(n) / kBlock) * sizeof(uint16_t);
+}
+
+int fathom_pack_bitplanes(const void* K, int k_dtype, int n_kv_heads, int64_t n, int d, uint32_t* planes,
+                          uint16_t* scales, fathom_stream_t stream) {
+    if (!K || !planes || !scales || n < 1 || !dims_ok(n_kv_heads, d)) return FATHOM_EINVAL;
+    if (k_dtype != FATHOM_F32 && k_dtype != FATHOM_BF16) return FATHOM_EINVAL;
+    if (!is_device(K) || !is_device(planes) || !is_device(scales)) return FATHOM_EINVAL;
+    if (!device_status_ptr()) return FATHOM_ECUDA;
+    return to_status(launch_pack(K, k_dtype, n_kv_heads, n, d, planes, scales, (cudaStream_t)stream));
+}
+
+int fathom_alloc_depths(const void* q, int q_dtype, const float* sigma2, int n_q_heads, int n_kv_heads, int d,
+                        int budget_bits, int fixed_r, uint8_t* depths, fathom_stream_t stream) {
+    if (!q || !sigma2 || !depths || !dims_ok(n_kv_heads, d) || n_q_heads < 1 || n_q_heads % n_kv_heads)
+        return FATHOM_EINVAL;
+    if (q_dtype != FATHOM_F32 && q_dtype != FATHOM_BF16) return FATHOM_EINVAL;
+    if (budget_bits < 0 || fixed_r < 0 || fixed_r > d) return FATHOM_EINVAL;
+    if (!is_device(q) || !is_device(sigma2) || !is_device(depths)) return FATHOM_EINVAL;
+    return to_status(launch_depths(q, q_dtype, sigma2, n_q_heads, n_kv_heads, d, budget_bits, fixed_r, depths,
+                                   (cudaStream_t)stream));
+}
+
+int fathom_scan_scores(const fathom_store* store, const void* q, int q_dtype, const uint8_t* depths,
+                       int n_q_heads, float* scores, fathom_stream_t stream) {
+    const uint32_t* planes;
+    const uint16_t* scales;
+    int rc = resolve_store(store, &planes, &scales);
+    if (rc) return rc;
+    if (!q || !depths || !scores || !heads_ok(n_q_heads, store->n_kv_heads)) return FATHOM_EINVAL;
+    if (q_dtype != FATHOM_F32 && q_dtype != FATHOM_BF16) return FATHOM_EINVAL;
+    if (!is_device(q) || !is_device(depths) || !is_device(scores)) return FATHOM_EINVAL;
+    if (!scan_fits(store->d, n_q_heads, store->n_kv_heads)) return FATHOM_EUNSUPPORTED;
+    if (!device_status_ptr()) return FATHOM_ECUDA;
+    return to_status(launch_scan(planes, scales, store->n_kv_heads, store->d, store->n, store->n_pad, q, q_dtype,
+                                 depths, n_q_heads, scores, (cudaStream_t)stream));
+}
+
+size_t fathom_topk_workspace_bytes(int64_t n, int n_rows, int k) {
+    if (n < 1 || n_rows < 1 || k < 1 || k > kMaxTopK) return 0;
+    return topk_workspace_bytes(n, n_rows, k);
+}
+
+int fathom_topk(const float* scores, int64_t n, int64_t ld, int n_rows, int k, int32_t* idx, float* top_scores,
+                void* workspace, size_t workspace_bytes, fathom_stream_t stream) {
+    if (!scores || !idx || !workspace || n < 1 || ld < n || n_rows < 1 || k < 1 || k > n || k > kMaxTopK ||
+        n > INT32_MAX)
+        return FATHOM_EINVAL;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return FATHOM_EINVAL;
+    if (workspace_bytes < topk_workspace_bytes(n, n_rows, k)) return FATHOM_ENOMEM;
+    if (!is_device(scores) || !is_device(idx) || !is_device(workspace) || (top_scores && !is_device(top_scores)))
+        return FATHOM_EINVAL;
+    if (!device_status_ptr()) return FATHOM_ECUDA;
+    return to_status(launch_topk(scores, n, ld, n_rows, k, idx, top_scores, workspace, (cudaStream_t)stream));
+}
+
+size_t fathom_scan_workspace_bytes(const fathom_store* store, int n_q_heads, int k) {
+    if (!store || n_q_heads < 1 || k < 1 || k > kMaxTopK || store->n < 1) return 0;
+    size_t scores = ((sizeof(float) * (size_t)n_q_heads * (size_t)n_pad_of(store->n)) + 255) & ~size_t(255);
+    return scores + topk_workspace_bytes(store->n, n_q_heads, k);
+}
+
+int fathom_scan_topk(const fathom_store* store, const void* q, int q_dtype, const uint8_t* depths, int n_q_heads,
+                     int k, int32_t* idx, float* top_scores, void* workspace, size_t workspace_bytes,
+                     fathom_stream_t stream) {
+    const uint32_t* planes;
+    const uint16_t* scales;
+    int rc = resolve_store(store, &planes, &scales);
+    if (rc) return rc;
+    if (!q || !depths || !idx || !workspace || !heads_ok(n_q_heads, store->n_kv_heads)) return FATHOM_EINVAL;
+    if (q_dtype != FATHOM_F32 && q_dtype != FATHOM_BF16) return FATHOM_EINVAL;
+    if (k < 1 || k > store->n || k > kMaxTopK || store->n > INT32_MAX) return FATHOM_EINVAL;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return FATHOM_EINVAL;
+    if (workspace_bytes < fathom_scan_workspace_bytes(store, n_q_heads, k)) return FATHOM_ENOMEM;
+    if (!scan_fits(store->d, n_q_heads, store->n_kv_heads)) return FATHOM_EUNSUPPORTED;
+    if (!is_device(q) || !is_device(depths) || !is_device(idx) || !is_device(workspace) ||
+        (top_scores && !is_device(top_scores)))
+        return FATHOM_EINVAL;
+    if (!device_status_ptr()) return FATHOM_ECUDA;
+    float* scores = static_cast<float*>(workspace);
+    size_t off = ((sizeof(float) * (size_t)n_q_heads * (size_t)store->n_pad) + 255) & ~size_t(255);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = launch_scan(planes, scales, store->n_kv_heads, store->d, store->n, store->n_pad, q, q_dtype,
+                                depths, n_q_heads, scores, s);
+    if (e != cudaSuccess) return FATHOM_ECUDA;
+    e = launch_topk(scores, store->n, store->n_pad, n_q_heads, k, idx, top_scores,
+                    static_cast<char*>(workspace) + off, s);
+    return to_status(e);
+}
+
+int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
+                         int rows_host_resident, const int32_t* idx, int n_q_heads, int n_kv_heads, int64_t n,
+                         int d, int k, float* out, fathom_stream_t stream) {
+    if (!q || !K_rows || !V_rows || !idx || !out || n < 1 || k < 1 || !dims_ok(n_kv_heads, d) ||
+        !heads_ok(n_q_heads, n_kv_heads))
+        return FATHOM_EINVAL;
+    if (q_dtype != FATHOM_F32 && q_dtype != FATHOM_BF16) return FATHOM_EINVAL;
+    if (d != 32 && d != 64 && d != 128 && d != 256) return FATHOM_EUNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(K_rows) & 15) || (reinterpret_cast<uintptr_t>(V_rows) & 15))
+        return FATHOM_EINVAL;
+    const void* kd = nullptr;
+    const void* vd = nullptr;
+    Where want = rows_host_resident ? Where::kHostPinned : Where::kDevice;
+    if (classify(K_rows, &kd) != want || classify(V_rows, &vd) != want) return FATHOM_EINVAL;
+    if (!is_device(q) || !is_device(idx) || !is_device(out)) return FATHOM_EINVAL;
+    if (!device_status_ptr()) return FATHOM_ECUDA;
+    return to_status(launch_attend(q, q_dtype, static_cast<const uint16_t*>(kd), static_cast<const uint16_t*>(vd),
+                                   idx, n_q_heads, n_kv_heads, n, d, k, out, (cudaStream_t)stream));
+}
+
+int fathom_last_device_status(fathom_stream_t stream) {
+    unsigned int* p = device_status_ptr();
+    if (!p) return -FATHOM_ECUDA;
+    unsigned int v = 0;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(&v, p, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return -FATHOM_ECUDA;
+    if (cudaMemsetAsync(p, 0, sizeof(v), s) != cudaSuccess) return -FATHOM_ECUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return -FATHOM_ECUDA;
+    return (int)v;
+}
+
+const char* fathom_status_string(int status) {
+    switch (status) {
+        case FATHOM_OK: return "ok";
+        case FATHOM_EINVAL: return "invalid argument";
+        case FATHOM_ENOMEM: return "workspace or buffer too small";
+        case FATHOM_ECUDA: return "CUDA error";
+        case FATHOM_ETIMEOUT: return "bounded device wait timed out";
+        case FATHOM_EUNSUPPORTED: return "unsupported shape or dtype";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

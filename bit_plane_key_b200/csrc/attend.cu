@@ -1,0 +1,191 @@
+// K5: exact attention over the selected keys only.
+//
+// ai-feeds.com summary, 方法 · 输出: each query produces top-k key indices and
+// true attention is then computed over those keys.
+//   o_h = sum_j p_j V[g][idx_j],  p = softmax_j(q_h . K[g][idx_j] / sqrt(d)),
+// g = h / (Hq/Hkv), K and V rows in bf16, fp32 accumulation, exp via exp2f.
+//
+// One thread-block cluster of kSplit CTAs per query head.  CTA r of the
+// cluster takes rows j = r, r + kSplit, ... of the head's k selected keys;
+// inside it each warp runs an online softmax over its rows (lane l holds
+// channels [l*d/32, (l+1)*d/32)).  The warps' partial (max, sum, o) merge in
+// shared memory, then CTA 0 merges the kSplit CTA partials through
+// distributed shared memory and writes o_h.  No workspace and no second
+// kernel.  Rows may live in device memory or in page-locked host memory.
+#include <cooperative_groups.h>
+
+#include "fathom_internal.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace fathom {
+namespace {
+
+constexpr int kSplit = 8;      // CTAs per head (cluster size)
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kUnroll = 4;     // rows in flight per warp
+
+template <int V>  // channels per lane: d / 32
+struct Row {
+    float x[V];
+};
+
+template <int V>
+__device__ __forceinline__ void load_row(const uint16_t* __restrict__ p, float* out) {
+    // V consecutive bf16 values
+    if constexpr (V == 4) {
+        uint2 u = *reinterpret_cast<const uint2*>(p);
+        out[0] = __uint_as_float(u.x << 16);
+        out[1] = __uint_as_float(u.x & 0xFFFF0000u);
+        out[2] = __uint_as_float(u.y << 16);
+        out[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    } else if constexpr (V == 8) {
+        uint4 u = *reinterpret_cast<const uint4*>(p);
+        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            out[2 * e] = __uint_as_float(w[e] << 16);
+            out[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+        }
+    } else if constexpr (V == 2) {
+        uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+        out[0] = __uint_as_float(u << 16);
+        out[1] = __uint_as_float(u & 0xFFFF0000u);
+    } else {
+#pragma unroll
+        for (int e = 0; e < V; ++e) out[e] = __uint_as_float((uint32_t)p[e] << 16);
+    }
+}
+
+template <int V>
+__global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kThreads)
+attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restrict__ Kr,
+              const uint16_t* __restrict__ Vr, const int32_t* __restrict__ idx, int Hq, int Hkv, int64_t n,
+              int k, float* __restrict__ out, unsigned int* status) {
+    constexpr int d = V * 32;
+    __shared__ float s_m[kWarps], s_l[kWarps];
+    __shared__ float s_o[kWarps][d];
+    __shared__ float c_m, c_l;        // this CTA's merged partial (read by CTA 0)
+    __shared__ float c_o[d];
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int r = (int)cluster.block_rank();
+    const int h = blockIdx.x / kSplit;
+    const int g = h / (Hq / Hkv);
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    const float scale = 1.4426950408889634f / sqrtf((float)d);  // log2(e)/sqrt(d)
+
+    float qv[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) qv[e] = load_q(q, q_dtype, (int64_t)h * d + lane * V + e) * scale;
+
+    float m = -INFINITY, l = 0.0f, o[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) o[e] = 0.0f;
+
+    const int32_t* ih = idx + (int64_t)h * k;
+    const int64_t head_base = (int64_t)g * n * d;
+    // rows of this warp: j = r + kSplit * (wp + kWarps * s)
+    const int stride = kSplit * kWarps;
+    for (int j0 = r + kSplit * wp; j0 < k; j0 += stride * kUnroll) {
+        float kv[kUnroll][V], vv[kUnroll][V];
+        bool ok[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            int j = j0 + u * stride;
+            ok[u] = false;
+            if (j < k) {
+                int64_t i = ih[j];
+                if (i >= 0 && i < n) {
+                    ok[u] = true;
+                    const int64_t off = head_base + i * d + lane * V;
+                    load_row<V>(Kr + off, kv[u]);
+                    load_row<V>(Vr + off, vv[u]);
+                } else if (lane == 0) {
+                    atomicOr(status, (unsigned)FATHOM_DEV_BAD_INDEX);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            float dot = 0.0f;
+#pragma unroll
+            for (int e = 0; e < V; ++e) dot = fmaf(qv[e], kv[u][e], dot);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+            if (!ok[u]) continue;   // warp-uniform
+            float mn = fmaxf(m, dot);
+            float a = exp2f(m - mn);     // 0 when m = -inf
+            float p = exp2f(dot - mn);
+            l = l * a + p;
+#pragma unroll
+            for (int e = 0; e < V; ++e) o[e] = fmaf(p, vv[u][e], o[e] * a);
+            m = mn;
+        }
+    }
+
+    // merge the warps of this CTA
+    if (lane == 0) {
+        s_m[wp] = m;
+        s_l[wp] = l;
+    }
+#pragma unroll
+    for (int e = 0; e < V; ++e) s_o[wp][lane * V + e] = o[e];
+    __syncthreads();
+    if (threadIdx.x < d) {
+        float M = -INFINITY;
+        for (int x = 0; x < kWarps; ++x) M = fmaxf(M, s_m[x]);
+        float L = 0.0f, O = 0.0f;
+        for (int x = 0; x < kWarps; ++x) {
+            float f = (s_m[x] == -INFINITY) ? 0.0f : exp2f(s_m[x] - M);
+            L = fmaf(s_l[x], f, L);
+            O = fmaf(s_o[x][threadIdx.x], f, O);
+        }
+        c_o[threadIdx.x] = O;
+        if (threadIdx.x == 0) {
+            c_m = M;
+            c_l = L;
+        }
+    }
+    cluster.sync();
+    if (r == 0 && threadIdx.x < d) {
+        float Ms[kSplit], Ls[kSplit], Os[kSplit];
+        float M = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < kSplit; ++x) {
+            Ms[x] = *cluster.map_shared_rank(&c_m, x);
+            Ls[x] = *cluster.map_shared_rank(&c_l, x);
+            Os[x] = cluster.map_shared_rank(c_o, x)[threadIdx.x];
+            M = fmaxf(M, Ms[x]);
+        }
+        float L = 0.0f, O = 0.0f;
+#pragma unroll
+        for (int x = 0; x < kSplit; ++x) {
+            float f = (Ms[x] == -INFINITY) ? 0.0f : exp2f(Ms[x] - M);
+            L = fmaf(Ls[x], f, L);
+            O = fmaf(Os[x], f, O);
+        }
+        out[(int64_t)h * d + threadIdx.x] = (L > 0.0f) ? O / L : 0.0f;
+    }
+    cluster.sync();   // keep every CTA's shared memory alive until CTA 0 has read it
+}
+
+}  // namespace
+
+cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
+                          const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k, float* out,
+                          cudaStream_t stream) {
+    dim3 grid((unsigned)(Hq * kSplit));
+    unsigned int* st = device_status_ptr();
+    switch (d) {
+        case 32: attend_kernel<1><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, out, st); break;
+        case 64: attend_kernel<2><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, out, st); break;
+        case 128: attend_kernel<4><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, out, st); break;
+        case 256: attend_kernel<8><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, out, st); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace fathom

@@ -1,0 +1,59 @@
+// Internal declarations shared by the CUDA translation units of libfathom.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "fathom.h"
+
+namespace fathom {
+
+constexpr int kBlock = 64;     // tokens per shared block scale
+constexpr int kPad = 128;      // key padding granule of the store
+constexpr int kMaxD = 256;     // largest supported head dimension
+constexpr int kMaxTopK = 4096; // largest supported k
+constexpr size_t kMaxSmem = 227 * 1024;  // opt-in shared memory per CTA on sm_100
+
+inline int64_t n_pad_of(int64_t n) { return ((n + kPad - 1) / kPad) * kPad; }
+
+// Per-device status word (FATHOM_DEV_* bits); its device address is passed
+// to every kernel that can set a bit.
+unsigned int* device_status_ptr();
+
+// Host launchers (each enqueues on `stream`; arguments already validated).
+cudaError_t launch_pack(const void* K, int k_dtype, int Hkv, int64_t n, int d, uint32_t* planes,
+                        uint16_t* scales, cudaStream_t stream);
+cudaError_t launch_depths(const void* q, int q_dtype, const float* sigma2, int Hq, int Hkv, int d,
+                          int budget, int fixed_r, uint8_t* depths, cudaStream_t stream);
+size_t scan_smem_bytes(int d, int G);
+cudaError_t launch_scan(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n,
+                        int64_t n_pad, const void* q, int q_dtype, const uint8_t* depths, int Hq,
+                        float* scores, cudaStream_t stream);
+size_t topk_workspace_bytes(int64_t n, int rows, int k);
+cudaError_t launch_topk(const float* scores, int64_t n, int64_t ld, int rows, int k, int32_t* idx,
+                        float* top_scores, void* ws, cudaStream_t stream);
+cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
+                          const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k, float* out,
+                          cudaStream_t stream);
+
+// fp32 <-> order-preserving u32: a > b as floats  <=>  key(a) > key(b).
+__device__ __forceinline__ uint32_t float_to_ordered(float f) {
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ordered_to_float(uint32_t k) {
+    uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+    return __uint_as_float(u);
+}
+
+__device__ __forceinline__ float load_q(const void* q, int dtype, int64_t i) {
+    if (dtype == FATHOM_BF16) {
+        uint16_t b = static_cast<const uint16_t*>(q)[i];
+        return __uint_as_float(static_cast<uint32_t>(b) << 16);
+    }
+    return static_cast<const float*>(q)[i];
+}
+
+}  // namespace fathom

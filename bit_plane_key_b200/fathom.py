@@ -1,0 +1,218 @@
+"""Python binding of libfathom (the C ABI in include/fathom.h).
+
+Argument marshalling only: every step of the scan runs in the library's CUDA
+kernels.  Tensors are torch tensors (device memory, or page-locked host memory
+for host-resident stores and rows); torch is used for allocation and streams.
+If libfathom.so is missing this module raises at import: there is no CPU or
+fallback path.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfathom.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("libfathom.so is not built; run `python -m bit_plane_key_b200.build` (needs nvcc)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, EINVAL, ENOMEM, ECUDA, ETIMEOUT, EUNSUPPORTED = range(6)
+F32, BF16 = 0, 1
+DEV_BAD_DEPTH, DEV_BAD_INDEX, DEV_TOPK_OVERFLOW = 1, 2, 4
+MAX_TOPK = 4096
+
+
+class FathomError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        msg = _lib.fathom_status_string(status).decode()
+        super().__init__("%s: %s (status %d)" % (what, msg, status))
+
+
+class fathom_store(ctypes.Structure):
+    _fields_ = [("n_kv_heads", ctypes.c_int32), ("d", ctypes.c_int32), ("n", ctypes.c_int64),
+                ("n_pad", ctypes.c_int64), ("host_resident", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("planes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+_P, _I, _L, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+_SP = ctypes.POINTER(fathom_store)
+
+
+def _sig(name, res, args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = args
+    return f
+
+
+_sig("fathom_n_pad", _L, [_L])
+_sig("fathom_planes_bytes", _Z, [_I, _I, _L])
+_sig("fathom_scales_bytes", _Z, [_I, _I, _L])
+_sig("fathom_pack_bitplanes", _I, [_P, _I, _I, _L, _I, _P, _P, _P])
+_sig("fathom_alloc_depths", _I, [_P, _I, _P, _I, _I, _I, _I, _I, _P, _P])
+_sig("fathom_scan_scores", _I, [_SP, _P, _I, _P, _I, _P, _P])
+_sig("fathom_topk_workspace_bytes", _Z, [_L, _I, _I])
+_sig("fathom_topk", _I, [_P, _L, _L, _I, _I, _P, _P, _P, _Z, _P])
+_sig("fathom_scan_workspace_bytes", _Z, [_SP, _I, _I])
+_sig("fathom_scan_topk", _I, [_SP, _P, _I, _P, _I, _I, _P, _P, _P, _Z, _P])
+_sig("fathom_sparse_attend", _I, [_P, _I, _P, _P, _I, _P, _I, _I, _L, _I, _I, _P, _P])
+_sig("fathom_last_device_status", _I, [_P])
+_sig("fathom_status_string", ctypes.c_char_p, [_I])
+
+
+def lib():
+    """The loaded ctypes library (for calls with raw pointers)."""
+    return _lib
+
+
+def _check(rc, what):
+    if rc != OK:
+        raise FathomError(rc, what)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype in (torch.bfloat16, torch.int16, torch.uint16):
+        return BF16
+    raise TypeError("expected float32 or bfloat16, got %s" % t.dtype)
+
+
+def n_pad(n):
+    return int(_lib.fathom_n_pad(int(n)))
+
+
+class Store:
+    """A packed bit-plane store: planes u32 [Hkv][d][4][n_pad/32], scales u16 [Hkv][d][n_pad/64]."""
+
+    def __init__(self, planes, scales, n, host_resident=None):
+        self.planes, self.scales, self.n = planes, scales, int(n)
+        self.n_kv_heads, self.d = int(planes.shape[0]), int(planes.shape[1])
+        self.n_pad = n_pad(n)
+        self.host_resident = (not planes.is_cuda) if host_resident is None else bool(host_resident)
+        self._c = fathom_store(self.n_kv_heads, self.d, self.n, self.n_pad, int(self.host_resident), 0,
+                               planes.data_ptr(), scales.data_ptr())
+
+    @property
+    def c(self):
+        return ctypes.byref(self._c)
+
+    def to_host(self):
+        """Copy of this store in page-locked host memory (host-resident)."""
+        return Store(self.planes.cpu().pin_memory(), self.scales.cpu().pin_memory(), self.n, host_resident=True)
+
+    def plane_bytes_read(self, union_depths):
+        """Plane + scale bytes a scan reads for union depths U [Hkv][d]."""
+        U = union_depths.to(torch.int64)
+        return int(U.sum()) * self.n_pad // 8 + int((U > 0).sum()) * (self.n_pad // 64) * 2
+
+
+def pack_bitplanes(K, planes=None, scales=None, stream=None):
+    """K [Hkv][n][d] (float32 or bfloat16, cuda) -> Store."""
+    Hkv, n, d = K.shape
+    npad = n_pad(n)
+    if planes is None:
+        planes = torch.empty((Hkv, d, 4, npad // 32), dtype=torch.int32, device=K.device)
+    if scales is None:
+        scales = torch.empty((Hkv, d, npad // 64), dtype=torch.int16, device=K.device)
+    _check(_lib.fathom_pack_bitplanes(_ptr(K), _dtype_code(K), Hkv, n, d, _ptr(planes), _ptr(scales),
+                                      _stream(stream)), "fathom_pack_bitplanes")
+    return Store(planes, scales, n, host_resident=False)
+
+
+def alloc_depths(q, sigma2, budget_bits, fixed_r=0, out=None, stream=None):
+    """q [Hq][d], sigma2 f32 [Hkv][d] -> depths u8 [Hq][d]."""
+    Hq, d = q.shape
+    Hkv = sigma2.shape[0]
+    if out is None:
+        out = torch.empty((Hq, d), dtype=torch.uint8, device=q.device)
+    _check(_lib.fathom_alloc_depths(_ptr(q), _dtype_code(q), _ptr(sigma2), Hq, Hkv, d, int(budget_bits),
+                                    int(fixed_r), _ptr(out), _stream(stream)), "fathom_alloc_depths")
+    return out
+
+
+def scan_scores(store, q, depths, out=None, stream=None):
+    """Scores f32 [Hq][n_pad] (padding keys -inf)."""
+    Hq = q.shape[0]
+    if out is None:
+        out = torch.empty((Hq, store.n_pad), dtype=torch.float32, device=q.device)
+    _check(_lib.fathom_scan_scores(store.c, _ptr(q), _dtype_code(q), _ptr(depths), Hq, _ptr(out),
+                                   _stream(stream)), "fathom_scan_scores")
+    return out
+
+
+def topk_workspace_bytes(n, rows, k):
+    return int(_lib.fathom_topk_workspace_bytes(int(n), int(rows), int(k)))
+
+
+def topk(scores, n, k, idx=None, top_scores=None, workspace=None, stream=None):
+    """Top-k of score rows [rows][ld] over the first n columns."""
+    rows, ld = scores.shape
+    if idx is None:
+        idx = torch.empty((rows, k), dtype=torch.int32, device=scores.device)
+    if top_scores is None:
+        top_scores = torch.empty((rows, k), dtype=torch.float32, device=scores.device)
+    nb = topk_workspace_bytes(n, rows, k)
+    if workspace is None:
+        workspace = torch.empty(max(nb, 1), dtype=torch.uint8, device=scores.device)
+    _check(_lib.fathom_topk(_ptr(scores), int(n), int(ld), rows, int(k), _ptr(idx), _ptr(top_scores),
+                            _ptr(workspace), workspace.numel(), _stream(stream)), "fathom_topk")
+    return idx, top_scores
+
+
+def scan_workspace_bytes(store, n_q_heads, k):
+    return int(_lib.fathom_scan_workspace_bytes(store.c, int(n_q_heads), int(k)))
+
+
+def scan_topk(store, q, depths, k, idx=None, top_scores=None, workspace=None, stream=None):
+    """idx i32 [Hq][k] and top scores f32 [Hq][k]."""
+    Hq = q.shape[0]
+    if idx is None:
+        idx = torch.empty((Hq, k), dtype=torch.int32, device=q.device)
+    if top_scores is None:
+        top_scores = torch.empty((Hq, k), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(scan_workspace_bytes(store, Hq, k), 1), dtype=torch.uint8, device=q.device)
+    _check(_lib.fathom_scan_topk(store.c, _ptr(q), _dtype_code(q), _ptr(depths), Hq, int(k), _ptr(idx),
+                                 _ptr(top_scores), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "fathom_scan_topk")
+    return idx, top_scores
+
+
+def scan_scores_view(workspace, n_q_heads, n_pad_keys):
+    """The scan's scores inside a fathom_scan_topk workspace: f32 [Hq][n_pad]."""
+    return workspace[: 4 * n_q_heads * n_pad_keys].view(torch.float32).view(n_q_heads, n_pad_keys)
+
+
+def sparse_attend(q, K_rows, V_rows, idx, n_kv_heads=None, out=None, stream=None):
+    """o f32 [Hq][d]; K_rows/V_rows bf16 [Hkv][n][d] on the device or page-locked host."""
+    Hq, d = q.shape
+    Hkv, n, _ = K_rows.shape
+    k = idx.shape[1]
+    host = not K_rows.is_cuda
+    if out is None:
+        out = torch.empty((Hq, d), dtype=torch.float32, device=q.device)
+    _check(_lib.fathom_sparse_attend(_ptr(q), _dtype_code(q), _ptr(K_rows), _ptr(V_rows), int(host), _ptr(idx),
+                                     Hq, Hkv, n, d, int(k), _ptr(out), _stream(stream)), "fathom_sparse_attend")
+    return out
+
+
+def last_device_status(stream=None):
+    v = _lib.fathom_last_device_status(_stream(stream))
+    if v < 0:
+        raise FathomError(-v, "fathom_last_device_status")
+    return v

@@ -1,0 +1,217 @@
+/*
+ * fathom.h -- C ABI of the Fathom variable-depth bit-plane key scan for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What the method computes (page title, then section):
+ *   "Fathom: Per-Query Read Depth for Sparse Decoding over Offloaded KV Caches"
+ *   (arXiv 2609.17652 abstract): a 4-bit K cache stored channel-major as bit
+ *   planes, so that a prefix of t planes is exactly the channel's t-bit
+ *   quantizer; each query spends a bit budget by reverse water-filling over the
+ *   variance-weighted importance of its channels; the scan ranks all n keys
+ *   for a top-k step.
+ *   "Fathom:面向卸载 KV Cache 的稀疏解码的逐查询读取深度" (ai-feeds.com summary),
+ *   方法 · 关键模块 1-5: bit-plane store, per-query read depth by reverse
+ *   water-filling, per-layer budgets, basis rule (paper Sec 3.5), scan kernel
+ *   that pulls only budgeted planes and outputs top-k indices; 输出: true
+ *   attention over the selected keys.
+ *   evolve.pub review, Strengths: one shared block scale (paper Sec 3.2),
+ *   depth rule from the 4x-per-bit error reduction (Sec 3.3), contiguous
+ *   host-link runs (Sec 3.6).
+ *
+ * Conventions for every entry point:
+ *   - The caller owns all memory.  Only the one entry point marked otherwise
+ *     ever touches memory it did not receive; no call allocates.
+ *   - Device pointers must be cudaMalloc'd (or equivalent) on the current
+ *     device.  "Host-resident" pointers must be page-locked host memory
+ *     (cudaHostAlloc / cudaHostRegister), mapped into the device address space
+ *     (always true with unified addressing on 64-bit Linux).
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream) and
+ *     return after enqueueing.  Argument errors are detected on the host
+ *     before any launch and return FATHOM_EINVAL; nothing has been enqueued.
+ *     FATHOM_ECUDA means a CUDA API or launch error (cudaGetLastError is
+ *     left set for the caller to inspect).
+ *   - Kernels never trap or assert.  Problems only the device can see (a
+ *     depth above 4, an out-of-range index) are recorded in a per-device
+ *     status word that fathom_last_device_status() reads and clears; the
+ *     offending element is skipped.
+ *   - Layouts are row-major C arrays; the shapes below use the names
+ *     Hkv = number of KV heads, Hq = number of query heads (a multiple of
+ *     Hkv, query head h reads KV head h / (Hq/Hkv)), d = head dimension
+ *     (a multiple of 32, at most 256), n = number of keys,
+ *     n_pad = n rounded up to a multiple of 128.
+ */
+#ifndef FATHOM_H
+#define FATHOM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* fathom_stream_t;
+
+enum {
+    FATHOM_OK = 0,
+    FATHOM_EINVAL = 1,       /* bad argument (null pointer, size, alignment, pinning) */
+    FATHOM_ENOMEM = 2,       /* caller-provided workspace or buffer too small */
+    FATHOM_ECUDA = 3,        /* CUDA runtime or launch error */
+    FATHOM_ETIMEOUT = 4,     /* a bounded device wait gave up (device status only) */
+    FATHOM_EUNSUPPORTED = 5  /* valid but unsupported shape or dtype */
+};
+
+typedef enum { FATHOM_F32 = 0, FATHOM_BF16 = 1 } fathom_dtype;
+
+/* Bits of the device status word (fathom_last_device_status). */
+enum {
+    FATHOM_DEV_BAD_DEPTH = 1u << 0,   /* a depth above 4 was read; that channel was skipped */
+    FATHOM_DEV_BAD_INDEX = 1u << 1,   /* an index outside [0,n) reached sparse attention; skipped */
+    FATHOM_DEV_TOPK_OVERFLOW = 1u << 2 /* internal: a top-k buffer overflowed (never expected) */
+};
+
+/*
+ * The packed K index of one layer (bit-plane store).
+ *   planes  u32 [Hkv][d][4][n_pad/32]: bit (i % 32) of word (i / 32) of plane j
+ *           holds bit (3-j) of key i's 4-bit code (plane 0 = most significant);
+ *           padding keys hold 0.  A channel's four planes are contiguous, so the
+ *           first t planes of a channel are one contiguous run of t*n_pad/8
+ *           bytes.
+ *   scales  u16 [Hkv][d][n_pad/64]: fp16 bit pattern of the block scale Delta
+ *           of (KV head, channel, 64-token block); 0 for all-padding blocks.
+ *   host_resident: 0 = both arrays in device memory, 1 = both in page-locked
+ *           host memory (the scan then streams only the budgeted planes over
+ *           the host link).
+ */
+typedef struct {
+    int32_t n_kv_heads;
+    int32_t d;
+    int64_t n;
+    int64_t n_pad;
+    int32_t host_resident;
+    int32_t reserved;
+    const uint32_t* planes;
+    const uint16_t* scales;
+} fathom_store;
+
+/* n rounded up to a multiple of 128; the padded key count of a store. */
+int64_t fathom_n_pad(int64_t n);
+/* Bytes of the planes / scales arrays of a store; 0 for invalid sizes. */
+size_t fathom_planes_bytes(int n_kv_heads, int d, int64_t n);
+size_t fathom_scales_bytes(int n_kv_heads, int d, int64_t n);
+
+/*
+ * Pack a K cache into the bit-plane store (quantize + plane layout).
+ * [ai-feeds summary 关键模块 1; evolve.pub Strengths (Sec 3.2); FAQ "How does
+ *  Fathom's bit-plane KV cache work?"]
+ * For each (KV head, channel, 64-token block): amax = max |x| over the
+ * block's real keys, Delta = fp16_rn(amax/8), code = clamp(floor(x/Delta),
+ * -8, 7) + 8 (code 8 when Delta = 0; floor taken on the exact quotient).
+ *   K       device, [Hkv][n][d], dtype FATHOM_F32 or FATHOM_BF16; finite values.
+ *   planes  device, fathom_planes_bytes() bytes, fully overwritten.
+ *   scales  device, fathom_scales_bytes() bytes, fully overwritten.
+ * To build a host-resident store, pack into device buffers and copy them to
+ * page-locked host memory.
+ * Errors: EINVAL for null pointers, n < 1, Hkv < 1, d not a multiple of 32
+ * or d > 256, unknown dtype.
+ */
+int fathom_pack_bitplanes(const void* K, int k_dtype, int n_kv_heads, int64_t n, int d,
+                          uint32_t* planes, uint16_t* scales, fathom_stream_t stream);
+
+/*
+ * Per-query read depths.
+ * [arXiv abstract; ai-feeds summary 关键模块 2-3; evolve.pub Strengths (Sec 3.3)]
+ * fixed_r == 0: reverse water-filling.  w_c = fl32(fl32(q_c*q_c)*sigma2_c)
+ *   (IEEE fp32, no fused multiply-add); the candidates (c,t), t = 0..3,
+ *   valued w_c 4^-t, are ordered by value descending, then c ascending, then
+ *   t ascending; the first min(budget_bits, 4d) are taken and depth t_c is
+ *   the number taken on channel c.  So sum_c t_c = min(B, 4d).
+ * fixed_r > 0: comparison scans at a fixed depth: 4 planes on the fixed_r
+ *   channels with the largest |q_c| (ties to the lower channel), 0 elsewhere
+ *   (r = 16 is the "68-bit" scan, r = 32 the "136-bit" one).
+ *   q       device, [Hq][d], FATHOM_F32 or FATHOM_BF16.
+ *   sigma2  device, f32 [Hkv][d], the per-channel key statistic (>= 0).
+ *   depths  device, u8 [Hq][d], overwritten.
+ * Errors: EINVAL for null pointers, budget_bits < 0, fixed_r < 0 or > d,
+ * Hq not a multiple of Hkv, d not a multiple of 32 or d > 256.
+ */
+int fathom_alloc_depths(const void* q, int q_dtype, const float* sigma2, int n_q_heads,
+                        int n_kv_heads, int d, int budget_bits, int fixed_r, uint8_t* depths,
+                        fathom_stream_t stream);
+
+/*
+ * Variable-depth scan: approximate scores of every key for every query head.
+ * [ai-feeds summary 关键模块 4 (basis rule, paper Sec 3.5) and 5; arXiv abstract]
+ * s[h][i] = sum_c q[h][c] * Delta[b(i)][c] * sum_{j < t[h][c]} (2 b_{i,c,j} - 1) 2^(2-j)
+ * Only the first U_c = max over the KV group of t[h][c] planes of channel c
+ * are read; planes beyond are never touched.
+ *   store   a packed store (device or host-resident).
+ *   q       device, [Hq][d], FATHOM_F32 or FATHOM_BF16.
+ *   depths  device, u8 [Hq][d], values 0..4.
+ *   scores  device, f32 [Hq][store->n_pad]; keys >= n are written -inf.
+ * Errors: EINVAL as above, or a host-resident store whose pointers are not
+ * page-locked, or a device store whose pointers are not device memory.
+ */
+int fathom_scan_scores(const fathom_store* store, const void* q, int q_dtype, const uint8_t* depths,
+                       int n_q_heads, float* scores, fathom_stream_t stream);
+
+/*
+ * Top-k of score rows: the k largest of scores[r][0..n), ties to the lower
+ * index, listed in that order.  [ai-feeds summary 关键模块 5, 输出]
+ *   scores      device, f32 [n_rows][ld] (ld >= n); NaN is not allowed.
+ *   idx         device, i32 [n_rows][k].
+ *   top_scores  device, f32 [n_rows][k], or NULL.
+ *   workspace   device, at least fathom_topk_workspace_bytes(n, n_rows, k) bytes,
+ *               256-byte aligned; contents need not be initialised.
+ * Errors: EINVAL for k < 1, k > n, k > 4096, n_rows < 1; ENOMEM for a short
+ * workspace.
+ */
+size_t fathom_topk_workspace_bytes(int64_t n, int n_rows, int k);
+int fathom_topk(const float* scores, int64_t n, int64_t ld, int n_rows, int k, int32_t* idx,
+                float* top_scores, void* workspace, size_t workspace_bytes, fathom_stream_t stream);
+
+/*
+ * Scan + top-k of one decode step of one layer (fathom_scan_scores followed
+ * by fathom_topk on the scores, which live in the workspace).
+ *   idx         device, i32 [Hq][k].
+ *   top_scores  device, f32 [Hq][k], or NULL.
+ *   workspace   device, fathom_scan_workspace_bytes(store, Hq, k) bytes,
+ *               256-byte aligned.
+ */
+size_t fathom_scan_workspace_bytes(const fathom_store* store, int n_q_heads, int k);
+int fathom_scan_topk(const fathom_store* store, const void* q, int q_dtype, const uint8_t* depths,
+                     int n_q_heads, int k, int32_t* idx, float* top_scores, void* workspace,
+                     size_t workspace_bytes, fathom_stream_t stream);
+
+/*
+ * Exact attention over the selected keys only.  [ai-feeds summary 输出]
+ * out[h] = softmax_j(q[h] . K[g][idx[h][j]] / sqrt(d)) V[g][idx[h][j]],
+ * g = h / (Hq/Hkv), fp32 accumulation.
+ *   q       device, [Hq][d], FATHOM_F32 or FATHOM_BF16.
+ *   K_rows, V_rows  bf16 bit patterns [Hkv][n][d]; device memory, or
+ *           page-locked host memory when rows_host_resident = 1.
+ *   idx     device, i32 [Hq][k], each in [0, n) (others are skipped and
+ *           flagged FATHOM_DEV_BAD_INDEX).
+ *   out     device, f32 [Hq][d].
+ * Errors: EINVAL for null pointers, k < 1, bad head counts, d not a
+ * multiple of 32 or d > 256, rows not where rows_host_resident says.
+ */
+int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
+                         int rows_host_resident, const int32_t* idx, int n_q_heads, int n_kv_heads,
+                         int64_t n, int d, int k, float* out, fathom_stream_t stream);
+
+/*
+ * Reads and clears this device's status word (FATHOM_DEV_* bits) after
+ * synchronising `stream`.  Returns the bits (>= 0), or -FATHOM_ECUDA.
+ */
+int fathom_last_device_status(fathom_stream_t stream);
+
+/* Static description of a status code. */
+const char* fathom_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FATHOM_H */

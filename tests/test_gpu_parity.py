@@ -1,0 +1,384 @@
+"""GPU parity: every step of the path through the C ABI against the oracle.
+
+Bit-exact: packing (planes and scales), depths, top-k indices of given
+scores.  Tolerance: scan scores, |s_gpu - s_ref| <= 1e-4 * sum_c |q_c khat_c|
+(fp32 accumulation of at most 2d terms; worst case a few 1e-5); attention,
+||o - o_ref|| <= 1e-3 ||o_ref||.  Top-k of the scan against the fp64 oracle:
+equal index sets except keys whose fp64 score lies within the score
+tolerance of the k-th score.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+from bit_plane_key_b200 import fathom as F  # noqa: E402
+
+DEV = torch.device("cuda:0")
+SCORE_RTOL = 1e-4
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def dev(a):
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).to(DEV)
+    if a.dtype == np.uint32:
+        return torch.from_numpy(a.view(np.int32)).to(DEV)
+    return torch.from_numpy(a).to(DEV)
+
+
+def bf16(a_bits):
+    return dev(a_bits).view(torch.bfloat16)
+
+
+def host(t, dtype=None):
+    a = t.detach().cpu().numpy()
+    return a.view(dtype) if dtype is not None else a
+
+
+def make(config=1, n=None, Hkv=None, Hq=None, d=None, q_bf16=None, values=False, needles=None, layer=0):
+    inp = synth.layer_inputs(config, layer=layer, n=n, n_kv_heads=Hkv, n_q_heads=Hq, d=d, with_values=values,
+                             needles=needles)
+    if q_bf16 is not None and q_bf16 and "q_bf16" not in inp:
+        inp["q_bf16"] = synth.f32_to_bf16_bits(inp["q"])
+        inp["q"] = synth.bf16_bits_to_f32(inp["q_bf16"])
+    return inp
+
+
+def q_dev(inp):
+    return bf16(inp["q_bf16"]) if "q_bf16" in inp else dev(inp["q"])
+
+
+def check_scores(ref, planes_np, scales_np, n, q, dep, s_gpu, i0=0, i1=None):
+    i1 = n if i1 is None else i1
+    s_ref, a_ref = ref.scores(planes_np, scales_np, n, q, dep, i0, i1, with_abs=True)
+    err = np.abs(s_gpu[:, i0:i1].astype(np.float64) - s_ref)
+    tol = SCORE_RTOL * a_ref + 1e-30
+    bad = err > tol
+    assert not bad.any(), "score mismatch at %s: gpu %s ref %s" % (
+        np.argwhere(bad)[:5].tolist(), s_gpu[:, i0:i1][bad][:5], s_ref[bad][:5])
+    return s_ref, a_ref
+
+
+# --------------------------------------------------------------------------
+# a0: packing, bit-exact
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("n,Hkv,d", [(4096, 1, 128), (1, 1, 32), (63, 2, 64), (64, 1, 32), (4097, 2, 128),
+                                     (1000, 3, 256), (130, 1, 96)])
+def test_pack_bit_exact(ref, n, Hkv, d):
+    inp = make(1, n=n, Hkv=Hkv, Hq=Hkv, d=d)
+    K = inp["K"]
+    K[0, : min(n, 64), 0] = 0.0          # an all-zero block: Delta = 0
+    st = F.pack_bitplanes(dev(K))
+    planes, scales = ref.pack(K)
+    assert np.array_equal(host(st.planes, np.uint32), planes)
+    assert np.array_equal(host(st.scales, np.uint16), scales)
+
+
+def test_pack_bf16_input(ref):
+    inp = make(1, n=777, Hkv=2, Hq=2, d=128)
+    kb = synth.f32_to_bf16_bits(inp["K"])
+    st = F.pack_bitplanes(bf16(kb))
+    planes, scales = ref.pack(synth.bf16_bits_to_f32(kb))
+    assert np.array_equal(host(st.planes, np.uint32), planes)
+    assert np.array_equal(host(st.scales, np.uint16), scales)
+
+
+def test_pack_edge_values(ref):
+    """Keys at cell edges, +-amax, tiny and huge magnitudes."""
+    rng = np.random.default_rng(5)
+    n, d = 256, 32
+    K = (rng.standard_normal((1, n, d)) * 10.0 ** rng.integers(-6, 6, (1, 1, d))).astype(np.float32)
+    for c in range(d):
+        amax = np.max(np.abs(K[0, :64, c]))
+        delta = np.float32(np.float16(amax / np.float32(8)))
+        K[0, 1:17, c] = (np.arange(-8, 8) * delta).astype(np.float32)   # exact cell edges
+        K[0, 17, c] = -amax
+    st = F.pack_bitplanes(dev(K))
+    planes, scales = ref.pack(K)
+    assert np.array_equal(host(st.planes, np.uint32), planes)
+    assert np.array_equal(host(st.scales, np.uint16), scales)
+
+
+# --------------------------------------------------------------------------
+# a1-a2, a7: depths, bit-exact
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("d", [32, 128, 256])
+@pytest.mark.parametrize("qtype", ["f32", "bf16"])
+def test_depths_bit_exact(ref, d, qtype):
+    rng = np.random.default_rng(d)
+    Hkv, G = 2, 4
+    sig = synth.channel_sigma(rng, Hkv, d)
+    s2 = (sig * sig).astype(np.float32)
+    q = rng.standard_normal((Hkv * G, d)).astype(np.float32)
+    q[0, :5] = 0.0
+    q[1] = 1.0                          # equal importances: tie rule
+    if qtype == "bf16":
+        qb = synth.f32_to_bf16_bits(q)
+        qd, qf = bf16(qb), synth.bf16_bits_to_f32(qb)
+    else:
+        qd, qf = dev(q), q
+    s2d = dev(s2)
+    for B in (0, 1, 7, 46, 64, 68, 92, 136, 4 * d - 1, 4 * d, 4 * d + 50):
+        got = host(F.alloc_depths(qd, s2d, B))
+        want = ref.alloc_depths(qf, s2, B)
+        assert np.array_equal(got, want), B
+        assert np.all(got.sum(1) == min(B, 4 * d))
+    for r in (1, 16, 32, d):
+        got = host(F.alloc_depths(qd, s2d, 0, fixed_r=r))
+        assert np.array_equal(got, ref.alloc_depths(qf, s2, 0, fixed_r=r)), r
+
+
+def test_depths_extreme_importance(ref):
+    """Subnormal, zero and huge importances keep the exact order."""
+    d = 128
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal((4, d)).astype(np.float32)
+    s2 = np.exp(rng.uniform(-100, 80, (1, d))).astype(np.float32)
+    s2[0, :4] = [0.0, 1e-45, 3e38, 1e-40]
+    for B in (10, 92, 300):
+        got = host(F.alloc_depths(dev(q), dev(s2), B))
+        assert np.array_equal(got, ref.alloc_depths(q, s2, B)), B
+
+
+# --------------------------------------------------------------------------
+# a4: scan scores within tolerance (+ the basis rule at every depth)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("case", ["config1", "gqa_ragged", "d256_g2", "g8", "depth_mix"])
+def test_scan_scores(ref, case):
+    if case == "config1":
+        inp = make(1)                                       # Hkv=1, n=4096, d=128, f32 q
+        B = 64
+    elif case == "gqa_ragged":
+        inp = make(2, n=5000, Hkv=2, Hq=8, d=128)           # bf16 q, GQA 4, ragged tail
+        B = 92
+    elif case == "d256_g2":
+        inp = make(1, n=3000, Hkv=2, Hq=4, d=256)
+        B = 136
+    elif case == "g8":
+        inp = make(2, n=1100, Hkv=1, Hq=8, d=64)
+        B = 46
+    else:
+        inp = make(1, n=2100, Hkv=1, Hq=4, d=128)
+        B = None
+    K, q = inp["K"], inp["q"]
+    n = K.shape[1]
+    st = F.pack_bitplanes(dev(K))
+    planes, scales = ref.pack(K)
+    if B is None:   # arbitrary depths 0..4 in every head: heads read less than the union
+        dep = np.random.default_rng(3).integers(0, 5, q.shape).astype(np.uint8)
+    else:
+        dep = ref.alloc_depths(q, inp["sigma2"], B)
+    s = host(F.scan_scores(st, q_dev(inp), dev(dep)))
+    assert s.shape == (q.shape[0], F.n_pad(n))
+    assert np.all(np.isneginf(s[:, n:]))
+    check_scores(ref, planes, scales, n, q, dep, s)
+
+
+def test_scan_all_depths_uniform(ref):
+    """t = 0..4 for every channel: full-depth and zero-depth corners."""
+    inp = make(1, n=700, Hkv=1, Hq=1, d=128)
+    st = F.pack_bitplanes(dev(inp["K"]))
+    planes, scales = ref.pack(inp["K"])
+    for t in range(5):
+        dep = np.full((1, 128), t, np.uint8)
+        s = host(F.scan_scores(st, dev(inp["q"]), dev(dep)))
+        if t == 0:
+            assert np.all(s[:, :700] == 0.0)
+        check_scores(ref, planes, scales, 700, inp["q"], dep, s)
+
+
+def test_scan_bad_depth_flagged(ref):
+    inp = make(1, n=256, Hkv=1, Hq=1, d=32)
+    st = F.pack_bitplanes(dev(inp["K"]))
+    dep = np.full((1, 32), 2, np.uint8)
+    dep[0, 3] = 9
+    F.last_device_status()
+    s = host(F.scan_scores(st, dev(inp["q"]), dev(dep)))
+    assert F.last_device_status() & F.DEV_BAD_DEPTH
+    planes, scales = ref.pack(inp["K"])
+    dep[0, 3] = 0            # the bad channel is skipped
+    check_scores(ref, planes, scales, 256, inp["q"], dep, s)
+    assert F.last_device_status() == 0
+
+
+def test_six_key_example_on_gpu():
+    with open(os.path.join(GOLDEN, "six_key_example.json")) as f:
+        ex = json.load(f)
+    K = np.array(ex["keys_x"], np.float32)[None]
+    q = np.array(ex["q"], np.float32)[None]
+    s2 = np.array(ex["sigma2"], np.float32)[None]
+    # d must be a multiple of 32: pad channels with zero keys, zero q, zero sigma2
+    Kp = np.zeros((1, 6, 32), np.float32)
+    Kp[:, :, :4] = K
+    qp = np.zeros((1, 32), np.float32)
+    qp[:, :4] = q
+    s2p = np.zeros((1, 32), np.float32)
+    s2p[:, :4] = s2
+    st = F.pack_bitplanes(dev(Kp))
+    for B, want in ex["expected_scores"].items():
+        dep = host(F.alloc_depths(dev(qp), dev(s2p), int(B)))
+        assert dep[0, :4].tolist() == ex["expected_depths"][B]
+        s = host(F.scan_scores(st, dev(qp), dev(dep)))[0, :6]
+        np.testing.assert_allclose(s, want, rtol=0, atol=1e-5)
+        idx, _ = F.scan_topk(st, dev(qp), dev(dep), 3)
+        assert host(idx)[0].tolist() == ex["expected_top3"][B]
+
+
+# --------------------------------------------------------------------------
+# a5: top-k, bit-exact on given scores
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("n,rows,k,kind", [
+    (100, 3, 1, "normal"), (100, 3, 100, "normal"), (4096, 2, 64, "normal"), (20000, 4, 2048, "normal"),
+    (131072, 2, 2048, "normal"), (200000, 2, 4096, "ties"), (50000, 2, 2048, "equal"),
+    (70000, 2, 1000, "narrow"), (9000, 1, 9000, "ties")])
+def test_topk_bit_exact(ref, n, rows, k, kind):
+    rng = np.random.default_rng(n + k)
+    if kind == "normal":
+        s = rng.standard_normal((rows, n)).astype(np.float32)
+    elif kind == "ties":
+        s = np.round(rng.standard_normal((rows, n)), 1).astype(np.float32)
+    elif kind == "equal":
+        s = np.full((rows, n), 1.5, np.float32)
+        s[:, ::7] = -2.0
+    else:  # one octave, 12-bit bins overflow: forces the deeper levels
+        s = (1.0 + rng.random((rows, n)) * 1e-3).astype(np.float32)
+    ld = n + 5
+    sd = torch.full((rows, ld), float("nan"), device=DEV)
+    sd[:, :n] = dev(s)
+    idx, top = F.topk(sd, n, k)
+    idx, top = host(idx), host(top)
+    for r in range(rows):
+        want = ref.topk(s[r], k)
+        assert np.array_equal(idx[r], want), r
+        assert np.array_equal(top[r], s[r][want])
+    assert F.last_device_status() == 0
+
+
+# --------------------------------------------------------------------------
+# a4 + a5 against the fp64 oracle
+# --------------------------------------------------------------------------
+def topk_sets_agree(ref, s_ref, a_ref, idx_gpu, k):
+    """Equal sets, except keys whose fp64 score is within tolerance of the k-th."""
+    want = ref.topk(s_ref, k)
+    kth = s_ref[want[-1]]
+    band = np.abs(s_ref - kth) <= 2 * SCORE_RTOL * a_ref
+    gw, ww = set(idx_gpu.tolist()), set(want.tolist())
+    diff = gw.symmetric_difference(ww)
+    assert all(band[i] for i in diff), sorted(diff)[:10]
+
+
+@pytest.mark.parametrize("config,n,Hkv,Hq,B,k", [(1, 4096, 1, 1, 64, 64), (2, 9000, 2, 8, 92, 2048),
+                                                 (2, 20000, 1, 4, 68, 1024), (2, 3000, 2, 8, 0, 16)])
+def test_scan_topk_vs_fp64(ref, config, n, Hkv, Hq, B, k):
+    inp = make(config, n=n, Hkv=Hkv, Hq=Hq)
+    K, q = inp["K"], inp["q"]
+    st = F.pack_bitplanes(dev(K))
+    planes, scales = ref.pack(K)
+    dep = host(F.alloc_depths(q_dev(inp), dev(inp["sigma2"]), B))
+    assert np.array_equal(dep, ref.alloc_depths(q, inp["sigma2"], B))
+    idx, top = F.scan_topk(st, q_dev(inp), dev(dep), k)
+    idx, top = host(idx), host(top)
+    s_ref, a_ref = ref.scores(planes, scales, n, q, dep, with_abs=True)
+    for h in range(Hq):
+        topk_sets_agree(ref, s_ref[h], a_ref[h], idx[h], k)
+        assert np.all(np.diff(top[h]) <= 0)
+        assert len(set(idx[h].tolist())) == k
+    if B == 0:
+        assert np.array_equal(idx, np.tile(np.arange(k), (Hq, 1)))
+
+
+def test_scan_topk_consistent_with_own_scores(ref):
+    """Given the scan's own fp32 scores, the top-k is exactly (score desc, index asc)."""
+    inp = make(2, n=12345, Hkv=2, Hq=8)
+    st = F.pack_bitplanes(dev(inp["K"]))
+    dep = F.alloc_depths(q_dev(inp), dev(inp["sigma2"]), 92)
+    ws = torch.empty(F.scan_workspace_bytes(st, 8, 512), dtype=torch.uint8, device=DEV)
+    idx, top = F.scan_topk(st, q_dev(inp), dep, 512, workspace=ws)
+    s = host(F.scan_scores_view(ws, 8, st.n_pad))[:, :12345]
+    idx = host(idx)
+    for h in range(8):
+        order = np.lexsort((np.arange(12345), -s[h].astype(np.float64)))[:512]
+        assert np.array_equal(idx[h], order)
+
+
+# --------------------------------------------------------------------------
+# a3: host-resident store gives the same scan
+# --------------------------------------------------------------------------
+def test_host_resident_store(ref):
+    inp = make(2, n=7000, Hkv=2, Hq=8)
+    st = F.pack_bitplanes(dev(inp["K"]))
+    hst = st.to_host()
+    dep = F.alloc_depths(q_dev(inp), dev(inp["sigma2"]), 92)
+    s_dev = host(F.scan_scores(st, q_dev(inp), dep))
+    s_host = host(F.scan_scores(hst, q_dev(inp), dep))
+    assert np.array_equal(s_dev, s_host)
+    i_dev, _ = F.scan_topk(st, q_dev(inp), dep, 700)
+    i_host, _ = F.scan_topk(hst, q_dev(inp), dep, 700)
+    assert np.array_equal(host(i_dev), host(i_host))
+    planes, scales = ref.pack(inp["K"])
+    check_scores(ref, planes, scales, 7000, inp["q"], host(dep), s_host)
+
+
+def test_residency_mismatch_rejected():
+    inp = make(1, n=300, Hkv=1, Hq=1, d=32)
+    st = F.pack_bitplanes(dev(inp["K"]))
+    dep = F.alloc_depths(dev(inp["q"]), dev(inp["sigma2"]), 10)
+    pageable = F.Store(st.planes.cpu(), st.scales.cpu(), 300, host_resident=True)
+    with pytest.raises(F.FathomError) as e:
+        F.scan_scores(pageable, dev(inp["q"]), dep)
+    assert e.value.status == F.EINVAL
+    wrong = F.Store(st.planes, st.scales, 300, host_resident=True)
+    with pytest.raises(F.FathomError):
+        F.scan_scores(wrong, dev(inp["q"]), dep)
+    with pytest.raises(F.FathomError) as e:
+        F.scan_topk(st, dev(inp["q"]), dep, 301)
+    assert e.value.status == F.EINVAL
+    with pytest.raises(F.FathomError) as e:
+        F.scan_topk(st, dev(inp["q"]), dep, 10, workspace=torch.empty(64, dtype=torch.uint8, device=DEV))
+    assert e.value.status == F.ENOMEM
+
+
+# --------------------------------------------------------------------------
+# a6: exact sparse attention
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("d,k,host_rows", [(128, 2048, False), (128, 5, False), (64, 300, False), (256, 64, False),
+                                           (32, 1, False), (128, 1000, True)])
+def test_sparse_attend(ref, d, k, host_rows):
+    rng = np.random.default_rng(d + k)
+    Hkv, G, n = 2, 4, 5000
+    inp = make(2, n=n, Hkv=Hkv, Hq=Hkv * G, d=d, values=True)
+    idx = np.stack([rng.choice(n, k, replace=False) for _ in range(Hkv * G)]).astype(np.int32)
+    Kr, Vr = bf16(inp["K_rows"]), bf16(inp["V_rows"])
+    if host_rows:
+        Kr, Vr = Kr.cpu().pin_memory(), Vr.cpu().pin_memory()
+    out = host(F.sparse_attend(q_dev(inp), Kr, Vr, dev(idx)))
+    want = ref.attend(inp["q"], inp["K_rows"], inp["V_rows"], idx)
+    for h in range(Hkv * G):
+        assert np.linalg.norm(out[h] - want[h]) <= 1e-3 * np.linalg.norm(want[h]), h
+    assert F.last_device_status() == 0
+
+
+def test_sparse_attend_bad_index_flagged(ref):
+    inp = make(2, n=300, Hkv=1, Hq=4, d=128, values=True)
+    idx = np.tile(np.arange(10, dtype=np.int32), (4, 1))
+    idx[1, 3] = 300
+    idx[2, 0] = -1
+    F.last_device_status()
+    out = host(F.sparse_attend(q_dev(inp), bf16(inp["K_rows"]), bf16(inp["V_rows"]), dev(idx)))
+    assert F.last_device_status() & F.DEV_BAD_INDEX
+    want = ref.attend(inp["q"][:1], inp["K_rows"], inp["V_rows"], idx[:1])
+    assert np.linalg.norm(out[0] - want[0]) <= 1e-3 * np.linalg.norm(want[0])
+    ok = np.delete(idx[1], 3)[None]
+    want1 = ref.attend(inp["q"][1:2], inp["K_rows"], inp["V_rows"], ok)
+    assert np.linalg.norm(out[1] - want1[0]) <= 1e-3 * np.linalg.norm(want1[0])
