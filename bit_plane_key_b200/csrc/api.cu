@@ -215,6 +215,16 @@ int fathom_last_device_status(fathom_stream_t stream) {
     return (int)v;
 }
 
+int fathom_read_probe(const void* src, size_t bytes, int host_resident, uint64_t* sink, int ctas,
+                      fathom_stream_t stream) {
+    if (!src || !sink || bytes < 16 || (bytes & 15) || (reinterpret_cast<uintptr_t>(src) & 15) || ctas < 1)
+        return FATHOM_EINVAL;
+    const void* d = nullptr;
+    Where want = host_resident ? Where::kHostPinned : Where::kDevice;
+    if (classify(src, &d) != want || !is_device(sink)) return FATHOM_EINVAL;
+    return to_status(launch_probe(d, bytes, reinterpret_cast<unsigned long long*>(sink), ctas, (cudaStream_t)stream));
+}
+
 const char* fathom_status_string(int status) {
     switch (status) {
         case FATHOM_OK: return "ok";

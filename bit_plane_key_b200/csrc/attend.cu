@@ -26,10 +26,6 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kUnroll = 4;     // rows in flight per warp
 
-template <int V>  // channels per lane: d / 32
-struct Row {
-    float x[V];
-};
 
 template <int V>
 __device__ __forceinline__ void load_row(const uint16_t* __restrict__ p, float* out) {
@@ -133,40 +129,43 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
 #pragma unroll
     for (int e = 0; e < V; ++e) s_o[wp][lane * V + e] = o[e];
     __syncthreads();
-    if (threadIdx.x < d) {
+    {
         float M = -INFINITY;
         for (int x = 0; x < kWarps; ++x) M = fmaxf(M, s_m[x]);
-        float L = 0.0f, O = 0.0f;
+        float f[kWarps];
+        float L = 0.0f;
         for (int x = 0; x < kWarps; ++x) {
-            float f = (s_m[x] == -INFINITY) ? 0.0f : exp2f(s_m[x] - M);
-            L = fmaf(s_l[x], f, L);
-            O = fmaf(s_o[x][threadIdx.x], f, O);
+            f[x] = (s_m[x] == -INFINITY) ? 0.0f : exp2f(s_m[x] - M);
+            L = fmaf(s_l[x], f[x], L);
         }
-        c_o[threadIdx.x] = O;
+        for (int c = threadIdx.x; c < d; c += kThreads) {
+            float O = 0.0f;
+            for (int x = 0; x < kWarps; ++x) O = fmaf(s_o[x][c], f[x], O);
+            c_o[c] = O;
+        }
         if (threadIdx.x == 0) {
             c_m = M;
             c_l = L;
         }
     }
     cluster.sync();
-    if (r == 0 && threadIdx.x < d) {
-        float Ms[kSplit], Ls[kSplit], Os[kSplit];
-        float M = -INFINITY;
+    if (r == 0) {
+        float f[kSplit];
+        float M = -INFINITY, L = 0.0f;
+#pragma unroll
+        for (int x = 0; x < kSplit; ++x) M = fmaxf(M, *cluster.map_shared_rank(&c_m, x));
 #pragma unroll
         for (int x = 0; x < kSplit; ++x) {
-            Ms[x] = *cluster.map_shared_rank(&c_m, x);
-            Ls[x] = *cluster.map_shared_rank(&c_l, x);
-            Os[x] = cluster.map_shared_rank(c_o, x)[threadIdx.x];
-            M = fmaxf(M, Ms[x]);
+            float mx = *cluster.map_shared_rank(&c_m, x);
+            f[x] = (mx == -INFINITY) ? 0.0f : exp2f(mx - M);
+            L = fmaf(*cluster.map_shared_rank(&c_l, x), f[x], L);
         }
-        float L = 0.0f, O = 0.0f;
+        for (int c = threadIdx.x; c < d; c += kThreads) {
+            float O = 0.0f;
 #pragma unroll
-        for (int x = 0; x < kSplit; ++x) {
-            float f = (Ms[x] == -INFINITY) ? 0.0f : exp2f(Ms[x] - M);
-            L = fmaf(Ls[x], f, L);
-            O = fmaf(Os[x], f, O);
+            for (int x = 0; x < kSplit; ++x) O = fmaf(cluster.map_shared_rank(c_o, x)[c], f[x], O);
+            out[(int64_t)h * d + c] = (L > 0.0f) ? O / L : 0.0f;
         }
-        out[(int64_t)h * d + threadIdx.x] = (L > 0.0f) ? O / L : 0.0f;
     }
     cluster.sync();   // keep every CTA's shared memory alive until CTA 0 has read it
 }

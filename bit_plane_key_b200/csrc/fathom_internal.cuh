@@ -38,6 +38,9 @@ cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, co
                           const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k, float* out,
                           cudaStream_t stream);
 
+cudaError_t launch_probe(const void* src, size_t bytes, unsigned long long* sink, int ctas,
+                         cudaStream_t stream);
+
 // fp32 <-> order-preserving u32: a > b as floats  <=>  key(a) > key(b).
 __device__ __forceinline__ uint32_t float_to_ordered(float f) {
     uint32_t u = __float_as_uint(f);

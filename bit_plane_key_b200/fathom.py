@@ -62,6 +62,7 @@ _sig("fathom_scan_topk", _I, [_SP, _P, _I, _P, _I, _I, _P, _P, _P, _Z, _P])
 _sig("fathom_sparse_attend", _I, [_P, _I, _P, _P, _I, _P, _I, _I, _L, _I, _I, _P, _P])
 _sig("fathom_last_device_status", _I, [_P])
 _sig("fathom_status_string", ctypes.c_char_p, [_I])
+_sig("fathom_read_probe", _I, [_P, _Z, _I, _P, _I, _P])
 
 
 def lib():
@@ -216,3 +217,12 @@ def last_device_status(stream=None):
     if v < 0:
         raise FathomError(-v, "fathom_last_device_status")
     return v
+
+
+def read_probe(src, sink, ctas=None, stream=None):
+    """Stream all of `src` (device or page-locked host tensor) through the SMs."""
+    host = not src.is_cuda
+    if ctas is None:
+        ctas = torch.cuda.get_device_properties(sink.device).multi_processor_count * 8
+    _check(_lib.fathom_read_probe(_ptr(src), src.numel() * src.element_size(), int(host), _ptr(sink), int(ctas),
+                                  _stream(stream)), "fathom_read_probe")

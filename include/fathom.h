@@ -19,8 +19,8 @@
  *   host-link runs (Sec 3.6).
  *
  * Conventions for every entry point:
- *   - The caller owns all memory.  Only the one entry point marked otherwise
- *     ever touches memory it did not receive; no call allocates.
+ *   - The caller owns all memory; no call allocates.  The library's only
+ *     state is one status word per device (see below).
  *   - Device pointers must be cudaMalloc'd (or equivalent) on the current
  *     device.  "Host-resident" pointers must be page-locked host memory
  *     (cudaHostAlloc / cudaHostRegister), mapped into the device address space
@@ -206,6 +206,18 @@ int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, con
  * synchronising `stream`.  Returns the bits (>= 0), or -FATHOM_ECUDA.
  */
 int fathom_last_device_status(fathom_stream_t stream);
+
+/*
+ * Measurement utility (not part of the method): streams `bytes` from `src`
+ * with 16-byte loads from `ctas` CTAs of 256 threads and XORs a checksum into
+ * *sink (device u64).  With host_resident = 1, `src` is page-locked host
+ * memory and the kernel measures the host link as the scan's loads use it;
+ * with 0, device memory (HBM read bandwidth).  Time it with CUDA events.
+ * Errors: EINVAL for null or misaligned pointers, bytes not a multiple of 16,
+ * or `src` not where host_resident says.
+ */
+int fathom_read_probe(const void* src, size_t bytes, int host_resident, uint64_t* sink, int ctas,
+                      fathom_stream_t stream);
 
 /* Static description of a status code. */
 const char* fathom_status_string(int status);

@@ -85,22 +85,28 @@ def sigma2_of_keys(K):
     return (s / max(n, 1)).astype(np.float32)
 
 
-def plant_needles(rng, K, q_head, kv_head=0, count=16, cosine=0.9):
-    """Overwrite `count` seeded key positions of `kv_head` with needles.
+def needle_positions(rng, n, count=16):
+    return np.sort(rng.choice(n, size=count, replace=False))
 
-    Needle = |k_orig| * (cosine * q_hat + sqrt(1 - cosine^2) * u_perp), with
-    u_perp a random unit vector orthogonal to q.  Returns the positions.
-    """
-    n = K.shape[1]
-    pos = np.sort(rng.choice(n, size=count, replace=False))
+
+def needle_rows(rng, rows, q_head, cosine=0.9):
+    """New key rows for needles: |k_orig| * (cosine * q_hat + sqrt(1 - cosine^2) * u_perp),
+    u_perp a random unit vector orthogonal to q.  rows: [count][d] originals."""
     qv = np.asarray(q_head, np.float64)
     q_hat = qv / np.linalg.norm(qv)
-    for p in pos:
-        k0 = K[kv_head, p].astype(np.float64)
+    out = np.empty(rows.shape, np.float32)
+    for e in range(rows.shape[0]):
         u = rng.standard_normal(qv.size)
         u -= u.dot(q_hat) * q_hat
         u /= np.linalg.norm(u)
-        K[kv_head, p] = (np.linalg.norm(k0) * (cosine * q_hat + np.sqrt(1 - cosine * cosine) * u)).astype(np.float32)
+        out[e] = np.linalg.norm(rows[e].astype(np.float64)) * (cosine * q_hat + np.sqrt(1 - cosine * cosine) * u)
+    return out
+
+
+def plant_needles(rng, K, q_head, kv_head=0, count=16, cosine=0.9):
+    """Overwrite `count` seeded key positions of `kv_head` with needles; returns the positions."""
+    pos = needle_positions(rng, K.shape[1], count)
+    K[kv_head, pos] = needle_rows(rng, K[kv_head, pos], q_head, cosine)
     return pos
 
 
@@ -151,4 +157,56 @@ def layer_inputs(config, layer=0, n=None, n_kv_heads=None, n_q_heads=None, d=Non
     if with_values:
         out["K_rows"] = f32_to_bf16_bits(K)
         out["V_rows"] = values_bf16(rng_for(config, layer, 4), Hkv, n, d)
+    return out
+
+
+def layer_inputs_cuda(config, layer=0, n=None, n_kv_heads=None, n_q_heads=None, d=None, device="cuda",
+                      with_values=True, needles=None):
+    """One layer of a workload generated on the GPU (torch's Philox generator,
+    seeded like the numpy path): same recipe, different draws.  Returns torch
+    tensors on `device`: K f32, K_rows/V_rows bf16 [Hkv][n][d], q (f32 or bf16)
+    [Hq][d], sigma2 f32 [Hkv][d]; plus numpy copies of q and sigma2 and the
+    needle positions."""
+    import torch
+    cfg = CONFIGS[config]
+    n = cfg.get("n", 4096) if n is None else n
+    Hkv = cfg["n_kv_heads"] if n_kv_heads is None else n_kv_heads
+    Hq = cfg["n_q_heads"] if n_q_heads is None else n_q_heads
+    d = cfg["d"] if d is None else d
+    sigma = channel_sigma(rng_for(config, layer, 0), Hkv, d)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(1000 * int(config) + int(layer))
+    K = torch.empty((Hkv, n, d), dtype=torch.float32, device=device)
+    sig_t = torch.from_numpy(sigma.astype(np.float32)).to(device)
+    for g in range(Hkv):
+        K[g].normal_(generator=gen)
+        K[g].mul_(sig_t[g][None, :])
+    q = queries(rng_for(config, layer, 2), Hq, d)
+    out = {}
+    if cfg["q_dtype"] == "bf16":
+        qb = f32_to_bf16_bits(q)
+        q = bf16_bits_to_f32(qb)
+        out["q_dev"] = torch.from_numpy(qb.view(np.int16)).to(device).view(torch.bfloat16)
+    else:
+        out["q_dev"] = torch.from_numpy(q).to(device)
+    out["q"] = q
+    nd = cfg.get("needles", 0) if needles is None else needles
+    if nd:
+        rng = rng_for(config, layer, 3)
+        pos = needle_positions(rng, n, nd)
+        rows = K[0, torch.from_numpy(pos).to(device)].cpu().numpy()
+        K[0, torch.from_numpy(pos).to(device)] = torch.from_numpy(needle_rows(rng, rows, q[0])).to(device)
+        out["needles"] = pos
+    s2 = torch.empty((Hkv, d), dtype=torch.float64, device=device)
+    for g in range(Hkv):
+        s2[g] = K[g].double().square().mean(dim=0)
+    out["sigma2_dev"] = s2.float()
+    out["sigma2"] = out["sigma2_dev"].cpu().numpy()
+    out["K"] = K
+    if with_values:
+        out["K_rows"] = K.to(torch.bfloat16)
+        V = torch.empty((Hkv, n, d), dtype=torch.bfloat16, device=device)
+        for g in range(Hkv):
+            V[g].normal_(generator=gen)
+        out["V_rows"] = V
     return out

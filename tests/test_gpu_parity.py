@@ -241,7 +241,7 @@ def test_six_key_example_on_gpu():
 @pytest.mark.parametrize("n,rows,k,kind", [
     (100, 3, 1, "normal"), (100, 3, 100, "normal"), (4096, 2, 64, "normal"), (20000, 4, 2048, "normal"),
     (131072, 2, 2048, "normal"), (200000, 2, 4096, "ties"), (50000, 2, 2048, "equal"),
-    (70000, 2, 1000, "narrow"), (9000, 1, 9000, "ties")])
+    (70000, 2, 1000, "narrow"), (4096, 1, 4096, "ties"), (9000, 1, 4096, "ties")])
 def test_topk_bit_exact(ref, n, rows, k, kind):
     rng = np.random.default_rng(n + k)
     if kind == "normal":
