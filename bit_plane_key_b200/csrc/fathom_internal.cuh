@@ -41,9 +41,11 @@ cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, co
 cudaError_t launch_probe(const void* src, size_t bytes, unsigned long long* sink, int ctas,
                          cudaStream_t stream);
 
-// fp32 <-> order-preserving u32: a > b as floats  <=>  key(a) > key(b).
+// fp32 <-> order-preserving u32: a > b as real numbers  <=>  key(a) > key(b),
+// and a == b  <=>  key(a) == key(b) (-0 and +0 share the key of +0).
 __device__ __forceinline__ uint32_t float_to_ordered(float f) {
     uint32_t u = __float_as_uint(f);
+    if (u == 0x80000000u) u = 0u;
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 __device__ __forceinline__ float ordered_to_float(uint32_t k) {
