@@ -14,9 +14,9 @@ constexpr int kMaxDevices = 64;
 unsigned int* g_status_ptr[kMaxDevices] = {};
 std::mutex g_status_mu;
 
-// Where a pointer lives.  Returns the device-usable address through `dev`.
-enum class Where { kDevice, kHostPinned, kOther };
+}  // namespace
 
+// Where a pointer lives.  Returns the device-usable address through `dev`.
 Where classify(const void* p, const void** dev) {
     cudaPointerAttributes a;
     cudaError_t e = cudaPointerGetAttributes(&a, p);
@@ -64,8 +64,6 @@ int resolve_store(const fathom_store* s, const uint32_t** planes, const uint16_t
     *scales = static_cast<const uint16_t*>(ds);
     return FATHOM_OK;
 }
-
-}  // namespace
 
 unsigned int* device_status_ptr() {
     int dev = 0;

@@ -22,6 +22,16 @@ inline int64_t n_pad_of(int64_t n) { return ((n + kPad - 1) / kPad) * kPad; }
 // to every kernel that can set a bit.
 unsigned int* device_status_ptr();
 
+// Host-side argument checks shared by the entry points (api.cu).
+enum class Where { kDevice, kHostPinned, kOther };
+Where classify(const void* p, const void** dev);
+bool is_device(const void* p);
+bool dims_ok(int Hkv, int d);
+bool heads_ok(int Hq, int Hkv);
+bool scan_fits(int d, int Hq, int Hkv);
+int to_status(cudaError_t e);
+int resolve_store(const fathom_store* s, const uint32_t** planes, const uint16_t** scales);
+
 // Host launchers (each enqueues on `stream`; arguments already validated).
 cudaError_t launch_pack(const void* K, int k_dtype, int Hkv, int64_t n, int d, uint32_t* planes,
                         uint16_t* scales, cudaStream_t stream);

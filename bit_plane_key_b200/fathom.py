@@ -63,6 +63,8 @@ _sig("fathom_sparse_attend", _I, [_P, _I, _P, _P, _I, _P, _I, _I, _L, _I, _I, _P
 _sig("fathom_last_device_status", _I, [_P])
 _sig("fathom_status_string", ctypes.c_char_p, [_I])
 _sig("fathom_read_probe", _I, [_P, _Z, _I, _P, _I, _P])
+_sig("fathom_noalloc_scratch_bytes", _Z, [])
+_sig("fathom_scan_topk_noalloc", _I, [_SP, _P, _I, _P, _I, _I, _P, _P, _P])
 
 
 def lib():
@@ -226,3 +228,14 @@ def read_probe(src, sink, ctas=None, stream=None):
         ctas = torch.cuda.get_device_properties(sink.device).multi_processor_count * 8
     _check(_lib.fathom_read_probe(_ptr(src), src.numel() * src.element_size(), int(host), _ptr(sink), int(ctas),
                                   _stream(stream)), "fathom_read_probe")
+
+
+def noalloc_scratch_bytes():
+    return int(_lib.fathom_noalloc_scratch_bytes())
+
+
+def scan_topk_noalloc(store, q, depths, k, idx, top_scores=None, stream=None):
+    """fathom_scan_topk on the library's fixed scratch array (no workspace; idx preallocated)."""
+    _check(_lib.fathom_scan_topk_noalloc(store.c, _ptr(q), _dtype_code(q), _ptr(depths), q.shape[0], int(k),
+                                         _ptr(idx), _ptr(top_scores), _stream(stream)), "fathom_scan_topk_noalloc")
+    return idx, top_scores

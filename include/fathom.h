@@ -185,6 +185,30 @@ int fathom_scan_topk(const fathom_store* store, const void* q, int q_dtype, cons
                      size_t workspace_bytes, fathom_stream_t stream);
 
 /*
+ * Scan + top-k without any caller-provided workspace.  The paper has no
+ * counterpart: this is a service to callers that cannot allocate device
+ * memory (an engine whose memory is all handed to its own pool, a plug-in
+ * inside a host program that forbids cudaMalloc/cudaFree on its serving
+ * path).  Same inputs, outputs and results as fathom_scan_topk; the scratch
+ * comes from one fixed array of fathom_noalloc_scratch_bytes() bytes (24 MiB)
+ * in the library's own device memory, which every GPU that loads the library
+ * holds until the process exits.  No call allocates or frees anything.
+ *   - A step needing more than that (fathom_scan_workspace_bytes(store, Hq, k)
+ *     above the maximum) returns FATHOM_ENOMEM before any work is enqueued.
+ *     Example that fits: Hq = 32, n = 131072, k = 2048 (about 20 MB).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and keeps it; make
+ *     that first call before any stream capture.
+ *   - Every call shares the array, which keeps the previous call's contents
+ *     (each call re-initialises what it needs).  Calls that overlap on the
+ *     GPU (different streams or host threads) race on it: serialise them.
+ * Other errors as fathom_scan_topk.
+ */
+size_t fathom_noalloc_scratch_bytes(void);
+int fathom_scan_topk_noalloc(const fathom_store* store, const void* q, int q_dtype, const uint8_t* depths,
+                             int n_q_heads, int k, int32_t* idx, float* top_scores, fathom_stream_t stream);
+
+/*
  * Exact attention over the selected keys only.  [ai-feeds summary 输出]
  * out[h] = softmax_j(q[h] . K[g][idx[h][j]] / sqrt(d)) V[g][idx[h][j]],
  * g = h / (Hq/Hkv), fp32 accumulation.
