@@ -52,6 +52,8 @@ def parse():
     p.add_argument("--n", type=int, default=1 << 20)
     p.add_argument("--no-extras", action="store_true", help="skip the HBM-resident and fixed-r comparison runs")
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    p.add_argument("--kernel", default=None, choices=["scan"],
+                   help="time one kernel alone on this workload (a kernel benchmark, not the step metric)")
     return p.parse_args()
 
 
@@ -317,10 +319,57 @@ def e2e_steps(torch, F, layer, budget, steps, warmup, flush):
     return total, h2d, d2h
 
 
+def kernel_bench(args):
+    """The scan kernel alone: store packed on the device (HBM) or copied to
+    page-locked memory (host), depths at budget B, scores of all 2^20 keys of
+    the 32 query heads; CUDA events around each launch, L2 flushed between.
+    Only the store, q, depths and scores stay allocated (a small footprint for
+    profilers)."""
+    import torch
+    import synth
+    from bit_plane_key_b200 import fathom as F
+    dev = torch.device("cuda", 0)
+    inp = synth.layer_inputs_cuda(CONFIG, n=args.n, device=dev, with_values=False)
+    st = F.pack_bitplanes(inp["K"])
+    torch.cuda.synchronize()
+    del inp["K"]
+    torch.cuda.empty_cache()
+    if args.resident == "host":
+        st = st.to_host()
+    dep = F.alloc_depths(inp["q_dev"], inp["sigma2_dev"], args.budget)
+    U = dep.view(8, 4, 128).amax(dim=1)
+    nbytes = st.plane_bytes_read(U)
+    scores = torch.empty((32, st.n_pad), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        F.scan_scores(st, inp["q_dev"], dep, out=scores)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        F.scan_scores(st, inp["q_dev"], dep, out=scores)
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ms = float(np.mean(ts))
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    peaks_file = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    hbm = float(json.load(open(peaks_file)).get("hbm_gbs", 6650.0)) if os.path.exists(peaks_file) else 6650.0
+    print(json.dumps({"kernel": "scan", "resident": args.resident, "n": args.n, "budget_bits": args.budget,
+                      "ms_mean": ms, "ms_min": float(np.min(ts)), "gkeys_per_s": args.n * 8 / (ms * 1e-3) / 1e9,
+                      "bytes_per_launch": nbytes, "gbs": gbs,
+                      "hbm_frac": gbs / hbm if args.resident == "hbm" else None}), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.kernel:
+        kernel_bench(args)
         return
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
