@@ -182,6 +182,83 @@ int fathom_scan_topk(const fathom_store* store, const void* q, int q_dtype, cons
     return to_status(e);
 }
 
+namespace {
+inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Checks a batch of stores and returns the bytes of all sessions' scores
+// (0 on an invalid batch).
+size_t batched_score_bytes(const fathom_store* stores, int S, int Hq) {
+    if (!stores || S < 1 || S > kMaxSets) return 0;
+    size_t total = 0;
+    for (int s = 0; s < S; ++s) {
+        const fathom_store& st = stores[s];
+        if (st.n < 1 || st.n_kv_heads != stores[0].n_kv_heads || st.d != stores[0].d) return 0;
+        total += a256(sizeof(float) * (size_t)Hq * (size_t)n_pad_of(st.n));
+    }
+    return total;
+}
+}  // namespace
+
+size_t fathom_scan_batched_workspace_bytes(const fathom_store* stores, int n_sessions, int n_q_heads, int k) {
+    if (n_q_heads < 1 || k < 1 || k > kMaxTopK) return 0;
+    const size_t sb = batched_score_bytes(stores, n_sessions, n_q_heads);
+    if (sb == 0) return 0;
+    int64_t max_n = 0;
+    for (int s = 0; s < n_sessions; ++s) max_n = stores[s].n > max_n ? stores[s].n : max_n;
+    return sb + topk_workspace_bytes(max_n, n_sessions * n_q_heads, k);
+}
+
+int fathom_scan_topk_batched(const fathom_store* stores, int n_sessions, const void* q, int q_dtype,
+                             const uint8_t* depths, int n_q_heads, int k, int32_t* idx, float* top_scores,
+                             void* workspace, size_t workspace_bytes, fathom_stream_t stream) {
+    if (!stores || n_sessions < 1 || n_sessions > kMaxSets || !q || !depths || !idx || !workspace)
+        return FATHOM_EINVAL;
+    if (q_dtype != FATHOM_F32 && q_dtype != FATHOM_BF16) return FATHOM_EINVAL;
+    if (k < 1 || k > kMaxTopK || !heads_ok(n_q_heads, stores[0].n_kv_heads)) return FATHOM_EINVAL;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return FATHOM_EINVAL;
+    const size_t need = fathom_scan_batched_workspace_bytes(stores, n_sessions, n_q_heads, k);
+    if (need == 0) return FATHOM_EINVAL;
+    if (workspace_bytes < need) return FATHOM_ENOMEM;
+    SessionMap sm;
+    RowMap rm;
+    sm.nsess = n_sessions;
+    rm.nsets = n_sessions;
+    rm.rows_per_set = n_q_heads;
+    rm.max_n = 0;
+    int tiles = 0;
+    size_t off = 0;
+    for (int s = 0; s < n_sessions; ++s) {
+        const fathom_store& st = stores[s];
+        if (k > st.n || st.n > INT32_MAX) return FATHOM_EINVAL;
+        int rc = resolve_store(&st, &sm.planes[s], &sm.scales[s]);
+        if (rc) return rc;
+        sm.n[s] = st.n;
+        sm.n_pad[s] = st.n_pad;
+        sm.score_base[s] = (int64_t)(off / sizeof(float));
+        sm.tile0[s] = tiles;
+        const int64_t t = (st.n_pad + 1023) / 1024;
+        if (t > INT32_MAX - tiles) return FATHOM_EINVAL;
+        tiles += (int)t;
+        rm.base[s] = sm.score_base[s];
+        rm.ld[s] = st.n_pad;
+        rm.n[s] = st.n;
+        rm.max_n = st.n > rm.max_n ? st.n : rm.max_n;
+        off += a256(sizeof(float) * (size_t)n_q_heads * (size_t)st.n_pad);
+    }
+    sm.tile0[n_sessions] = tiles;
+    if (!is_device(q) || !is_device(depths) || !is_device(idx) || !is_device(workspace) ||
+        (top_scores && !is_device(top_scores)))
+        return FATHOM_EINVAL;
+    if (!scan_fits(stores[0].d, n_q_heads, stores[0].n_kv_heads)) return FATHOM_EUNSUPPORTED;
+    if (!device_status_ptr()) return FATHOM_ECUDA;
+    float* scores = static_cast<float*>(workspace);
+    cudaStream_t cs = (cudaStream_t)stream;
+    cudaError_t e = launch_scan_batched(sm, stores[0].n_kv_heads, stores[0].d, q, q_dtype, depths, n_q_heads, scores, cs);
+    if (e != cudaSuccess) return FATHOM_ECUDA;
+    return to_status(launch_topk_map(scores, rm, n_sessions * n_q_heads, k, idx, top_scores,
+                                     static_cast<char*>(workspace) + off, cs));
+}
+
 int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
                          int rows_host_resident, const int32_t* idx, int n_q_heads, int n_kv_heads, int64_t n,
                          int d, int k, float* out, fathom_stream_t stream) {

@@ -42,8 +42,37 @@ cudaError_t launch_scan(const uint32_t* planes, const uint16_t* scales, int Hkv,
                         int64_t n_pad, const void* q, int q_dtype, const uint8_t* depths, int Hq,
                         float* scores, cudaStream_t stream);
 size_t topk_workspace_bytes(int64_t n, int rows, int k);
+
+// Where the score rows are: rows are grouped in sets of `rows_per_set`
+// (the query heads of one session); row r of set s starts at
+// base[s] + (r % rows_per_set) * ld[s] and has n[s] valid scores.
+constexpr int kMaxSets = 64;
+struct RowMap {
+    int rows_per_set;
+    int nsets;
+    int64_t max_n;
+    int64_t base[kMaxSets];
+    int64_t ld[kMaxSets];
+    int64_t n[kMaxSets];
+};
 cudaError_t launch_topk(const float* scores, int64_t n, int64_t ld, int rows, int k, int32_t* idx,
                         float* top_scores, void* ws, cudaStream_t stream);
+cudaError_t launch_topk_map(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
+                            float* top_scores, void* ws, cudaStream_t stream);
+
+// Sessions of a batched scan: session s owns tiles [tile0[s], tile0[s+1]) of
+// the flattened grid and writes scores [Hq][n_pad[s]] at score_base[s].
+struct SessionMap {
+    int nsess;
+    const uint32_t* planes[kMaxSets];
+    const uint16_t* scales[kMaxSets];
+    int64_t n[kMaxSets];
+    int64_t n_pad[kMaxSets];
+    int64_t score_base[kMaxSets];
+    int tile0[kMaxSets + 1];
+};
+cudaError_t launch_scan_batched(const SessionMap& map, int Hkv, int d, const void* q, int q_dtype,
+                                const uint8_t* depths, int Hq, float* scores, cudaStream_t stream);
 cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
                           const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k, float* out,
                           cudaStream_t stream);

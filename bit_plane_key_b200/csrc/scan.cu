@@ -47,10 +47,7 @@ constexpr int kThreads = 128;                // (16 blocks) x (8 variants)
 constexpr int kChunk = 16;                   // active channels per stage
 constexpr int kCPad = 20;                    // words per (word, variant) code row; 20 = 4 mod 8
 constexpr uint32_t kHalfExp = 0x3F000000u;   // bits of 0.5f: exponent byte of F
-#ifndef FATHOM_SCAN_PACKED
-#define FATHOM_SCAN_PACKED 1
-#endif
-constexpr bool kScanPacked = FATHOM_SCAN_PACKED;   // fp32x2 FMAs (two keys per instruction)
+constexpr bool kScanPacked = true;           // fp32x2 FMAs: two keys of a block per instruction
 
 struct ScanSmem {
     static size_t bytes(int d, int G) {
@@ -93,14 +90,16 @@ __device__ __forceinline__ uint32_t code_variant(const uint32_t* p, int sv) {
     return x;
 }
 
+// One (tile of 1024 keys, KV head g) of one store; q, depths and scores are
+// the store's own [Hq][d], [Hq][d] and [Hq][n_pad] arrays.
 template <int G, bool kPacked>
-__global__ void __launch_bounds__(kThreads)
-scan_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ scales, int d, int64_t n,
-            int64_t n_pad, const void* __restrict__ q, int q_dtype, const uint8_t* __restrict__ depths,
-            float* __restrict__ scores, unsigned int* status) {
+__device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ scales,
+                                          int d, int64_t n, int64_t n_pad, int tile, int g,
+                                          const void* __restrict__ q, int q_dtype,
+                                          const uint8_t* __restrict__ depths, float* __restrict__ scores,
+                                          unsigned int* status) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int g = blockIdx.y;
-    const int64_t tile0 = (int64_t)blockIdx.x * kTileKeys;
+    const int64_t tile0 = (int64_t)tile * kTileKeys;
     const int64_t words_total = n_pad / 32;
     const int64_t nblk_total = n_pad / kBlock;
     const int64_t wrem = words_total - tile0 / 32;
@@ -343,16 +342,59 @@ scan_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ sc
 }
 
 template <int G>
+__global__ void __launch_bounds__(kThreads)
+scan_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ scales, int d, int64_t n,
+            int64_t n_pad, const void* __restrict__ q, int q_dtype, const uint8_t* __restrict__ depths,
+            float* __restrict__ scores, unsigned int* status) {
+    scan_tile<G, kScanPacked>(planes, scales, d, n, n_pad, (int)blockIdx.x, (int)blockIdx.y, q, q_dtype, depths,
+                              scores, status);
+}
+
+// Batched sessions: blockIdx.x runs over the tiles of all sessions.
+template <int G>
+__global__ void __launch_bounds__(kThreads)
+scan_batched_kernel(const __grid_constant__ SessionMap map, int d, int Hq, const void* __restrict__ q, int q_dtype,
+                    const uint8_t* __restrict__ depths, float* __restrict__ scores, unsigned int* status) {
+    const int t = (int)blockIdx.x;
+    int lo = 0, hi = map.nsess - 1;   // last session with tile0 <= t
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (map.tile0[mid] <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    const int sidx = lo;
+    const size_t qstride = (size_t)Hq * d;
+    const void* qs = (q_dtype == FATHOM_BF16)
+                         ? static_cast<const void*>(static_cast<const uint16_t*>(q) + sidx * qstride)
+                         : static_cast<const void*>(static_cast<const float*>(q) + sidx * qstride);
+    scan_tile<G, kScanPacked>(map.planes[sidx], map.scales[sidx], d, map.n[sidx], map.n_pad[sidx],
+                              t - map.tile0[sidx], (int)blockIdx.y, qs, q_dtype, depths + sidx * qstride,
+                              scores + map.score_base[sidx], status);
+}
+
+template <int G>
 cudaError_t launch_scan_g(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n,
                           int64_t n_pad, const void* q, int q_dtype, const uint8_t* depths, float* scores,
                           cudaStream_t stream) {
     size_t smem = ScanSmem::bytes(d, G);
-    auto kern = scan_kernel<G, kScanPacked>;
+    auto kern = scan_kernel<G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((n_pad + kTileKeys - 1) / kTileKeys), (unsigned)Hkv);
     kern<<<grid, kThreads, smem, stream>>>(planes, scales, d, n, n_pad, q, q_dtype, depths, scores,
                                            device_status_ptr());
+    return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t launch_scan_batched_g(const SessionMap& map, int Hkv, int d, const void* q, int q_dtype,
+                                  const uint8_t* depths, int Hq, float* scores, cudaStream_t stream) {
+    size_t smem = ScanSmem::bytes(d, G);
+    auto kern = scan_batched_kernel<G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)map.tile0[map.nsess], (unsigned)Hkv);
+    kern<<<grid, kThreads, smem, stream>>>(map, d, Hq, q, q_dtype, depths, scores, device_status_ptr());
     return cudaGetLastError();
 }
 
@@ -368,6 +410,17 @@ cudaError_t launch_scan(const uint32_t* planes, const uint16_t* scales, int Hkv,
         case 2: return launch_scan_g<2>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, stream);
         case 4: return launch_scan_g<4>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, stream);
         case 8: return launch_scan_g<8>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_scan_batched(const SessionMap& map, int Hkv, int d, const void* q, int q_dtype,
+                                const uint8_t* depths, int Hq, float* scores, cudaStream_t stream) {
+    switch (Hq / Hkv) {
+        case 1: return launch_scan_batched_g<1>(map, Hkv, d, q, q_dtype, depths, Hq, scores, stream);
+        case 2: return launch_scan_batched_g<2>(map, Hkv, d, q, q_dtype, depths, Hq, scores, stream);
+        case 4: return launch_scan_batched_g<4>(map, Hkv, d, q, q_dtype, depths, Hq, scores, stream);
+        case 8: return launch_scan_batched_g<8>(map, Hkv, d, q, q_dtype, depths, Hq, scores, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -66,12 +66,20 @@ Workspace carve(void* ws, int rows, int k) {
     return w;
 }
 
+__device__ __forceinline__ void row_span(const RowMap& m, int row, int64_t* off, int64_t* n) {
+    const int set = row / m.rows_per_set;
+    *off = m.base[set] + (int64_t)(row - set * m.rows_per_set) * m.ld[set];
+    *n = m.n[set];
+}
+
 __device__ __forceinline__ uint64_t composite(uint32_t key, int64_t i) {
     return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)i);
 }
 
-__global__ void topk_init(Workspace w, int64_t n, int rows) {
+__global__ void topk_init(Workspace w, const __grid_constant__ RowMap m, int rows) {
     const int row = blockIdx.x;
+    int64_t off, n;
+    row_span(m, row, &off, &n);
     uint32_t* h = w.hist + (size_t)row * kBins;
     for (int b = threadIdx.x; b < kBins; b += blockDim.x) {
         h[b] = 0;
@@ -93,18 +101,21 @@ __global__ void topk_init(Workspace w, int64_t n, int rows) {
 }
 
 __global__ void __launch_bounds__(kPassThreads)
-topk_hist(const float* __restrict__ scores, int64_t n, int64_t ld, int rows, Workspace w, int level) {
+topk_hist(const float* __restrict__ scores, const __grid_constant__ RowMap m, int rows, Workspace w, int level) {
     __shared__ uint32_t h[kBins];
     const int row = blockIdx.y;
     const RowState st = w.state[row];
     if (st.phase != 0) return;
+    int64_t off, n;
+    row_span(m, row, &off, &n);
+    if ((int64_t)blockIdx.x * kChunk >= n) return;
     for (int b = threadIdx.x; b < kBins; b += kPassThreads) h[b] = 0;
     __syncthreads();
     const int sh = kLevelShift[level];
     const uint32_t mask = (1u << kLevelBits[level]) - 1u;
     const int64_t i0 = (int64_t)blockIdx.x * kChunk;
     const int64_t i1 = min(n, i0 + kChunk);
-    const float* s = scores + (int64_t)row * ld;
+    const float* s = scores + off;
     for (int64_t i = i0 + threadIdx.x; i < i1; i += kPassThreads) {
         uint32_t key = float_to_ordered(s[i]);
         bool in = (st.shift == 32) || ((key >> st.shift) == st.prefix);
@@ -171,13 +182,16 @@ topk_select(Workspace w, int rows, int k, int level) {
 }
 
 __global__ void __launch_bounds__(kPassThreads)
-topk_compact(const float* __restrict__ scores, int64_t n, int64_t ld, int k, Workspace w,
+topk_compact(const float* __restrict__ scores, const __grid_constant__ RowMap m, int k, Workspace w,
              unsigned int* status) {
     const int row = blockIdx.y;
     const RowState st = w.state[row];
+    int64_t off, n;
+    row_span(m, row, &off, &n);
     const int64_t i0 = (int64_t)blockIdx.x * kChunk;
+    if (i0 >= n) return;
     const int64_t i1 = min(n, i0 + kChunk);
-    const float* s = scores + (int64_t)row * ld;
+    const float* s = scores + off;
     const int lane = threadIdx.x & 31;
     RowState* gst = w.state + row;
     for (int64_t base = i0; base < i1; base += kPassThreads) {
@@ -237,13 +251,15 @@ __device__ void bitonic_desc(uint64_t* buf, int S) {
 }
 
 __global__ void __launch_bounds__(kFinishThreads)
-topk_finish(const float* __restrict__ scores, int64_t n, int64_t ld, int k, Workspace w, int32_t* __restrict__ idx,
-            float* __restrict__ top_scores, unsigned int* status) {
+topk_finish(const float* __restrict__ scores, const __grid_constant__ RowMap m, int k, Workspace w,
+            int32_t* __restrict__ idx, float* __restrict__ top_scores, unsigned int* status) {
     extern __shared__ uint64_t buf[];
     __shared__ int warp_cnt[32];
     __shared__ int s_got;
     const int row = blockIdx.x;
     const RowState st = w.state[row];
+    int64_t off, n;
+    row_span(m, row, &off, &n);
     const int ns = min(st.count_above, k);
     int total;
     if (st.phase == 1) {
@@ -259,7 +275,7 @@ topk_finish(const float* __restrict__ scores, int64_t n, int64_t ld, int k, Work
         for (int e = threadIdx.x; e < ns; e += blockDim.x) buf[e] = w.sure[(size_t)row * k + e];
         if (threadIdx.x == 0) s_got = 0;
         __syncthreads();
-        const float* s = scores + (int64_t)row * ld;
+        const float* s = scores + off;
         const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
         for (int64_t base = 0; base < n; base += blockDim.x) {
             int got = s_got;
@@ -303,22 +319,34 @@ size_t topk_workspace_bytes(int64_t n, int rows, int k) {
            align256(sizeof(uint64_t) * (size_t)rows * k) + align256(sizeof(uint64_t) * (size_t)rows * kCap);
 }
 
-cudaError_t launch_topk(const float* scores, int64_t n, int64_t ld, int rows, int k, int32_t* idx,
-                        float* top_scores, void* ws, cudaStream_t stream) {
+cudaError_t launch_topk_map(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
+                            float* top_scores, void* ws, cudaStream_t stream) {
     Workspace w = carve(ws, rows, k);
     unsigned int* status = device_status_ptr();
-    const unsigned chunks = (unsigned)((n + kChunk - 1) / kChunk);
-    topk_init<<<rows, 256, 0, stream>>>(w, n, rows);
+    const unsigned chunks = (unsigned)((map.max_n + kChunk - 1) / kChunk);
+    topk_init<<<rows, 256, 0, stream>>>(w, map, rows);
     for (int level = 0; level < 3; ++level) {
-        topk_hist<<<dim3(chunks, rows), kPassThreads, 0, stream>>>(scores, n, ld, rows, w, level);
+        topk_hist<<<dim3(chunks, rows), kPassThreads, 0, stream>>>(scores, map, rows, w, level);
         topk_select<<<rows, 1024, 0, stream>>>(w, rows, k, level);
     }
-    topk_compact<<<dim3(chunks, rows), kPassThreads, 0, stream>>>(scores, n, ld, k, w, status);
+    topk_compact<<<dim3(chunks, rows), kPassThreads, 0, stream>>>(scores, map, k, w, status);
     const size_t smem = sizeof(uint64_t) * kSortMax;
     cudaError_t e = cudaFuncSetAttribute(topk_finish, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    topk_finish<<<rows, kFinishThreads, smem, stream>>>(scores, n, ld, k, w, idx, top_scores, status);
+    topk_finish<<<rows, kFinishThreads, smem, stream>>>(scores, map, k, w, idx, top_scores, status);
     return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const float* scores, int64_t n, int64_t ld, int rows, int k, int32_t* idx,
+                        float* top_scores, void* ws, cudaStream_t stream) {
+    RowMap m;
+    m.rows_per_set = rows;
+    m.nsets = 1;
+    m.max_n = n;
+    m.base[0] = 0;
+    m.ld[0] = ld;
+    m.n[0] = n;
+    return launch_topk_map(scores, m, rows, k, idx, top_scores, ws, stream);
 }
 
 }  // namespace fathom

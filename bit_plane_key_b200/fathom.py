@@ -64,6 +64,8 @@ _sig("fathom_last_device_status", _I, [_P])
 _sig("fathom_status_string", ctypes.c_char_p, [_I])
 _sig("fathom_read_probe", _I, [_P, _Z, _I, _P, _I, _P])
 _sig("fathom_noalloc_scratch_bytes", _Z, [])
+_sig("fathom_scan_batched_workspace_bytes", _Z, [_SP, _I, _I, _I])
+_sig("fathom_scan_topk_batched", _I, [_SP, _I, _P, _I, _P, _I, _I, _P, _P, _P, _Z, _P])
 _sig("fathom_scan_topk_noalloc", _I, [_SP, _P, _I, _P, _I, _I, _P, _P, _P])
 
 
@@ -193,6 +195,35 @@ def scan_topk(store, q, depths, k, idx=None, top_scores=None, workspace=None, st
     _check(_lib.fathom_scan_topk(store.c, _ptr(q), _dtype_code(q), _ptr(depths), Hq, int(k), _ptr(idx),
                                  _ptr(top_scores), _ptr(workspace), workspace.numel(), _stream(stream)),
            "fathom_scan_topk")
+    return idx, top_scores
+
+
+def _store_array(stores):
+    arr = (fathom_store * len(stores))()
+    for i, st in enumerate(stores):
+        arr[i] = st._c
+    return arr
+
+
+def scan_batched_workspace_bytes(stores, n_q_heads, k):
+    arr = _store_array(stores)
+    return int(_lib.fathom_scan_batched_workspace_bytes(arr, len(stores), int(n_q_heads), int(k)))
+
+
+def scan_topk_batched(stores, q, depths, k, idx=None, top_scores=None, workspace=None, stream=None):
+    """Sessions `stores` (list of Store), q [S][Hq][d], depths [S][Hq][d] -> idx, top scores [S][Hq][k]."""
+    S, Hq = q.shape[0], q.shape[1]
+    arr = _store_array(stores)
+    if idx is None:
+        idx = torch.empty((S, Hq, k), dtype=torch.int32, device=q.device)
+    if top_scores is None:
+        top_scores = torch.empty((S, Hq, k), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nb = int(_lib.fathom_scan_batched_workspace_bytes(arr, S, Hq, int(k)))
+        workspace = torch.empty(max(nb, 1), dtype=torch.uint8, device=q.device)
+    _check(_lib.fathom_scan_topk_batched(arr, S, _ptr(q), _dtype_code(q), _ptr(depths), Hq, int(k), _ptr(idx),
+                                         _ptr(top_scores), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "fathom_scan_topk_batched")
     return idx, top_scores
 
 

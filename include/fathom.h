@@ -185,6 +185,28 @@ int fathom_scan_topk(const fathom_store* store, const void* q, int q_dtype, cons
                      size_t workspace_bytes, fathom_stream_t stream);
 
 /*
+ * Scan + top-k of several sessions in one pass (many sessions resident at
+ * once; arXiv abstract).  Session s has its own store stores[s] (all with
+ * the same Hkv and d, each device- or host-resident, lengths may differ) and
+ * its own queries; one launch scans the tiles of every session, then one
+ * top-k pass serves all S x Hq rows.  Results equal S separate
+ * fathom_scan_topk calls.
+ *   stores      host array of n_sessions (1..64) store descriptors.
+ *   q           device, [S][Hq][d], FATHOM_F32 or FATHOM_BF16.
+ *   depths      device, u8 [S][Hq][d] (fathom_alloc_depths with S*Hq query heads
+ *               and S*Hkv KV heads fills it in one call).
+ *   idx         device, i32 [S][Hq][k];  top_scores f32 [S][Hq][k] or NULL.
+ *   workspace   device, fathom_scan_batched_workspace_bytes() bytes, 256-byte aligned;
+ *               session s's scores start at the s-th 256-byte-aligned slice.
+ * Errors: EINVAL for bad sessions (count, mismatched Hkv/d, k > some n,
+ * residency), ENOMEM for a short workspace.
+ */
+size_t fathom_scan_batched_workspace_bytes(const fathom_store* stores, int n_sessions, int n_q_heads, int k);
+int fathom_scan_topk_batched(const fathom_store* stores, int n_sessions, const void* q, int q_dtype,
+                             const uint8_t* depths, int n_q_heads, int k, int32_t* idx, float* top_scores,
+                             void* workspace, size_t workspace_bytes, fathom_stream_t stream);
+
+/*
  * Scan + top-k without any caller-provided workspace.  The paper has no
  * counterpart: this is a service to callers that cannot allocate device
  * memory (an engine whose memory is all handed to its own pool, a plug-in

@@ -382,3 +382,46 @@ def test_sparse_attend_bad_index_flagged(ref):
     ok = np.delete(idx[1], 3)[None]
     want1 = ref.attend(inp["q"][1:2], inp["K_rows"], inp["V_rows"], ok)
     assert np.linalg.norm(out[1] - want1[0]) <= 1e-3 * np.linalg.norm(want1[0])
+
+
+# --------------------------------------------------------------------------
+# batched sessions (ragged lengths, per-session sigma, mixed residency)
+# --------------------------------------------------------------------------
+def test_scan_topk_batched_matches_single_sessions(ref):
+    lengths = [3000, 777, 12345, 1024, 5000]
+    Hkv, Hq, B, k = 2, 8, 68, 128
+    stores, qs, s2s, inps = [], [], [], []
+    for sidx, n in enumerate(lengths):
+        inp = make(4, n=n, Hkv=Hkv, Hq=Hq, layer=sidx)
+        st = F.pack_bitplanes(dev(inp["K"]))
+        stores.append(st.to_host() if sidx % 2 else st)
+        qs.append(inp["q_bf16"])
+        s2s.append(inp["sigma2"])
+        inps.append(inp)
+    q = bf16(np.stack(qs))                                   # [S][Hq][d]
+    s2 = dev(np.concatenate(s2s))                            # [S*Hkv][d]
+    dep = F.alloc_depths(q.view(-1, 128), s2, B).view(len(lengths), Hq, 128)
+    idx, top = F.scan_topk_batched(stores, q, dep, k)
+    idx, top = host(idx), host(top)
+    for sidx, n in enumerate(lengths):
+        i1, t1 = F.scan_topk(stores[sidx], q[sidx], dep[sidx], k)
+        assert np.array_equal(idx[sidx], host(i1)), sidx
+        assert np.array_equal(top[sidx], host(t1)), sidx
+        planes, scales = ref.pack(inps[sidx]["K"])
+        d_h = host(dep[sidx])
+        assert np.array_equal(d_h, ref.alloc_depths(inps[sidx]["q"], inps[sidx]["sigma2"], B))
+        s_ref, a_ref = ref.scores(planes, scales, n, inps[sidx]["q"], d_h, with_abs=True)
+        for h in range(Hq):
+            topk_sets_agree(ref, s_ref[h], a_ref[h], idx[sidx, h], k)
+    assert F.last_device_status() == 0
+
+
+def test_scan_topk_batched_rejects_bad_batches():
+    a = F.pack_bitplanes(dev(make(4, n=500, Hkv=2, Hq=8)["K"]))
+    b = F.pack_bitplanes(dev(make(4, n=600, Hkv=1, Hq=4)["K"]))
+    q = torch.zeros((2, 8, 128), dtype=torch.bfloat16, device=DEV)
+    dep = torch.zeros((2, 8, 128), dtype=torch.uint8, device=DEV)
+    with pytest.raises(F.FathomError):          # mismatched KV heads
+        F.scan_topk_batched([a, b], q, dep, 16)
+    with pytest.raises(F.FathomError):          # k above a session's length
+        F.scan_topk_batched([a, a], q, dep, 501)
