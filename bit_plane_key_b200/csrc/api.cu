@@ -276,7 +276,8 @@ int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, con
     if (!is_device(q) || !is_device(idx) || !is_device(out)) return FATHOM_EINVAL;
     if (!device_status_ptr()) return FATHOM_ECUDA;
     return to_status(launch_attend(q, q_dtype, static_cast<const uint16_t*>(kd), static_cast<const uint16_t*>(vd),
-                                   idx, n_q_heads, n_kv_heads, n, d, k, out, (cudaStream_t)stream));
+                                   idx, n_q_heads, n_kv_heads, n, d, k, rows_host_resident, out,
+                                   (cudaStream_t)stream));
 }
 
 int fathom_last_device_status(fathom_stream_t stream) {

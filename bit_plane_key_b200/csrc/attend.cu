@@ -6,12 +6,16 @@
 // g = h / (Hq/Hkv), K and V rows in bf16, fp32 accumulation, exp via exp2f.
 //
 // One thread-block cluster of kSplit CTAs per query head.  CTA r of the
-// cluster takes rows j = r, r + kSplit, ... of the head's k selected keys;
-// inside it each warp runs an online softmax over its rows (lane l holds
-// channels [l*d/32, (l+1)*d/32)).  The warps' partial (max, sum, o) merge in
-// shared memory, then CTA 0 merges the kSplit CTA partials through
-// distributed shared memory and writes o_h.  No workspace and no second
-// kernel.  Rows may live in device memory or in page-locked host memory.
+// cluster takes every kSplit-th of the head's k selected keys; inside it each
+// warp runs an online softmax over its rows (lane l holds channels
+// [l*d/32, (l+1)*d/32)).  The warps' partial (max, sum, o) merge in shared
+// memory, then CTA 0 merges the kSplit CTA partials through distributed
+// shared memory and writes o_h.  No workspace and no second kernel.
+// Rows may live in device memory or in page-locked host memory.  Over the
+// host link, gathering rows in address order is about twice as fast as in
+// score order, so for host-resident rows every CTA first sorts the head's
+// indices in shared memory; the head's 32 warps then sweep the sorted list
+// together (the softmax sum does not depend on the order).
 #include <cooperative_groups.h>
 
 #include "fathom_internal.cuh"
@@ -25,6 +29,7 @@ constexpr int kSplit = 8;      // CTAs per head (cluster size)
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kUnroll = 4;     // rows in flight per warp
+constexpr int kSortCap = kMaxTopK;   // indices sorted in shared memory
 
 
 template <int V>
@@ -58,8 +63,9 @@ template <int V>
 __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kThreads)
 attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restrict__ Kr,
               const uint16_t* __restrict__ Vr, const int32_t* __restrict__ idx, int Hq, int Hkv, int64_t n,
-              int k, float* __restrict__ out, unsigned int* status) {
+              int k, int sort_rows, float* __restrict__ out, unsigned int* status) {
     constexpr int d = V * 32;
+    __shared__ int32_t s_idx[kSortCap];
     __shared__ float s_m[kWarps], s_l[kWarps];
     __shared__ float s_o[kWarps][d];
     __shared__ float c_m, c_l;        // this CTA's merged partial (read by CTA 0)
@@ -82,17 +88,40 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
 
     const int32_t* ih = idx + (int64_t)h * k;
     const int64_t head_base = (int64_t)g * n * d;
-    // rows of this warp: j = r + kSplit * (wp + kWarps * s)
+    if (sort_rows) {
+        // bitonic sort (ascending) of the head's indices, padded to a power of two
+        int P = 1;
+        while (P < k) P <<= 1;
+        for (int e = threadIdx.x; e < P; e += kThreads) s_idx[e] = (e < k) ? ih[e] : INT32_MAX;
+        __syncthreads();
+        for (int size = 2; size <= P; size <<= 1) {
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                for (int t = threadIdx.x; t < P / 2; t += kThreads) {
+                    const int i = 2 * t - (t & (stride - 1)), j = i + stride;
+                    const bool up = (i & size) == 0;
+                    const int32_t a = s_idx[i], b2 = s_idx[j];
+                    if ((a > b2) == up) {
+                        s_idx[i] = b2;
+                        s_idx[j] = a;
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        ih = s_idx;
+    }
+    // rows of this warp: positions p = r + kSplit * (wp + kWarps * m) of the (sorted) list,
+    // so the head's 32 warps sweep the list together, in address order when sorted
     const int stride = kSplit * kWarps;
-    for (int j0 = r + kSplit * wp; j0 < k; j0 += stride * kUnroll) {
+    for (int p0 = r + kSplit * wp; p0 < k; p0 += stride * kUnroll) {
         float kv[kUnroll][V], vv[kUnroll][V];
         bool ok[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            int j = j0 + u * stride;
+            const int p = p0 + u * stride;
             ok[u] = false;
-            if (j < k) {
-                int64_t i = ih[j];
+            if (p < k) {
+                const int64_t i = ih[p];
                 if (i >= 0 && i < n) {
                     ok[u] = true;
                     const int64_t off = head_base + i * d + lane * V;
@@ -173,15 +202,16 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
 }  // namespace
 
 cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
-                          const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k, float* out,
+                          const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k, int sort_rows, float* out,
                           cudaStream_t stream) {
     dim3 grid((unsigned)(Hq * kSplit));
     unsigned int* st = device_status_ptr();
+    const int sr = (sort_rows && k <= kSortCap) ? 1 : 0;
     switch (d) {
-        case 32: attend_kernel<1><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, out, st); break;
-        case 64: attend_kernel<2><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, out, st); break;
-        case 128: attend_kernel<4><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, out, st); break;
-        case 256: attend_kernel<8><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, out, st); break;
+        case 32: attend_kernel<1><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, sr, out, st); break;
+        case 64: attend_kernel<2><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, sr, out, st); break;
+        case 128: attend_kernel<4><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, sr, out, st); break;
+        case 256: attend_kernel<8><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, sr, out, st); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
