@@ -316,18 +316,24 @@ def test_scan_topk_consistent_with_own_scores(ref):
 # a3: host-resident store gives the same scan
 # --------------------------------------------------------------------------
 def test_host_resident_store(ref):
-    inp = make(2, n=7000, Hkv=2, Hq=8)
-    st = F.pack_bitplanes(dev(inp["K"]))
-    hst = st.to_host()
-    dep = F.alloc_depths(q_dev(inp), dev(inp["sigma2"]), 92)
-    s_dev = host(F.scan_scores(st, q_dev(inp), dep))
-    s_host = host(F.scan_scores(hst, q_dev(inp), dep))
-    assert np.array_equal(s_dev, s_host)
-    i_dev, _ = F.scan_topk(st, q_dev(inp), dep, 700)
-    i_host, _ = F.scan_topk(hst, q_dev(inp), dep, 700)
-    assert np.array_equal(host(i_dev), host(i_host))
-    planes, scales = ref.pack(inp["K"])
-    check_scores(ref, planes, scales, 7000, inp["q"], host(dep), s_host)
+    """Host-resident and device-resident stores give the same scan, both
+    within the score tolerance of the oracle."""
+    for Hq in (8, 4):   # GQA groups of 4 and of 2
+        inp = make(2, n=7000, Hkv=2, Hq=Hq)
+        st = F.pack_bitplanes(dev(inp["K"]))
+        hst = st.to_host()
+        dep = F.alloc_depths(q_dev(inp), dev(inp["sigma2"]), 92)
+        s_dev = host(F.scan_scores(st, q_dev(inp), dep))
+        s_host = host(F.scan_scores(hst, q_dev(inp), dep))
+        planes, scales = ref.pack(inp["K"])
+        s_ref, a_ref = check_scores(ref, planes, scales, 7000, inp["q"], host(dep), s_host)
+        check_scores(ref, planes, scales, 7000, inp["q"], host(dep), s_dev)
+        assert np.array_equal(s_dev, s_host)
+        i_dev, _ = F.scan_topk(st, q_dev(inp), dep, 700)
+        i_host, _ = F.scan_topk(hst, q_dev(inp), dep, 700)
+        for h in range(Hq):
+            topk_sets_agree(ref, s_ref[h], a_ref[h], host(i_dev)[h], 700)
+            topk_sets_agree(ref, s_ref[h], a_ref[h], host(i_host)[h], 700)
 
 
 def test_residency_mismatch_rejected():
@@ -413,6 +419,9 @@ def test_scan_topk_batched_matches_single_sessions(ref):
         s_ref, a_ref = ref.scores(planes, scales, n, inps[sidx]["q"], d_h, with_abs=True)
         for h in range(Hq):
             topk_sets_agree(ref, s_ref[h], a_ref[h], idx[sidx, h], k)
+            topk_sets_agree(ref, s_ref[h], a_ref[h], host(i1)[h], k)
+            sel = idx[sidx, h]
+            assert np.all(np.abs(top[sidx, h] - s_ref[h][sel]) <= SCORE_RTOL * a_ref[h][sel])
     assert F.last_device_status() == 0
 
 
