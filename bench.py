@@ -372,37 +372,21 @@ def main():
         kernel_bench(args)
         return
     import torch
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+    from bit_plane_key_b200.ranks import Ranks, layer_of_rank, throughput
     local = int(os.environ.get("LOCAL_RANK", "0"))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+    ranks = Ranks("nccl", device=dev, sync=torch.cuda.synchronize)
+    world, rank = ranks.world, ranks.rank
     from bit_plane_key_b200 import fathom as F
-
-    def barrier():
-        if dist:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    def max_over_ranks(x):
-        if not dist:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     peaks_file = os.path.join(ROOT, "MEASURED_PEAKS.json")
     peaks = json.load(open(peaks_file)) if os.path.exists(peaks_file) else {}
     hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
     link = link_peak(F, torch, dev)
 
-    layer = Layer(F, torch, args, layer=rank, resident=args.resident, dev=dev)
+    layer = Layer(F, torch, args, layer=layer_of_rank(rank), resident=args.resident, dev=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     gpu_index = torch.cuda.current_device()
     visible = os.environ.get("CUDA_VISIBLE_DEVICES")
@@ -415,9 +399,8 @@ def main():
                       clocks_gpu=gpu_index if rank == 0 else None)
     barrier()
     total_ms = max_over_ranks(float(res["step_ms"].sum()))
-    ms_per_step = total_ms / args.steps
+    value, ms_per_step = throughput(args.n * layer.Hkv, world, total_ms, args.steps)
     keys_per_step = args.n * layer.Hkv * world
-    value = keys_per_step / (ms_per_step * 1e-3) / 1e9
 
     # roofline of the scan: algorithmic bytes (union planes + their scales) per launch / mean launch time
     scan_bytes, U = layer.union_bytes()
@@ -497,9 +480,7 @@ def main():
                 "gpu_launches": Layer.LAUNCHES_PER_STEP * args.steps,
                 "needle_recall_head0": recall, "cpu_baseline": cpu, "compare": extras}
         print(json.dumps(line), flush=True)
-    if dist:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
 
 
 if __name__ == "__main__":

@@ -15,24 +15,27 @@
 // in place).  With F_t = 1/2 (1 + P_t/16), an fp32 number whose mantissa bits
 // 22..19 are exactly P_t,
 //   v_t = 2^(3-t)(2m + 1) - 8 = 32 F_t - 24 + 2^(3-t),
-// so a channel adds (32 q Delta) F_t per key and head, and q Delta (2^(3-t) - 24)
-// per (block, head) once.
+// so a (channel, head) pair adds (32 q Delta) F_t per key, and
+// Delta q (2^(3-t) - 24) per (block, head) once.
 //
-// Work.  One CTA of 128 threads per (tile of 1024 keys, KV head).  The tile's
-// active channels are streamed in chunks of 16:
-//   stage: thread (channel group of 4, plane word w) loads the U_c plane
-//     words of its channels and transposes them to byte codes: variant word
-//     s (s = 0..7) holds the codes of keys s, s+8, s+16, s+24 of the word,
-//     one byte each, bits 6..3 = planes 0..3 (rotate + mask per plane and
-//     variant, i.e. half an operation per plane bit), stored to a double
-//     buffer in shared memory with conflict-free 16-byte stores;
-//   compute: thread (block b, variant s) owns the 8 keys s + 8k of words 2b
-//     and 2b+1.  Per channel one byte permute builds F for a key, heads that
-//     read the channel add coef*F with packed fp32x2 FMAs (two keys of the
-//     same block share the coefficient), heads that read fewer planes than
-//     the union mask F first, heads that read nothing cost nothing.
-//   The next chunk's plane words are loaded into registers before the
-//   current chunk is computed, so the loads overlap the arithmetic.
+// Work.  One CTA per (tile of 1024 keys, KV head).  A channel's codes in a
+// tile are 8 x 32 words: word (s, w) holds the codes of keys 32w + s + 8k,
+// k = 0..3, one per byte at bits 6..3.  The tile's active channels
+// (U_c > 0) are streamed in chunks of 16:
+//   stage: thread (channel group, plane word w) loads the U_c plane words of
+//     its channels (row pointers prepared once per tile) and transposes them
+//     to the 8 code words (s, w) (rotate + mask per plane and word), stored
+//     with conflict-free 32-bit stores.  Thread (channel, block) pairs form
+//     the coefficients 32 q Delta of every head and add Delta q (2^(3-t) - 24)
+//     into a per-(block, head) constant kept in registers.
+//   compute: warp (head h, key split) walks head h's item list of the chunk:
+//     the channels h reads, first those read to the union depth, then those
+//     read to fewer planes (their code bytes masked to t planes).  Lane
+//     (block b, variant half) owns 32 / S keys of block b: per item one
+//     coefficient load, 64-bit loads of its code words, and per key one byte
+//     permute building F and one FMA.  No per-head branch, no unread channel.
+//   The next chunk's plane words and scales are loaded into registers before
+//   the current chunk is computed, so the loads overlap the arithmetic.
 // The same kernel serves a host-resident store: its loads then cross the host
 // link as 128-byte runs per (channel, plane) and tile.
 #include "fathom_internal.cuh"
@@ -43,62 +46,87 @@ namespace {
 constexpr int kTileKeys = 1024;
 constexpr int kTileWords = kTileKeys / 32;   // 32 plane words per tile row
 constexpr int kTileBlocks = kTileKeys / kBlock;
-constexpr int kThreads = 128;                // (16 blocks) x (8 variants)
+constexpr int kChanWords = 8 * kTileWords;   // code words of one channel in a tile
 constexpr int kChunk = 16;                   // active channels per stage
-constexpr int kCPad = 20;                    // words per (word, variant) code row; 20 = 4 mod 8
 constexpr uint32_t kHalfExp = 0x3F000000u;   // bits of 0.5f: exponent byte of F
-constexpr bool kScanPacked = true;           // fp32x2 FMAs: two keys of a block per instruction
 
-struct ScanSmem {
-    static size_t bytes(int d, int G) {
-        size_t s = sizeof(uint32_t) * 2 * kTileWords * 8 * kCPad;   // codes, double-buffered
-        s += sizeof(float) * 2 * kChunk * kTileBlocks * G;          // coefficients, double-buffered
-        s += sizeof(float) * (size_t)d * G * 2;                     // 32 q, constant factor
-        s += sizeof(uint32_t) * (size_t)d * G;                      // masks
-        s += sizeof(uint32_t) * (size_t)d * 3;                      // meta, channel, U
-        s += (size_t)G * d + 64;                                    // t [G][d]
-        return s;
-    }
+// Launch geometry for G query heads per KV head.
+template <int G>
+struct Geo {
+    static constexpr int S = G >= 4 ? 1 : 4 / G;    // warps per query head (key splits)
+    static constexpr int NW = G * S;                // warps per CTA
+    static constexpr int T = 32 * NW;               // threads per CTA
+    static constexpr int NSV = 4 / S;               // code variants per compute thread
+    static constexpr int CPT = kChunk / NW;         // staged channels per thread
+    static constexpr int DPT = kChunk * kTileBlocks / T;   // staged (channel, block) scales per thread
+    static constexpr int MinBlocks = T <= 128 ? 4 : 2;
+    static_assert(CPT >= 1 && DPT >= 1 && NSV >= 1, "geometry");
 };
 
-__device__ __forceinline__ uint64_t pack2(uint32_t lo, uint32_t hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
-    return r;
-}
-__device__ __forceinline__ void fma2(uint64_t& acc, uint64_t a, uint64_t b) {
-    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
-}
-__device__ __forceinline__ float2 unpack2(uint64_t v) {
-    uint32_t lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
-    return make_float2(__uint_as_float(lo), __uint_as_float(hi));
-}
-// fp32 mask keeping sign, exponent and the top t code bits (mantissa 22..19)
-__device__ __forceinline__ uint32_t depth_mask(uint32_t t) {
-    return 0xFF800000u | ((((0xFu << (4u - t)) & 0xFu)) << 19);
+// Shared memory of one CTA (byte offsets; every region 16-byte aligned for d % 32 == 0).
+struct ScanSmem {
+    int d, G;
+    __host__ __device__ size_t codes() const { return 0; }   // [2][kChunk][8][32] u32
+    __host__ __device__ size_t coef() const { return codes() + 2u * kChunk * kChanWords * 4; }   // [2][G][kChunk][16] f32
+    __host__ __device__ size_t prow() const { return coef() + 2u * G * kChunk * kTileBlocks * 4; }   // [d] plane-0 row ptr
+    __host__ __device__ size_t srow() const { return prow() + (size_t)d * 8; }      // [d] scale row ptr
+    __host__ __device__ size_t items() const { return srow() + (size_t)d * 8; }     // [G][d] u32
+    __host__ __device__ size_t q32() const { return items() + (size_t)G * d * 4; }   // [d][G] f32
+    __host__ __device__ size_t qk() const { return q32() + (size_t)G * d * 4; }      // [d][G] f32
+    __host__ __device__ size_t off() const { return qk() + (size_t)G * d * 4; }      // [G][d/8 + 4] i32
+    __host__ __device__ size_t act() const { return off() + (size_t)G * (d / 8 + 4) * 4; }   // [d] i32
+    __host__ __device__ size_t uni() const { return act() + (size_t)d * 4; }         // [d] u8
+    __host__ __device__ size_t tdep() const { return uni() + (size_t)d; }            // [G][d] u8
+    __host__ __device__ size_t bytes() const { return (tdep() + (size_t)G * d + 15) & ~size_t(15); }
+};
+
+// F of byte k of a code word (he = kHalfExp)
+__device__ __forceinline__ float f_of(uint32_t x, uint32_t he, uint32_t k) {
+    return __uint_as_float(__byte_perm(x, he, 0x7044u | (k << 8)));
 }
 
-// Transposes one 32-key plane word column of a channel (U planes) into the
-// byte-code variant `sv`: byte k = code of key sv + 8k, planes at bits 6..3.
-template <int U>
-__device__ __forceinline__ uint32_t code_variant(const uint32_t* p, int sv) {
-    uint32_t x = 0;
+// G consecutive floats of shared memory (16-byte aligned when G >= 4), or zeros
+template <int G>
+__device__ __forceinline__ void load_g(const float* p, bool ok, float (&v)[G]) {
+    if constexpr (G % 4 == 0) {
 #pragma unroll
-    for (int j = 0; j < U; ++j)
-        x |= __funnelshift_r(p[j], p[j], (uint32_t)(sv + j - 6) & 31u) & (0x01010101u << (6 - j));
-    return x;
+        for (int i = 0; i < G; i += 4) {
+            const float4 t = *reinterpret_cast<const float4*>(p + i);
+            v[i] = t.x; v[i + 1] = t.y; v[i + 2] = t.z; v[i + 3] = t.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < G; ++i) v[i] = p[i];
+    }
+#pragma unroll
+    for (int i = 0; i < G; ++i) v[i] = ok ? v[i] : 0.0f;
 }
 
 // One (tile of 1024 keys, KV head g) of one store; q, depths and scores are
 // the store's own [Hq][d], [Hq][d] and [Hq][n_pad] arrays.
-template <int G, bool kPacked>
+template <int G>
 __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ scales,
                                           int d, int64_t n, int64_t n_pad, int tile, int g,
                                           const void* __restrict__ q, int q_dtype,
                                           const uint8_t* __restrict__ depths, float* __restrict__ scores,
                                           unsigned int* status) {
+    using Z = Geo<G>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
+    const ScanSmem lay{d, G};
+    uint32_t* s_codes = reinterpret_cast<uint32_t*>(smem_raw + lay.codes());
+    float* s_coef = reinterpret_cast<float*>(smem_raw + lay.coef());
+    const uint32_t** s_prow = reinterpret_cast<const uint32_t**>(smem_raw + lay.prow());
+    const uint16_t** s_srow = reinterpret_cast<const uint16_t**>(smem_raw + lay.srow());
+    uint32_t* s_items = reinterpret_cast<uint32_t*>(smem_raw + lay.items());
+    float* s_q32 = reinterpret_cast<float*>(smem_raw + lay.q32());
+    float* s_qk = reinterpret_cast<float*>(smem_raw + lay.qk());
+    int* s_off = reinterpret_cast<int*>(smem_raw + lay.off());
+    int* s_act = reinterpret_cast<int*>(smem_raw + lay.act());
+    uint8_t* s_U = smem_raw + lay.uni();
+    uint8_t* s_t = smem_raw + lay.tdep();
+    __shared__ int s_L;
+    const int off_stride = d / 8 + 4;
+
     const int64_t tile0 = (int64_t)tile * kTileKeys;
     const int64_t words_total = n_pad / 32;
     const int64_t nblk_total = n_pad / kBlock;
@@ -106,23 +134,11 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
     const int nwords = wrem < kTileWords ? (int)wrem : kTileWords;   // multiple of 4
     const int nblocks = nwords / 2;
 
-    uint32_t* s_codes = reinterpret_cast<uint32_t*>(smem_raw);                 // [2][32][8][kCPad]
-    float* s_coef = reinterpret_cast<float*>(s_codes + 2 * kTileWords * 8 * kCPad);   // [2][kChunk][16][G]
-    float* s_q32 = s_coef + 2 * kChunk * kTileBlocks * G;                        // [L][G]: 32 q (0 if t = 0)
-    float* s_kc = s_q32 + (size_t)d * G;                                         // [L][G]: (2^(3-t) - 24) / 32
-    uint32_t* s_mask = reinterpret_cast<uint32_t*>(s_kc + (size_t)d * G);        // [L][G]
-    uint32_t* s_meta = s_mask + (size_t)d * G;                                   // [L]: act | part << 8
-    int* s_act = reinterpret_cast<int*>(s_meta + d);                             // [L]: channel
-    int* s_U = s_act + d;                                                        // [L]: union depth
-    uint8_t* s_t = reinterpret_cast<uint8_t*>(s_U + d);                          // [G][d]
-    __shared__ int s_L;
-
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // ---- plan: depths, union, active channels, per (channel, head) factors ----
-    for (int e = tid; e < G * d; e += kThreads) {
-        int hh = e / d, c = e - hh * d;
-        int t = depths[((int64_t)g * G + hh) * d + c];
+    // ---- plan: depths, union list, row pointers, per-head item lists, per-(channel, head) factors ----
+    for (int e = tid; e < G * d; e += Z::T) {
+        int t = depths[(int64_t)g * G * d + e];
         if (t > 4) {
             atomicOr(status, (unsigned)FATHOM_DEV_BAD_DEPTH);
             t = 0;
@@ -135,25 +151,13 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
         for (int c0 = 0; c0 < d; c0 += 32) {
             const int c = c0 + lane;
             int U = 0;
-            uint32_t act = 0;
 #pragma unroll
-            for (int hh = 0; hh < G; ++hh) {
-                const int t = s_t[hh * d + c];
-                U = max(U, t);
-                act |= (t > 0 ? 1u : 0u) << hh;
-            }
-            uint32_t part = 0;
-#pragma unroll
-            for (int hh = 0; hh < G; ++hh) {
-                const int t = s_t[hh * d + c];
-                part |= (t > 0 && t < U ? 1u : 0u) << hh;
-            }
+            for (int hh = 0; hh < G; ++hh) U = max(U, (int)s_t[hh * d + c]);
             const unsigned m = __ballot_sync(0xffffffffu, U > 0);
             if (U > 0) {
                 const int pos = base + __popc(m & ((1u << lane) - 1u));
                 s_act[pos] = c;
-                s_U[pos] = U;
-                s_meta[pos] = act | (part << 8);
+                s_U[pos] = (uint8_t)U;
             }
             base += __popc(m);
         }
@@ -162,197 +166,215 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
     __syncthreads();
     const int L = s_L;
     const int nchunks = (L + kChunk - 1) / kChunk;
-    for (int e = tid; e < L * G; e += kThreads) {
+    for (int a = tid; a < L; a += Z::T) {
+        const int64_t row = (int64_t)g * d + s_act[a];
+        s_prow[a] = planes + row * 4 * words_total + tile0 / 32;
+        s_srow[a] = scales + row * nblk_total + tile0 / kBlock;
+    }
+    for (int e = tid; e < L * G; e += Z::T) {
         const int a = e / G, hh = e - a * G;
         const int c = s_act[a];
         const int t = s_t[hh * d + c];
         const float qv = load_q(q, q_dtype, ((int64_t)g * G + hh) * d + c);
         s_q32[e] = (t > 0) ? 32.0f * qv : 0.0f;
-        s_kc[e] = (t > 0) ? (__uint_as_float((uint32_t)(130 - t) << 23) - 24.0f) * 0.03125f : 0.0f;
-        s_mask[e] = (t > 0) ? depth_mask((uint32_t)t) : 0u;
+        s_qk[e] = (t > 0) ? qv * (__uint_as_float((uint32_t)(130 - t) << 23) - 24.0f) : 0.0f;
+    }
+    if (warp < G) {
+        // item list of head h = warp, chunk by chunk: channels read to the
+        // union depth, then channels read to fewer planes.  An item holds the
+        // word offset of the channel's codes in a chunk buffer (slot *
+        // kChanWords, bits 0..11) and, for a shallower read, the byte mask
+        // (bits 16..23)
+        const int h = warp;
+        uint32_t* items = s_items + h * d;
+        int* off = s_off + h * off_stride;
+        int base = 0;
+        for (int a0 = 0; a0 < L; a0 += 32) {
+            const int a = a0 + lane;
+            const int t = (a < L) ? (int)s_t[h * d + s_act[a]] : 0;
+            const int U = (a < L) ? (int)s_U[a] : 0;
+            const bool full = t > 0 && t == U, part = t > 0 && t < U;
+            const unsigned mf = __ballot_sync(0xffffffffu, full);
+            const unsigned mp = __ballot_sync(0xffffffffu, part);
+            const int nf0 = __popc(mf & 0xFFFFu), np0 = __popc(mp & 0xFFFFu);
+            const int nf1 = __popc(mf >> 16), np1 = __popc(mp >> 16);
+            const int start0 = base, start1 = base + nf0 + np0;
+            const bool upper = lane >= 16;
+            const unsigned below = ((1u << lane) - 1u) & (upper ? 0xFFFF0000u : 0x0000FFFFu);
+            const int cstart = upper ? start1 : start0, cnf = upper ? nf1 : nf0;
+            const uint32_t slot = (uint32_t)(a & 15) * kChanWords;
+            if (full) items[cstart + __popc(mf & below)] = slot;
+            if (part) items[cstart + cnf + __popc(mp & below)] = slot | (((0x780u >> t) & 0x78u) << 16);
+            if (lane == 0) {
+                const int ch = a0 / 16;
+                off[2 * ch] = start0;
+                off[2 * ch + 1] = start0 + nf0;
+                off[2 * ch + 2] = start1;
+                off[2 * ch + 3] = start1 + nf1;
+            }
+            base = start1 + nf1 + np1;
+        }
+        if (lane == 0) off[2 * nchunks] = base;
     }
     __syncthreads();
 
-    // ---- stage / compute roles ----
-    const int cg = warp, w = lane;               // stage: channel group of 4, plane word
-    const int b = tid >> 3, s = tid & 7;         // compute: block (words 2b, 2b+1), variant
+    // ---- stage role: channels cg*CPT + i of a chunk at plane word w; scales (al, bb) ----
+    const int cg = warp, w = lane;
+    const bool wok = w < nwords;
+    const int bb = tid & 15;   // block of this thread's scales (the same for every u: T is a multiple of 16)
+    uint32_t pw[Z::CPT][4];
+    float pd[Z::DPT];
+    float cstp[G];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) cstp[hh] = 0.0f;
 
-    uint32_t pw[4][4];   // prefetched plane words: [channel in group][plane]
-    float pd[2];         // prefetched scales of (channel, block) items tid and tid + 128
     auto load_chunk = [&](int ch) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int a = ch * kChunk + cg * 4 + i;
-            const int U = (a < L) ? s_U[a] : 0;
-            const uint32_t* row = planes + ((int64_t)g * d + ((a < L) ? s_act[a] : 0)) * 4 * words_total +
-                                  tile0 / 32 + w;
+        for (int i = 0; i < Z::CPT; ++i) {
+            const int a = ch * kChunk + cg * Z::CPT + i;   // warp-uniform
+            const int U = (a < L && wok) ? s_U[a] : 0;
+            const uint32_t* p = ((a < L) ? s_prow[a] : planes) + w;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                pw[i][j] = (j < U && w < nwords) ? __ldg(row + (int64_t)j * words_total) : 0u;
+            for (int j = 0; j < 4; ++j) pw[i][j] = (j < U) ? __ldg(p + j * words_total) : 0u;
         }
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = tid + u * kThreads, al = e >> 4, bb = e & 15;
-            const int a = ch * kChunk + al;
-            pd[u] = (a < L && bb < nblocks)
-                        ? __half2float(__ushort_as_half(__ldg(scales + ((int64_t)g * d + s_act[a]) * nblk_total +
-                                                              tile0 / kBlock + bb)))
-                        : 0.0f;
+        for (int u = 0; u < Z::DPT; ++u) {
+            const int a = ch * kChunk + ((tid + u * Z::T) >> 4);
+            pd[u] = (a < L && bb < nblocks) ? __half2float(__ushort_as_half(__ldg(s_srow[a] + bb))) : 0.0f;
         }
     };
     auto store_chunk = [&](int ch, int buf) {
-        uint32_t x[4][8];
+        uint32_t* cbase = s_codes + (size_t)buf * kChunk * kChanWords + w;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int a = ch * kChunk + cg * 4 + i;
-            const int U = (a < L) ? s_U[a] : 0;
-            switch (U) {
-                case 4:
+        for (int i = 0; i < Z::CPT; ++i) {
+            const int al = cg * Z::CPT + i, a = ch * kChunk + al;
+            const int U = (a < L) ? s_U[a] : 0;   // warp-uniform
+            uint32_t x[8];
 #pragma unroll
-                    for (int sv = 0; sv < 8; ++sv) x[i][sv] = code_variant<4>(pw[i], sv);
-                    break;
-                case 3:
+            for (int sv = 0; sv < 8; ++sv) x[sv] = 0u;
 #pragma unroll
-                    for (int sv = 0; sv < 8; ++sv) x[i][sv] = code_variant<3>(pw[i], sv);
-                    break;
-                case 2:
+            for (int j = 0; j < 4; ++j) {
+                if (j < U) {
 #pragma unroll
-                    for (int sv = 0; sv < 8; ++sv) x[i][sv] = code_variant<2>(pw[i], sv);
-                    break;
-                case 1:
-#pragma unroll
-                    for (int sv = 0; sv < 8; ++sv) x[i][sv] = code_variant<1>(pw[i], sv);
-                    break;
-                default:
-#pragma unroll
-                    for (int sv = 0; sv < 8; ++sv) x[i][sv] = 0u;
+                    for (int sv = 0; sv < 8; ++sv)
+                        x[sv] |= __funnelshift_r(pw[i][j], pw[i][j], (uint32_t)(sv + j - 6) & 31u) &
+                                 (0x01010101u << (6 - j));
+                }
             }
+#pragma unroll
+            for (int sv = 0; sv < 8; ++sv) cbase[al * kChanWords + sv * kTileWords] = x[sv];
         }
-        uint32_t* base = s_codes + (size_t)buf * kTileWords * 8 * kCPad;
+        float* cf = s_coef + (size_t)buf * G * kChunk * kTileBlocks;
 #pragma unroll
-        for (int sv = 0; sv < 8; ++sv) {
-            // XOR swizzle of the variant row keeps both these stores and the
-            // compute-phase loads free of bank conflicts
-            const int prow = w * 8 + (sv ^ (w & 7));
-            *reinterpret_cast<uint4*>(base + (size_t)prow * kCPad + cg * 4) = make_uint4(x[0][sv], x[1][sv], x[2][sv], x[3][sv]);
-        }
-        float* cbuf = s_coef + (size_t)buf * kChunk * kTileBlocks * G;
+        for (int u = 0; u < Z::DPT; ++u) {
+            const int al = (tid + u * Z::T) >> 4, a = ch * kChunk + al;   // a < d: nchunks * 16 <= d
+            float qv[G], kv[G];
+            load_g<G>(s_q32 + a * G, a < L, qv);
+            load_g<G>(s_qk + a * G, a < L, kv);
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = tid + u * kThreads, al = e >> 4, bb = e & 15;
-            const int a = min(ch * kChunk + al, max(L - 1, 0));
-#pragma unroll
-            for (int hh = 0; hh < G; ++hh) cbuf[(al * kTileBlocks + bb) * G + hh] = s_q32[a * G + hh] * pd[u];
+            for (int hh = 0; hh < G; ++hh) {
+                cf[(hh * kChunk + al) * kTileBlocks + bb] = qv[hh] * pd[u];
+                cstp[hh] = fmaf(kv[hh], pd[u], cstp[hh]);
+            }
         }
     };
 
-    float acc[G][8];
-    float cst[G];
+    // ---- compute role: head h; lane (block b, variant half) ----
+    const int h = warp / Z::S, sp = warp % Z::S;
+    const int b = lane & 15, sv0 = Z::NSV * (2 * sp + (lane >> 4));
+    // key of acc[i][wd][k]: 64 b + 32 wd + sv0 + i + 8 k
+    float acc[Z::NSV][2][4];
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-        cst[hh] = 0.0f;
+    for (int i = 0; i < Z::NSV; ++i)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[hh][e] = 0.0f;
-    }
+        for (int k = 0; k < 4; ++k) acc[i][0][k] = acc[i][1][k] = 0.0f;
+    const uint32_t he = kHalfExp;
+    const uint32_t* cth = s_codes + sv0 * kTileWords + 2 * b;                  // + buffer + slot + i * 32
+    const float* cfth = s_coef + (size_t)h * kChunk * kTileBlocks + b;         // + buffer + slot * 16
+
+    auto item = [&](const uint32_t* cb, const float* cfb, uint32_t it, bool masked) {
+        const uint32_t slot = it & 0xFFFu;
+        const uint32_t* rp = cb + slot;
+        const float c = cfb[slot >> 4];                       // slot / kChanWords * kTileBlocks
+        const uint32_t mk = __byte_perm(it, 0u, 0x2222u);     // byte 2 in all four bytes
+#pragma unroll
+        for (int i = 0; i < Z::NSV; ++i) {
+            const uint2 X = *reinterpret_cast<const uint2*>(rp + i * kTileWords);
+            const uint32_t x0 = masked ? (X.x & mk) : X.x, x1 = masked ? (X.y & mk) : X.y;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                acc[i][0][k] = fmaf(c, f_of(x0, he, (uint32_t)k), acc[i][0][k]);
+                acc[i][1][k] = fmaf(c, f_of(x1, he, (uint32_t)k), acc[i][1][k]);
+            }
+        }
+    };
 
     if (nchunks > 0) {
         load_chunk(0);
         store_chunk(0, 0);
     }
     __syncthreads();
+    const uint32_t* items = s_items + h * d;
+    const int* off = s_off + h * off_stride;
     for (int ch = 0; ch < nchunks; ++ch) {
         const int buf = ch & 1;
         if (ch + 1 < nchunks) load_chunk(ch + 1);
-        if (b < nblocks) {
-            const uint32_t* cbase = s_codes + (size_t)buf * kTileWords * 8 * kCPad;
-            const uint32_t* row0 = cbase + ((size_t)(2 * b) * 8 + (s ^ ((2 * b) & 7))) * kCPad;
-            const uint32_t* row1 = cbase + ((size_t)(2 * b + 1) * 8 + (s ^ ((2 * b + 1) & 7))) * kCPad;
-            const float* cbuf = s_coef + (size_t)buf * kChunk * kTileBlocks * G;
-            const int nloc = min(kChunk, L - ch * kChunk);
-            for (int i4 = 0; i4 < nloc; i4 += 4) {
-                const uint4 X0 = *reinterpret_cast<const uint4*>(row0 + i4);
-                const uint4 X1 = *reinterpret_cast<const uint4*>(row1 + i4);
-                const uint32_t xs0[4] = {X0.x, X0.y, X0.z, X0.w};
-                const uint32_t xs1[4] = {X1.x, X1.y, X1.z, X1.w};
-#pragma unroll
-                for (int ii = 0; ii < 4; ++ii) {
-                    if (i4 + ii >= nloc) break;
-                    const int al = i4 + ii, a = ch * kChunk + al;
-                    const uint32_t meta = s_meta[a];
-                    float cf[G], kc[G];
-                    uint32_t mk[G];
-#pragma unroll
-                    for (int hh = 0; hh < G; ++hh) {
-                        cf[hh] = cbuf[(al * kTileBlocks + b) * G + hh];
-                        kc[hh] = s_kc[a * G + hh];
-                        mk[hh] = s_mask[a * G + hh];
-                    }
-                    uint32_t F[8];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        F[k] = __byte_perm(xs0[ii], kHalfExp, 0x7044u | ((uint32_t)k << 8));
-                        F[4 + k] = __byte_perm(xs1[ii], kHalfExp, 0x7044u | ((uint32_t)k << 8));
-                    }
-#pragma unroll
-                    for (int hh = 0; hh < G; ++hh) {
-                        if (!(meta & (1u << hh))) continue;
-                        cst[hh] = fmaf(cf[hh], kc[hh], cst[hh]);
-                        uint32_t Fm[8];
-                        if (meta & (0x100u << hh)) {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) Fm[e] = F[e] & mk[hh];
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) Fm[e] = F[e];
-                        }
-                        if constexpr (kPacked) {
-                            const uint64_t c2 = pack2(__float_as_uint(cf[hh]), __float_as_uint(cf[hh]));
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                uint64_t a2 = pack2(__float_as_uint(acc[hh][2 * e]), __float_as_uint(acc[hh][2 * e + 1]));
-                                fma2(a2, c2, pack2(Fm[2 * e], Fm[2 * e + 1]));
-                                const float2 r = unpack2(a2);
-                                acc[hh][2 * e] = r.x;
-                                acc[hh][2 * e + 1] = r.y;
-                            }
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(cf[hh], __uint_as_float(Fm[e]), acc[hh][e]);
-                        }
-                    }
-                }
-            }
-        }
+        const uint32_t* cb = cth + (size_t)buf * kChunk * kChanWords;
+        const float* cfb = cfth + (size_t)buf * G * kChunk * kTileBlocks;
+        const int f0 = off[2 * ch], p0 = off[2 * ch + 1], e0 = off[2 * ch + 2];
+        for (int k = f0; k < p0; ++k) item(cb, cfb, items[k], false);
+        for (int k = p0; k < e0; ++k) item(cb, cfb, items[k], true);
         if (ch + 1 < nchunks) store_chunk(ch + 1, buf ^ 1);
         __syncthreads();
     }
 
-    // ---- epilogue: F[k] / F[4+k] are keys s + 8k of words 2b / 2b+1 ----
+    // ---- constants: the per-thread partials of each (block, head), summed in a fixed order ----
+    float* s_cred = reinterpret_cast<float*>(smem_raw + lay.codes());   // [NW][16][G]; the codes are dead now
+    float* s_cst = s_cred + Z::NW * 16 * G;                              // [G][16]
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+        const float v = cstp[hh] + __shfl_xor_sync(0xffffffffu, cstp[hh], 16);
+        if (lane < 16) s_cred[(warp * 16 + lane) * G + hh] = v;
+    }
+    __syncthreads();
+    if (tid < 16 * G) {
+        const int hh = tid >> 4, b16 = tid & 15;
+        float v = 0.0f;
+        for (int wv = 0; wv < Z::NW; ++wv) v += s_cred[(wv * 16 + b16) * G + hh];
+        s_cst[hh * 16 + b16] = v;
+    }
+    __syncthreads();
+
+    // ---- epilogue ----
     if (b < nblocks) {
+        const int64_t k0 = tile0 + 64 * b + sv0;   // key of acc[0][0][0]
+        float* out = scores + ((int64_t)g * G + h) * n_pad + k0;
+        const float cst = s_cst[h * 16 + b];
+        const bool whole = tile0 + kTileKeys <= n;
 #pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-            float* out = scores + ((int64_t)g * G + hh) * n_pad + tile0;
+        for (int i = 0; i < Z::NSV; ++i)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int64_t i = 32 * (2 * b + (e >> 2)) + s + 8 * (e & 3);
-                out[i] = (tile0 + i < n) ? acc[hh][e] + cst[hh] : -INFINITY;
-            }
-        }
+            for (int wd = 0; wd < 2; ++wd)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int o = 32 * wd + i + 8 * k;
+                    const float v = acc[i][wd][k] + cst;
+                    out[o] = (whole || k0 + o < n) ? v : -INFINITY;
+                }
     }
 }
 
 template <int G>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(Geo<G>::T, Geo<G>::MinBlocks)
 scan_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ scales, int d, int64_t n,
             int64_t n_pad, const void* __restrict__ q, int q_dtype, const uint8_t* __restrict__ depths,
             float* __restrict__ scores, unsigned int* status) {
-    scan_tile<G, kScanPacked>(planes, scales, d, n, n_pad, (int)blockIdx.x, (int)blockIdx.y, q, q_dtype, depths,
-                              scores, status);
+    scan_tile<G>(planes, scales, d, n, n_pad, (int)blockIdx.x, (int)blockIdx.y, q, q_dtype, depths, scores, status);
 }
 
 // Batched sessions: blockIdx.x runs over the tiles of all sessions.
 template <int G>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(Geo<G>::T, Geo<G>::MinBlocks)
 scan_batched_kernel(const __grid_constant__ SessionMap map, int d, int Hq, const void* __restrict__ q, int q_dtype,
                     const uint8_t* __restrict__ depths, float* __restrict__ scores, unsigned int* status) {
     const int t = (int)blockIdx.x;
@@ -367,40 +389,39 @@ scan_batched_kernel(const __grid_constant__ SessionMap map, int d, int Hq, const
     const void* qs = (q_dtype == FATHOM_BF16)
                          ? static_cast<const void*>(static_cast<const uint16_t*>(q) + sidx * qstride)
                          : static_cast<const void*>(static_cast<const float*>(q) + sidx * qstride);
-    scan_tile<G, kScanPacked>(map.planes[sidx], map.scales[sidx], d, map.n[sidx], map.n_pad[sidx],
-                              t - map.tile0[sidx], (int)blockIdx.y, qs, q_dtype, depths + sidx * qstride,
-                              scores + map.score_base[sidx], status);
+    scan_tile<G>(map.planes[sidx], map.scales[sidx], d, map.n[sidx], map.n_pad[sidx], t - map.tile0[sidx],
+                 (int)blockIdx.y, qs, q_dtype, depths + sidx * qstride, scores + map.score_base[sidx], status);
 }
 
 template <int G>
 cudaError_t launch_scan_g(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n,
                           int64_t n_pad, const void* q, int q_dtype, const uint8_t* depths, float* scores,
                           cudaStream_t stream) {
-    size_t smem = ScanSmem::bytes(d, G);
+    const size_t smem = ScanSmem{d, G}.bytes();
     auto kern = scan_kernel<G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((n_pad + kTileKeys - 1) / kTileKeys), (unsigned)Hkv);
-    kern<<<grid, kThreads, smem, stream>>>(planes, scales, d, n, n_pad, q, q_dtype, depths, scores,
-                                           device_status_ptr());
+    kern<<<grid, Geo<G>::T, smem, stream>>>(planes, scales, d, n, n_pad, q, q_dtype, depths, scores,
+                                            device_status_ptr());
     return cudaGetLastError();
 }
 
 template <int G>
 cudaError_t launch_scan_batched_g(const SessionMap& map, int Hkv, int d, const void* q, int q_dtype,
                                   const uint8_t* depths, int Hq, float* scores, cudaStream_t stream) {
-    size_t smem = ScanSmem::bytes(d, G);
+    const size_t smem = ScanSmem{d, G}.bytes();
     auto kern = scan_batched_kernel<G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)map.tile0[map.nsess], (unsigned)Hkv);
-    kern<<<grid, kThreads, smem, stream>>>(map, d, Hq, q, q_dtype, depths, scores, device_status_ptr());
+    kern<<<grid, Geo<G>::T, smem, stream>>>(map, d, Hq, q, q_dtype, depths, scores, device_status_ptr());
     return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t scan_smem_bytes(int d, int G) { return ScanSmem::bytes(d, G); }
+size_t scan_smem_bytes(int d, int G) { return ScanSmem{d, G}.bytes(); }
 
 cudaError_t launch_scan(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n, int64_t n_pad,
                         const void* q, int q_dtype, const uint8_t* depths, int Hq, float* scores,
