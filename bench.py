@@ -185,7 +185,11 @@ class Layer:
         self.dev_store = st
         if resident == "host":
             self.store = F.Store(self._pin(st.planes), self._pin(st.scales), self.n, host_resident=True)
-            self.K_rows, self.V_rows = self._pin(inp["K_rows"]), self._pin(inp["V_rows"])
+            # one interleaved [Hkv][n][2][d] page-locked buffer: a key's K and V
+            # rows cross the host link as one 512-byte run
+            self.K_rows, self.V_rows = F.kv_rows(self.Hkv, self.n, self.d, pin_memory=True)
+            self.K_rows.copy_(inp["K_rows"])
+            self.V_rows.copy_(inp["V_rows"])
         else:
             self.store = st
             self.K_rows, self.V_rows = inp["K_rows"], inp["V_rows"]

@@ -260,13 +260,14 @@ int fathom_scan_topk_batched(const fathom_store* stores, int n_sessions, const v
 }
 
 int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
-                         int rows_host_resident, const int32_t* idx, int n_q_heads, int n_kv_heads, int64_t n,
+                         int64_t row_stride, int rows_host_resident, const int32_t* idx, int n_q_heads, int n_kv_heads, int64_t n,
                          int d, int k, float* out, fathom_stream_t stream) {
     if (!q || !K_rows || !V_rows || !idx || !out || n < 1 || k < 1 || !dims_ok(n_kv_heads, d) ||
         !heads_ok(n_q_heads, n_kv_heads))
         return FATHOM_EINVAL;
     if (q_dtype != FATHOM_F32 && q_dtype != FATHOM_BF16) return FATHOM_EINVAL;
     if (d != 32 && d != 64 && d != 128 && d != 256) return FATHOM_EUNSUPPORTED;
+    if (row_stride < d || row_stride % 8) return FATHOM_EINVAL;
     if ((reinterpret_cast<uintptr_t>(K_rows) & 15) || (reinterpret_cast<uintptr_t>(V_rows) & 15))
         return FATHOM_EINVAL;
     const void* kd = nullptr;
@@ -276,7 +277,7 @@ int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, con
     if (!is_device(q) || !is_device(idx) || !is_device(out)) return FATHOM_EINVAL;
     if (!device_status_ptr()) return FATHOM_ECUDA;
     return to_status(launch_attend(q, q_dtype, static_cast<const uint16_t*>(kd), static_cast<const uint16_t*>(vd),
-                                   idx, n_q_heads, n_kv_heads, n, d, k, rows_host_resident, out,
+                                   row_stride, idx, n_q_heads, n_kv_heads, n, d, k, rows_host_resident, out,
                                    (cudaStream_t)stream));
 }
 

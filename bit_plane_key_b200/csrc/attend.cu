@@ -12,10 +12,12 @@
 // memory, then CTA 0 merges the kSplit CTA partials through distributed
 // shared memory and writes o_h.  No workspace and no second kernel.
 // Rows may live in device memory or in page-locked host memory.  Over the
-// host link, gathering rows in address order is about twice as fast as in
-// score order, so for host-resident rows every CTA first sorts the head's
-// indices in shared memory; the head's 32 warps then sweep the sorted list
-// together (the softmax sum does not depend on the order).
+// host link, gathering rows in address order is faster than in score order,
+// so for host-resident rows every CTA first sorts the head's indices in
+// shared memory; the head's 32 warps then sweep the sorted list together
+// (the softmax sum does not depend on the order).  Rows are addressed with a
+// row stride, so K and V may be two arrays or one interleaved [n][2][d]
+// array; the latter keeps a key's two rows in one run on the host link.
 #include <cooperative_groups.h>
 
 #include "fathom_internal.cuh"
@@ -28,7 +30,7 @@ namespace {
 constexpr int kSplit = 8;      // CTAs per head (cluster size)
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-constexpr int kUnroll = 4;     // rows in flight per warp
+constexpr int kUnroll = 8;     // rows in flight per warp
 constexpr int kSortCap = kMaxTopK;   // indices sorted in shared memory
 
 
@@ -62,8 +64,8 @@ __device__ __forceinline__ void load_row(const uint16_t* __restrict__ p, float* 
 template <int V>
 __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kThreads)
 attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restrict__ Kr,
-              const uint16_t* __restrict__ Vr, const int32_t* __restrict__ idx, int Hq, int Hkv, int64_t n,
-              int k, int sort_rows, float* __restrict__ out, unsigned int* status) {
+              const uint16_t* __restrict__ Vr, int64_t row_stride, const int32_t* __restrict__ idx, int Hq, int Hkv,
+              int64_t n, int k, int sort_rows, float* __restrict__ out, unsigned int* status) {
     constexpr int d = V * 32;
     __shared__ int32_t s_idx[kSortCap];
     __shared__ float s_m[kWarps], s_l[kWarps];
@@ -87,7 +89,7 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
     for (int e = 0; e < V; ++e) o[e] = 0.0f;
 
     const int32_t* ih = idx + (int64_t)h * k;
-    const int64_t head_base = (int64_t)g * n * d;
+    const int64_t head_base = (int64_t)g * n * row_stride;
     if (sort_rows) {
         // bitonic sort (ascending) of the head's indices, padded to a power of two
         int P = 1;
@@ -124,7 +126,7 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
                 const int64_t i = ih[p];
                 if (i >= 0 && i < n) {
                     ok[u] = true;
-                    const int64_t off = head_base + i * d + lane * V;
+                    const int64_t off = head_base + i * row_stride + lane * V;
                     load_row<V>(Kr + off, kv[u]);
                     load_row<V>(Vr + off, vv[u]);
                 } else if (lane == 0) {
@@ -202,19 +204,22 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
 }  // namespace
 
 cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
-                          const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k, int sort_rows, float* out,
-                          cudaStream_t stream) {
+                          int64_t row_stride, const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k,
+                          int sort_rows, float* out, cudaStream_t stream) {
     dim3 grid((unsigned)(Hq * kSplit));
     unsigned int* st = device_status_ptr();
     const int sr = (sort_rows && k <= kSortCap) ? 1 : 0;
+    auto go = [&](auto kern) {
+        kern<<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, row_stride, idx, Hq, Hkv, n, k, sr, out, st);
+        return cudaGetLastError();
+    };
     switch (d) {
-        case 32: attend_kernel<1><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, sr, out, st); break;
-        case 64: attend_kernel<2><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, sr, out, st); break;
-        case 128: attend_kernel<4><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, sr, out, st); break;
-        case 256: attend_kernel<8><<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, idx, Hq, Hkv, n, k, sr, out, st); break;
+        case 32: return go(attend_kernel<1>);
+        case 64: return go(attend_kernel<2>);
+        case 128: return go(attend_kernel<4>);
+        case 256: return go(attend_kernel<8>);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace fathom

@@ -74,7 +74,7 @@ struct SessionMap {
 cudaError_t launch_scan_batched(const SessionMap& map, int Hkv, int d, const void* q, int q_dtype,
                                 const uint8_t* depths, int Hq, float* scores, cudaStream_t stream);
 cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
-                          const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k, int sort_rows, float* out,
+                          int64_t row_stride, const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k, int sort_rows, float* out,
                           cudaStream_t stream);
 
 cudaError_t launch_probe(const void* src, size_t bytes, unsigned long long* sink, int ctas,

@@ -59,7 +59,7 @@ _sig("fathom_topk_workspace_bytes", _Z, [_L, _I, _I])
 _sig("fathom_topk", _I, [_P, _L, _L, _I, _I, _P, _P, _P, _Z, _P])
 _sig("fathom_scan_workspace_bytes", _Z, [_SP, _I, _I])
 _sig("fathom_scan_topk", _I, [_SP, _P, _I, _P, _I, _I, _P, _P, _P, _Z, _P])
-_sig("fathom_sparse_attend", _I, [_P, _I, _P, _P, _I, _P, _I, _I, _L, _I, _I, _P, _P])
+_sig("fathom_sparse_attend", _I, [_P, _I, _P, _P, _L, _I, _P, _I, _I, _L, _I, _I, _P, _P])
 _sig("fathom_last_device_status", _I, [_P])
 _sig("fathom_status_string", ctypes.c_char_p, [_I])
 _sig("fathom_read_probe", _I, [_P, _Z, _I, _P, _I, _P])
@@ -232,16 +232,29 @@ def scan_scores_view(workspace, n_q_heads, n_pad_keys):
     return workspace[: 4 * n_q_heads * n_pad_keys].view(torch.float32).view(n_q_heads, n_pad_keys)
 
 
+def kv_rows(n_kv_heads, n, d, device=None, pin_memory=False):
+    """K and V row views [Hkv][n][d] (bf16) of one interleaved [Hkv][n][2][d]
+    buffer: a key's K and V rows are adjacent, which is the layout to use for
+    rows kept in page-locked host memory."""
+    kv = torch.empty((n_kv_heads, n, 2, d), dtype=torch.bfloat16, device=device, pin_memory=pin_memory)
+    return kv[:, :, 0, :], kv[:, :, 1, :]
+
+
 def sparse_attend(q, K_rows, V_rows, idx, n_kv_heads=None, out=None, stream=None):
-    """o f32 [Hq][d]; K_rows/V_rows bf16 [Hkv][n][d] on the device or page-locked host."""
+    """o f32 [Hq][d]; K_rows/V_rows bf16 [Hkv][n][d] views with unit channel
+    stride and equal strides (two arrays, or the views of kv_rows()), on the
+    device or in page-locked host memory."""
     Hq, d = q.shape
     Hkv, n, _ = K_rows.shape
     k = idx.shape[1]
     host = not K_rows.is_cuda
+    if K_rows.stride() != V_rows.stride() or K_rows.stride(2) != 1 or K_rows.stride(0) != n * K_rows.stride(1):
+        raise ValueError("K_rows and V_rows need strides (n*s, s, 1), the same for both")
     if out is None:
         out = torch.empty((Hq, d), dtype=torch.float32, device=q.device)
-    _check(_lib.fathom_sparse_attend(_ptr(q), _dtype_code(q), _ptr(K_rows), _ptr(V_rows), int(host), _ptr(idx),
-                                     Hq, Hkv, n, d, int(k), _ptr(out), _stream(stream)), "fathom_sparse_attend")
+    _check(_lib.fathom_sparse_attend(_ptr(q), _dtype_code(q), _ptr(K_rows), _ptr(V_rows), int(K_rows.stride(1)),
+                                     int(host), _ptr(idx), Hq, Hkv, n, d, int(k), _ptr(out), _stream(stream)),
+           "fathom_sparse_attend")
     return out
 
 

@@ -235,17 +235,25 @@ int fathom_scan_topk_noalloc(const fathom_store* store, const void* q, int q_dty
  * out[h] = softmax_j(q[h] . K[g][idx[h][j]] / sqrt(d)) V[g][idx[h][j]],
  * g = h / (Hq/Hkv), fp32 accumulation.
  *   q       device, [Hq][d], FATHOM_F32 or FATHOM_BF16.
- *   K_rows, V_rows  bf16 bit patterns [Hkv][n][d]; device memory, or
- *           page-locked host memory when rows_host_resident = 1.
+ *   K_rows, V_rows  bf16 bit patterns: the row of key i of KV head g starts
+ *           at element (g * n + i) * row_stride; device memory, or page-locked
+ *           host memory when rows_host_resident = 1.  row_stride = d for two
+ *           plain [Hkv][n][d] arrays; row_stride = 2d with V_rows = K_rows + d
+ *           for one interleaved [Hkv][n][2][d] array, the layout to use for
+ *           host-resident rows: a key's K and V rows then cross the host link
+ *           as one 4d-byte run (on B200 over PCIe, K and V rows gathered from
+ *           two arrays gigabytes apart ran at about half the rate).
+ *           row_stride >= d and a multiple of 8; rows 16-byte aligned.
  *   idx     device, i32 [Hq][k], each in [0, n) (others are skipped and
  *           flagged FATHOM_DEV_BAD_INDEX).
  *   out     device, f32 [Hq][d].
  * Errors: EINVAL for null pointers, k < 1, bad head counts, d not a
- * multiple of 32 or d > 256, rows not where rows_host_resident says.
+ * multiple of 32 or d > 256, a bad row_stride, rows not where
+ * rows_host_resident says.
  */
 int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
-                         int rows_host_resident, const int32_t* idx, int n_q_heads, int n_kv_heads,
-                         int64_t n, int d, int k, float* out, fathom_stream_t stream);
+                         int64_t row_stride, int rows_host_resident, const int32_t* idx, int n_q_heads,
+                         int n_kv_heads, int64_t n, int d, int k, float* out, fathom_stream_t stream);
 
 /*
  * Reads and clears this device's status word (FATHOM_DEV_* bits) after

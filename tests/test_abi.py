@@ -63,4 +63,4 @@ def test_null_arguments_rejected_before_any_cuda_call(libpath):
     assert L.fathom_alloc_depths(None, 0, None, 1, 1, 32, 10, 0, None, None) == F.EINVAL
     assert L.fathom_topk(None, 10, 10, 1, 1, None, None, None, 0, None) == F.EINVAL
     assert L.fathom_scan_topk(None, None, 0, None, 1, 1, None, None, None, 0, None) == F.EINVAL
-    assert L.fathom_sparse_attend(None, 0, None, None, 0, None, 1, 1, 10, 128, 1, None, None) == F.EINVAL
+    assert L.fathom_sparse_attend(None, 0, None, None, 128, 0, None, 1, 1, 10, 128, 1, None, None) == F.EINVAL

@@ -137,9 +137,8 @@ def test_config5_decode_step_sampled_layers(ref):
         B = int(budgets[layer])
         inp = synth.layer_inputs_cuda(5, layer=layer, n=n, device=DEV, with_values=True)
         st = F.pack_bitplanes(inp["K"]).to_host()
-        Kr = torch.empty(inp["K_rows"].shape, dtype=torch.bfloat16, pin_memory=True)
+        Kr, Vr = F.kv_rows(8, n, 128, pin_memory=True)   # interleaved host rows, as a server keeps them
         Kr.copy_(inp["K_rows"])
-        Vr = torch.empty(inp["V_rows"].shape, dtype=torch.bfloat16, pin_memory=True)
         Vr.copy_(inp["V_rows"])
         dep = F.alloc_depths(inp["q_dev"], inp["sigma2_dev"], B)
         dep_h = dep.cpu().numpy()

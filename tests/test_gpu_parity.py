@@ -7,6 +7,7 @@ scores.  Tolerance: scan scores, |s_gpu - s_ref| <= 1e-4 * sum_c |q_c khat_c|
 equal index sets except keys whose fp64 score lies within the score
 tolerance of the k-th score.
 """
+import ctypes
 import json
 import os
 
@@ -358,21 +359,43 @@ def test_residency_mismatch_rejected():
 # --------------------------------------------------------------------------
 # a6: exact sparse attention
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("d,k,host_rows", [(128, 2048, False), (128, 5, False), (64, 300, False), (256, 64, False),
-                                           (32, 1, False), (128, 1000, True)])
-def test_sparse_attend(ref, d, k, host_rows):
+@pytest.mark.parametrize("d,k,host_rows,interleaved", [
+    (128, 2048, False, False), (128, 5, False, False), (64, 300, False, False), (256, 64, False, False),
+    (32, 1, False, False), (128, 1000, True, False), (128, 1000, True, True), (64, 777, False, True),
+    (256, 300, True, True)])
+def test_sparse_attend(ref, d, k, host_rows, interleaved):
     rng = np.random.default_rng(d + k)
     Hkv, G, n = 2, 4, 5000
     inp = make(2, n=n, Hkv=Hkv, Hq=Hkv * G, d=d, values=True)
     idx = np.stack([rng.choice(n, k, replace=False) for _ in range(Hkv * G)]).astype(np.int32)
     Kr, Vr = bf16(inp["K_rows"]), bf16(inp["V_rows"])
-    if host_rows:
+    if interleaved:   # one [Hkv][n][2][d] buffer, row stride 2d
+        Ki, Vi = F.kv_rows(Hkv, n, d, device=None if host_rows else DEV, pin_memory=host_rows)
+        Ki.copy_(Kr)
+        Vi.copy_(Vr)
+        assert Ki.stride(1) == 2 * d
+        Kr, Vr = Ki, Vi
+    elif host_rows:
         Kr, Vr = Kr.cpu().pin_memory(), Vr.cpu().pin_memory()
     out = host(F.sparse_attend(q_dev(inp), Kr, Vr, dev(idx)))
     want = ref.attend(inp["q"], inp["K_rows"], inp["V_rows"], idx)
     for h in range(Hkv * G):
         assert np.linalg.norm(out[h] - want[h]) <= 1e-3 * np.linalg.norm(want[h]), h
     assert F.last_device_status() == 0
+
+
+def test_sparse_attend_rejects_bad_row_stride():
+    inp = make(2, n=300, Hkv=1, Hq=4, d=128, values=True)
+    Kr, Vr = bf16(inp["K_rows"]), bf16(inp["V_rows"])
+    idx = dev(np.tile(np.arange(10, dtype=np.int32), (4, 1)))
+    out = torch.empty((4, 128), dtype=torch.float32, device=DEV)
+    q = q_dev(inp)
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for stride in (127, 100, 0):   # below d, or not a multiple of 8
+        rc = F.lib().fathom_sparse_attend(ctypes.c_void_p(q.data_ptr()), F.BF16, ctypes.c_void_p(Kr.data_ptr()),
+                                          ctypes.c_void_p(Vr.data_ptr()), stride, 0, ctypes.c_void_p(idx.data_ptr()),
+                                          4, 1, 300, 128, 10, ctypes.c_void_p(out.data_ptr()), s)
+        assert rc == F.EINVAL, stride
 
 
 def test_sparse_attend_bad_index_flagged(ref):
