@@ -233,6 +233,26 @@ class Layer:
     LAUNCHES_PER_STEP = 1 + 1 + 9 + 1   # depths, scan, top-k (init, 3x hist+select, compact, finish), attention
 
 
+def profiled_traffic(resident, units):
+    """Bytes per scan launch from the committed ncu capture of this scan
+    kernel (profiles/scan_*), scaled to `units` keys x KV heads; None when
+    scan.cu has changed since that capture."""
+    import hashlib
+    name = "scan_host_n262144_traffic.md" if resident == "host" else "scan_hbm_n1M_B92.md"
+    path = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(path):
+        return None, None
+    rec = None
+    for line in open(path):
+        if line.startswith("traffic_json:"):
+            rec = json.loads(line.split(":", 1)[1])
+    src = os.path.join(ROOT, "bit_plane_key_b200", "csrc", "scan.cu")
+    if rec is None or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["kernel_src_sha256"]:
+        return None, None
+    return rec["bytes_per_unit"] * units, "%s from profiles/%s, scaled from %d to %d units" % (
+        rec["counter"], name, rec["captured_units"], units)
+
+
 def link_peak(F, torch, dev, nbytes=1 << 30, reps=10):
     """Host link bandwidth: pinned H2D copy and SM zero-copy read, best of `reps`, GB/s."""
     src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
@@ -410,14 +430,17 @@ def main():
     scan_bytes, U = layer.union_bytes()
     scan_ms = float(res["scan_ms"].mean())
     achieved = scan_bytes / (scan_ms * 1e-3) / 1e9
+    traffic, traffic_src = profiled_traffic(args.resident, args.n * layer.Hkv)
     if args.resident == "host":
         roof = {"bound": "host_link", "achieved": achieved, "peak": link["peak_gbs"], "unit": "GB/s",
-                "frac": achieved / link["peak_gbs"], "traffic": None,
+                "frac": achieved / link["peak_gbs"], "traffic": traffic, "traffic_source": traffic_src,
+                "algorithmic_bytes": scan_bytes,
                 "peak_source": "measured in this run: max(pinned H2D copy %.1f, SM zero-copy read %.1f) GB/s"
                                % (link["h2d_copy_gbs"], link["zero_copy_read_gbs"])}
     else:
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                "traffic": None, "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)"}
+                "traffic": traffic, "traffic_source": traffic_src, "algorithmic_bytes": scan_bytes,
+                "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)"}
 
     e2e_total, h2d, d2h = e2e_steps(torch, F, layer, args.budget, args.steps, args.warmup, flush)
     e2e_total = max_over_ranks(e2e_total)
