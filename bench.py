@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--budget", type=int, default=92)
     p.add_argument("--k", type=int, default=2048)
     p.add_argument("--n", type=int, default=1 << 20)
+    p.add_argument("--kv-groups", type=int, default=1,
+                   help="KV-head groups of the pipelined decode step (1 = depths, scan, top-k, attention in turn)")
     p.add_argument("--no-extras", action="store_true", help="skip the HBM-resident and fixed-r comparison runs")
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     p.add_argument("--kernel", default=None, choices=["scan"],
@@ -61,7 +63,10 @@ def workload_config(args, resident):
     return {"workload": "qwen3-8b layer, n=%d keys, 8 KV heads / 32 q heads, d=128, B=%d bits, k=%d, %s-resident "
                         "bit planes and K/V rows, 16 needles" % (args.n, args.budget, args.k, resident),
             "n": args.n, "n_kv_heads": 8, "n_q_heads": 32, "d": 128, "budget_bits": args.budget, "k": args.k,
-            "resident": resident, "l2": "flushed between steps (256 MB write)"}
+            "resident": resident, "kv_groups": args.kv_groups,
+            "step": "one fathom_decode_step call: depths, scan, top-k, attention, pipelined over kv_groups "
+                    "groups of KV heads",
+            "l2": "flushed between steps (256 MB write)"}
 
 
 # ----------------------------------------------------------------------------
@@ -201,6 +206,7 @@ class Layer:
         self.top = torch.empty((self.Hq, args.k), dtype=torch.float32, device=dev)
         self.out = torch.empty((self.Hq, self.d), dtype=torch.float32, device=dev)
         self.ws = torch.empty(F.topk_workspace_bytes(self.n, self.Hq, args.k), dtype=torch.uint8, device=dev)
+        self.dws = None
 
     def _pin(self, t):
         h = self.torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
@@ -224,13 +230,26 @@ class Layer:
         if ev:
             ev[4].record()
 
+    def step_pipelined(self, budget, fixed_r=0, groups=1):
+        """The same step as one fathom_decode_step call, pipelined over
+        `groups` groups of KV heads."""
+        need = self.F.decode_workspace_bytes(self.store, self.Hq, self.args.k, groups)
+        if self.dws is None or self.dws.numel() < need:
+            self.dws = self.torch.empty(need, dtype=self.torch.uint8, device=self.dev)
+        self.F.decode_step(self.store, self.q, self.s2, budget, self.args.k, self.K_rows, self.V_rows,
+                           fixed_r=fixed_r, kv_groups=groups, depths=self.depths, idx=self.idx,
+                           top_scores=self.top, out=self.out, workspace=self.dws)
+
     def union_bytes(self):
         """Plane + scale bytes the scan reads for the current depths (per launch)."""
         G = self.Hq // self.Hkv
         U = self.depths.view(self.Hkv, G, self.d).amax(dim=1)
         return self.store.plane_bytes_read(U), U
 
-    LAUNCHES_PER_STEP = 1 + 1 + 9 + 1   # depths, scan, top-k (init, 3x hist+select, compact, finish), attention
+    @staticmethod
+    def launches_per_step(groups):
+        # depths, then per group: scan, top-k (init, 3x hist+select, compact, finish), attention
+        return 1 + groups * (1 + 9 + 1)
 
 
 def profiled_traffic(resident, units):
@@ -309,7 +328,33 @@ def timed_steps(torch, layer, budget, steps, warmup, fixed_r, flush, clocks_gpu=
     return res
 
 
-def e2e_steps(torch, F, layer, budget, steps, warmup, flush):
+def timed_pipelined(torch, layer, budget, steps, warmup, fixed_r, flush, groups, clocks_gpu=None):
+    """The pipelined one-call step: CUDA events around each step on the
+    launching stream (the call joins its second stream back to it)."""
+    for _ in range(warmup):
+        layer.step_pipelined(budget, fixed_r, groups)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    sampler = ClockSampler(clocks_gpu) if clocks_gpu is not None else None
+    if sampler:
+        sampler.__enter__()
+    try:
+        for s in range(steps):
+            flush.zero_()
+            evs[s][0].record()
+            layer.step_pipelined(budget, fixed_r, groups)
+            evs[s][1].record()
+        torch.cuda.synchronize()
+    finally:
+        if sampler:
+            sampler.__exit__(None, None, None)
+    res = {"step_ms": np.array([e[0].elapsed_time(e[1]) for e in evs])}
+    if sampler:
+        res["clocks"] = sampler.summary()
+    return res
+
+
+def e2e_steps(torch, F, layer, budget, steps, warmup, flush, groups=1):
     """The same step through the public API with host buffers: q and sigma2
     copied in from page-locked memory and idx + output read back, every step."""
     q_h = torch.empty(layer.q.shape, dtype=layer.q.dtype, pin_memory=True)
@@ -324,7 +369,7 @@ def e2e_steps(torch, F, layer, budget, steps, warmup, flush):
     def one():
         layer.q.copy_(q_h, non_blocking=True)
         layer.s2.copy_(s2_h, non_blocking=True)
-        layer.step(budget)
+        layer.step_pipelined(budget, 0, groups)
         idx_h.copy_(layer.idx, non_blocking=True)
         out_h.copy_(layer.out, non_blocking=True)
 
@@ -418,11 +463,15 @@ def main():
         entry = visible.split(",")[gpu_index].strip()
         gpu_index = int(entry) if entry.isdigit() else entry
 
+    groups = args.kv_groups
     barrier()
-    res = timed_steps(torch, layer, args.budget, args.steps, args.warmup, 0, flush,
-                      clocks_gpu=gpu_index if rank == 0 else None)
+    pipe = timed_pipelined(torch, layer, args.budget, args.steps, args.warmup, 0, flush, groups,
+                           clocks_gpu=gpu_index if rank == 0 else None)
     barrier()
-    total_ms = max_over_ranks(float(res["step_ms"].sum()))
+    total_ms = max_over_ranks(float(pipe["step_ms"].sum()))
+    # the same step as separate launches, each kernel bracketed by CUDA events
+    # on the launch stream: the per-kernel breakdown and the scan's roofline
+    res = timed_steps(torch, layer, args.budget, args.steps, args.warmup, 0, flush)
     value, ms_per_step = throughput(args.n * layer.Hkv, world, total_ms, args.steps)
     keys_per_step = args.n * layer.Hkv * world
 
@@ -442,7 +491,7 @@ def main():
                 "traffic": traffic, "traffic_source": traffic_src, "algorithmic_bytes": scan_bytes,
                 "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)"}
 
-    e2e_total, h2d, d2h = e2e_steps(torch, F, layer, args.budget, args.steps, args.warmup, flush)
+    e2e_total, h2d, d2h = e2e_steps(torch, F, layer, args.budget, args.steps, args.warmup, flush, groups)
     e2e_total = max_over_ranks(e2e_total)
     e2e_value = keys_per_step * args.steps / (e2e_total * 1e-3) / 1e9
 
@@ -455,10 +504,13 @@ def main():
     if not args.no_extras:
         # same layer, other read policies: fixed 68-bit (r=16) and 136-bit (r=32) scans
         for name, fr in (("fixed68_r16", 16), ("fixed136_r32", 32)):
+            p2 = timed_pipelined(torch, layer, 0, args.steps, args.warmup, fr, flush, groups)
             r2 = timed_steps(torch, layer, 0, args.steps, args.warmup, fr, flush)
             b2, _ = layer.union_bytes()
-            extras[name] = {"ms_per_step": float(r2["step_ms"].mean()), "scan_ms": float(r2["scan_ms"].mean()),
-                            "gkeys_per_s": args.n * layer.Hkv / (float(r2["step_ms"].mean()) * 1e-3) / 1e9,
+            extras[name] = {"ms_per_step": float(p2["step_ms"].mean()),
+                            "sequential_ms_per_step": float(r2["step_ms"].mean()),
+                            "scan_ms": float(r2["scan_ms"].mean()),
+                            "gkeys_per_s": args.n * layer.Hkv / (float(p2["step_ms"].mean()) * 1e-3) / 1e9,
                             "scan_bytes_per_key_per_kv_head": b2 / (layer.n * layer.Hkv)}
         layer.step(args.budget)
         if args.resident == "host":
@@ -466,13 +518,15 @@ def main():
             hb = layer.dev_store
             keep = layer.store, layer.K_rows, layer.V_rows
             layer.store, layer.K_rows, layer.V_rows = hb, layer.inp["K_rows"], layer.inp["V_rows"]
+            p3 = timed_pipelined(torch, layer, args.budget, args.steps, args.warmup, 0, flush, groups)
             r3 = timed_steps(torch, layer, args.budget, args.steps, args.warmup, 0, flush)
             b3, _ = layer.union_bytes()
             s3 = float(r3["scan_ms"].mean())
             extras["hbm_resident"] = {
-                "ms_per_step": float(r3["step_ms"].mean()), "scan_ms": s3, "topk_ms": float(r3["topk_ms"].mean()),
-                "attend_ms": float(r3["attend_ms"].mean()),
-                "gkeys_per_s": args.n * layer.Hkv / (float(r3["step_ms"].mean()) * 1e-3) / 1e9,
+                "ms_per_step": float(p3["step_ms"].mean()), "sequential_ms_per_step": float(r3["step_ms"].mean()),
+                "scan_ms": s3, "topk_ms": float(r3["topk_ms"].mean()), "attend_ms": float(r3["attend_ms"].mean()),
+                "depths_ms": float(r3["depths_ms"].mean()),
+                "gkeys_per_s": args.n * layer.Hkv / (float(p3["step_ms"].mean()) * 1e-3) / 1e9,
                 "scan_gbs": b3 / (s3 * 1e-3) / 1e9, "scan_hbm_frac": b3 / (s3 * 1e-3) / 1e9 / hbm_peak}
             layer.store, layer.K_rows, layer.V_rows = keep
 
@@ -497,14 +551,18 @@ def main():
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded generator)",
                 "config": workload_config(args, args.resident),
                 "breakdown_ms": {k: float(res[k].mean()) for k in ("depths_ms", "scan_ms", "topk_ms", "attend_ms")},
+                "sequential_ms_per_step": float(res["step_ms"].mean()),
+                "breakdown_note": "breakdown_ms and the roofline come from a second timed region running the same "
+                                  "step as separate launches, each bracketed by CUDA events; value and "
+                                  "ms_per_step time the pipelined one-call step (fathom_decode_step)",
                 "scan_bytes_per_key_per_kv_head": scan_bytes / (layer.n * layer.Hkv),
                 "union_plane_bits_per_key_per_kv_head": float(U.sum()) / layer.Hkv,
-                "roofline": roof, "link": link, "clocks": res.get("clocks"),
+                "roofline": roof, "link": link, "clocks": pipe.get("clocks"),
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                         "note": "q and sigma2 copied in and idx + attention output read back every step; the "
                                 "bit planes and K/V rows stay in page-locked host memory and cross the link "
                                 "inside the scan and attention kernels"},
-                "gpu_launches": Layer.LAUNCHES_PER_STEP * args.steps,
+                "gpu_launches": Layer.launches_per_step(groups) * args.steps,
                 "needle_recall_head0": recall, "cpu_baseline": cpu, "compare": extras}
         print(json.dumps(line), flush=True)
     ranks.close()

@@ -281,6 +281,50 @@ int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, con
                                    (cudaStream_t)stream));
 }
 
+size_t fathom_decode_workspace_bytes(const fathom_store* store, int n_q_heads, int k, int kv_groups) {
+    if (!store || store->n < 1 || n_q_heads < 1 || k < 1 || k > kMaxTopK || kv_groups < 1 || kv_groups > 64 ||
+        store->n_kv_heads < 1 || store->n_kv_heads % kv_groups || n_q_heads % store->n_kv_heads)
+        return 0;
+    return decode_workspace_bytes(store->n, n_q_heads, kv_groups, k);
+}
+
+int fathom_decode_step(const fathom_store* store, const void* q, int q_dtype, const float* sigma2, int n_q_heads,
+                       int budget_bits, int fixed_r, int k, const uint16_t* K_rows, const uint16_t* V_rows,
+                       int64_t row_stride, int rows_host_resident, int kv_groups, uint8_t* depths, int32_t* idx,
+                       float* top_scores, float* out, void* workspace, size_t workspace_bytes,
+                       fathom_stream_t stream) {
+    const uint32_t* planes;
+    const uint16_t* scales;
+    int rc = resolve_store(store, &planes, &scales);
+    if (rc) return rc;
+    const int Hkv = store->n_kv_heads, d = store->d;
+    const int64_t n = store->n;
+    if (!q || !sigma2 || !depths || !idx || !out || !K_rows || !V_rows || !workspace) return FATHOM_EINVAL;
+    if (!heads_ok(n_q_heads, Hkv) || kv_groups < 1 || kv_groups > 64 || Hkv % kv_groups) return FATHOM_EINVAL;
+    if (q_dtype != FATHOM_F32 && q_dtype != FATHOM_BF16) return FATHOM_EINVAL;
+    if (budget_bits < 0 || fixed_r < 0 || fixed_r > d) return FATHOM_EINVAL;
+    if (k < 1 || k > n || k > kMaxTopK || n > INT32_MAX) return FATHOM_EINVAL;
+    if (d != 32 && d != 64 && d != 128 && d != 256) return FATHOM_EUNSUPPORTED;
+    if (row_stride < d || row_stride % 8) return FATHOM_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(K_rows) & 15) || (reinterpret_cast<uintptr_t>(V_rows) & 15) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return FATHOM_EINVAL;
+    if (workspace_bytes < decode_workspace_bytes(n, n_q_heads, kv_groups, k)) return FATHOM_ENOMEM;
+    if (!scan_fits(d, n_q_heads, Hkv)) return FATHOM_EUNSUPPORTED;
+    const void* kd = nullptr;
+    const void* vd = nullptr;
+    Where want = rows_host_resident ? Where::kHostPinned : Where::kDevice;
+    if (classify(K_rows, &kd) != want || classify(V_rows, &vd) != want) return FATHOM_EINVAL;
+    if (!is_device(q) || !is_device(sigma2) || !is_device(depths) || !is_device(idx) || !is_device(out) ||
+        !is_device(workspace) || (top_scores && !is_device(top_scores)))
+        return FATHOM_EINVAL;
+    if (!device_status_ptr()) return FATHOM_ECUDA;
+    return to_status(launch_decode(planes, scales, Hkv, d, n, store->n_pad, q, q_dtype, sigma2, n_q_heads,
+                                   budget_bits, fixed_r, k, static_cast<const uint16_t*>(kd),
+                                   static_cast<const uint16_t*>(vd), row_stride, rows_host_resident, kv_groups, depths,
+                                   idx, top_scores, out, workspace, (cudaStream_t)stream));
+}
+
 int fathom_last_device_status(fathom_stream_t stream) {
     unsigned int* p = device_status_ptr();
     if (!p) return -FATHOM_ECUDA;

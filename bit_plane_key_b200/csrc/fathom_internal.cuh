@@ -73,6 +73,12 @@ struct SessionMap {
 };
 cudaError_t launch_scan_batched(const SessionMap& map, int Hkv, int d, const void* q, int q_dtype,
                                 const uint8_t* depths, int Hq, float* scores, cudaStream_t stream);
+size_t decode_workspace_bytes(int64_t n, int Hq, int groups, int k);
+cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n, int64_t n_pad,
+                          const void* q, int q_dtype, const float* sigma2, int Hq, int budget, int fixed_r, int k,
+                          const uint16_t* K_rows, const uint16_t* V_rows, int64_t row_stride, int rows_host,
+                          int groups, uint8_t* depths, int32_t* idx, float* top_scores, float* out, void* workspace,
+                          cudaStream_t stream);
 cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
                           int64_t row_stride, const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k, int sort_rows, float* out,
                           cudaStream_t stream);

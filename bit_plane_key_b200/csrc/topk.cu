@@ -9,15 +9,18 @@
 // each row to the bin holding the k-th key: level 0 histograms bits 31..20,
 // level 1 bits 19..8 inside the chosen bin, level 2 bits 7..0; a row stops
 // refining as soon as its chosen bin holds at most kCap keys.  Keys above the
-// bin are certainly selected ("sure"), keys inside it are candidates.  A
-// final CTA per row bitonic-sorts sure + candidates as 64-bit composites
-// (key << 32 | ~index) and keeps the first k.  If even the exact 32-bit key
-// is shared by more than kCap keys (e.g. every score equal), the ties are
-// taken in index order by an ordered block scan instead, which keeps the
-// lower-index rule exact.
+// bin are certainly selected ("sure"), keys inside it are candidates, and one
+// pass over the row compacts both.  A final CTA per row finds the exact k-th
+// key among its candidates by the same radix steps in shared memory, keeps
+// the sure keys and the candidates at or above it, and bitonic-sorts them as
+// 64-bit composites (key << 32 | ~index): about k entries.  If even the exact
+// 32-bit key is shared by more than kCap keys (e.g. every score equal), the
+// ties are taken in index order by an ordered block scan instead, which keeps
+// the lower-index rule exact.
 //
-// Kernels: init, (hist, select) x 3 levels, compact, finish.  Rows already
-// resolved leave the later levels at once.
+// Kernels: init, (hist, select) x 3 levels, compact, finish.  Level 0 always
+// runs over every row; levels 1 and 2 run as small grid-stride launches that
+// leave at once when no row is still refining (the common case).
 #include "fathom_internal.cuh"
 
 namespace fathom {
@@ -29,6 +32,7 @@ constexpr int kChunk = 4096;        // elements per CTA in the row passes
 constexpr int kPassThreads = 256;
 constexpr int kFinishThreads = 1024;
 constexpr int kSortMax = 16384;     // >= next_pow2(kMaxTopK + kCap)
+constexpr int kPer = kChunk / kPassThreads;   // elements per thread in the row passes
 
 __constant__ int kLevelShift[3] = {20, 8, 0};
 __constant__ int kLevelBits[3] = {12, 12, 8};
@@ -46,6 +50,7 @@ struct RowState {
 
 struct Workspace {
     RowState* state;
+    int* active;         // [4]: rows still refining after select level l
     uint32_t* hist;      // [3][rows][kBins]
     uint64_t* sure;      // [rows][k]
     uint64_t* cand;      // [rows][kCap]
@@ -58,6 +63,8 @@ Workspace carve(void* ws, int rows, int k) {
     char* p = static_cast<char*>(ws);
     w.state = reinterpret_cast<RowState*>(p);
     p += align256(sizeof(RowState) * rows);
+    w.active = reinterpret_cast<int*>(p);
+    p += align256(sizeof(int) * 4);
     w.hist = reinterpret_cast<uint32_t*>(p);
     p += align256(sizeof(uint32_t) * 3 * (size_t)rows * kBins);
     w.sure = reinterpret_cast<uint64_t*>(p);
@@ -86,6 +93,7 @@ __global__ void topk_init(Workspace w, const __grid_constant__ RowMap m, int row
         h[(size_t)rows * kBins + b] = 0;
         h[2 * (size_t)rows * kBins + b] = 0;
     }
+    if (row == 0 && threadIdx.x < 4) w.active[threadIdx.x] = 0;
     if (threadIdx.x == 0) {
         RowState s;
         s.prefix = 0;
@@ -100,31 +108,58 @@ __global__ void topk_init(Workspace w, const __grid_constant__ RowMap m, int row
     }
 }
 
-__global__ void __launch_bounds__(kPassThreads)
-topk_hist(const float* __restrict__ scores, const __grid_constant__ RowMap m, int rows, Workspace w, int level) {
-    __shared__ uint32_t h[kBins];
-    const int row = blockIdx.y;
+// Histogram of one chunk of one row into the row's level histogram.
+__device__ __forceinline__ void hist_chunk(const float* __restrict__ scores, const RowMap& m, int rows, Workspace w,
+                                           int level, int row, int chunk, uint32_t* h) {
     const RowState st = w.state[row];
-    if (st.phase != 0) return;
+    if (st.phase != 0) return;   // uniform over the CTA
     int64_t off, n;
     row_span(m, row, &off, &n);
-    if ((int64_t)blockIdx.x * kChunk >= n) return;
-    for (int b = threadIdx.x; b < kBins; b += kPassThreads) h[b] = 0;
+    const int64_t i0 = (int64_t)chunk * kChunk;
+    if (i0 >= n) return;
+    const int nb = 1 << kLevelBits[level];
+    for (int b = threadIdx.x; b < nb; b += kPassThreads) h[b] = 0;
     __syncthreads();
     const int sh = kLevelShift[level];
-    const uint32_t mask = (1u << kLevelBits[level]) - 1u;
-    const int64_t i0 = (int64_t)blockIdx.x * kChunk;
+    const uint32_t mask = (uint32_t)nb - 1u;
     const int64_t i1 = min(n, i0 + kChunk);
     const float* s = scores + off;
-    for (int64_t i = i0 + threadIdx.x; i < i1; i += kPassThreads) {
-        uint32_t key = float_to_ordered(s[i]);
-        bool in = (st.shift == 32) || ((key >> st.shift) == st.prefix);
+    float v[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {   // all loads of the chunk in flight at once
+        const int64_t i = i0 + j * kPassThreads + threadIdx.x;
+        v[j] = (i < i1) ? s[i] : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int64_t i = i0 + j * kPassThreads + threadIdx.x;
+        const uint32_t key = float_to_ordered(v[j]);
+        const bool in = (i < i1) && ((st.shift == 32) || ((key >> st.shift) == st.prefix));
         if (in) atomicAdd(&h[(key >> sh) & mask], 1u);
     }
     __syncthreads();
     uint32_t* gh = w.hist + ((size_t)level * rows + row) * kBins;
-    for (int b = threadIdx.x; b < kBins; b += kPassThreads)
+    for (int b = threadIdx.x; b < nb; b += kPassThreads)
         if (h[b]) atomicAdd(&gh[b], h[b]);
+    __syncthreads();   // h is reused by the CTA's next chunk
+}
+
+// Level 0: every (chunk, row).
+__global__ void __launch_bounds__(kPassThreads)
+topk_hist(const float* __restrict__ scores, const __grid_constant__ RowMap m, int rows, Workspace w) {
+    __shared__ uint32_t h[kBins];
+    hist_chunk(scores, m, rows, w, 0, (int)blockIdx.y, (int)blockIdx.x, h);
+}
+
+// Levels 1 and 2: a grid-stride pass over (row, chunk) that leaves at once
+// when the previous select left no row refining.
+__global__ void __launch_bounds__(kPassThreads)
+topk_hist_refine(const float* __restrict__ scores, const __grid_constant__ RowMap m, int rows, int chunks,
+                 Workspace w, int level) {
+    __shared__ uint32_t h[kBins];
+    if (w.active[level - 1] == 0) return;
+    for (int64_t item = blockIdx.x; item < (int64_t)rows * chunks; item += gridDim.x)
+        hist_chunk(scores, m, rows, w, level, (int)(item / chunks), (int)(item % chunks), h);
 }
 
 // One CTA (1024 threads) per row: find the bin holding the need-th largest key.
@@ -174,6 +209,7 @@ topk_select(Workspace w, int rows, int k, int level) {
                 ns.shift = kLevelShift[level];
                 ns.phase = (c <= (uint32_t)kCap) ? 1 : (ns.shift == 0 ? 2 : 0);
                 w.state[row] = ns;
+                if (ns.phase == 0) atomicAdd(&w.active[level], 1);
                 break;
             }
             acc += c;
@@ -194,23 +230,30 @@ topk_compact(const float* __restrict__ scores, const __grid_constant__ RowMap m,
     const float* s = scores + off;
     const int lane = threadIdx.x & 31;
     RowState* gst = w.state + row;
-    for (int64_t base = i0; base < i1; base += kPassThreads) {
-        int64_t i = base + threadIdx.x;
-        uint32_t key = 0;
+    float v[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {   // all loads of the chunk in flight at once
+        const int64_t i = i0 + j * kPassThreads + threadIdx.x;
+        v[j] = (i < i1) ? s[i] : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int64_t i = i0 + j * kPassThreads + threadIdx.x;
+        const uint32_t key = float_to_ordered(v[j]);
         bool above = false, eq = false;
         if (i < i1) {
-            key = float_to_ordered(s[i]);
             if (st.shift == 32) {
                 eq = true;
             } else {
-                uint32_t hi = key >> st.shift;
+                const uint32_t hi = key >> st.shift;
                 above = hi > st.prefix;
                 eq = hi == st.prefix;
             }
         }
         const bool take_c = eq && st.phase == 1;
-        unsigned ma = __ballot_sync(0xffffffffu, above);
-        unsigned mc = __ballot_sync(0xffffffffu, take_c);
+        const unsigned ma = __ballot_sync(0xffffffffu, above);
+        const unsigned mc = __ballot_sync(0xffffffffu, take_c);
+        if (!(ma | mc)) continue;   // warp-uniform: nothing of this warp is kept
         int base_a = 0, base_c = 0;
         if (lane == 0) {
             if (ma) base_a = atomicAdd(&gst->n_sure, __popc(ma));
@@ -220,12 +263,12 @@ topk_compact(const float* __restrict__ scores, const __grid_constant__ RowMap m,
         base_c = __shfl_sync(0xffffffffu, base_c, 0);
         const unsigned lower = (1u << lane) - 1u;
         if (above) {
-            int slot = base_a + __popc(ma & lower);
+            const int slot = base_a + __popc(ma & lower);
             if (slot < k) w.sure[(size_t)row * k + slot] = composite(key, i);
             else atomicOr(status, (unsigned)FATHOM_DEV_TOPK_OVERFLOW);
         }
         if (take_c) {
-            int slot = base_c + __popc(mc & lower);
+            const int slot = base_c + __popc(mc & lower);
             if (slot < kCap) w.cand[(size_t)row * kCap + slot] = composite(key, i);
             else atomicOr(status, (unsigned)FATHOM_DEV_TOPK_OVERFLOW);
         }
@@ -250,12 +293,52 @@ __device__ void bitonic_desc(uint64_t* buf, int S) {
     }
 }
 
+// With hist[0..nb) filled, finds the bin b holding the need-th largest key
+// (bins ordered high to low): *above = keys in bins above b, *cnt = keys in b.
+// Called by every thread of a kFinishThreads block; all get the result.
+__device__ void block_pick_bin(const uint32_t* hist, int nb, uint32_t need, int* s_bin, uint32_t* s_above,
+                               uint32_t* s_cnt, uint32_t* warp_tot) {
+    const int t = threadIdx.x, lane = t & 31, wp = t >> 5;
+    const int per = nb / kFinishThreads > 0 ? nb / kFinishThreads : 1;   // bins per thread
+    uint32_t mine = 0;
+    if (per * t < nb)
+        for (int e = 0; e < per; ++e) mine += hist[per * t + e];
+    uint32_t v = mine;   // sum over this thread and the higher lanes of its warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, v, o);
+        if (31 - lane >= o) v += y;
+    }
+    if (lane == 0) warp_tot[wp] = v;
+    __syncthreads();
+    uint32_t higher = 0;
+    for (int x = wp + 1; x < kFinishThreads / 32; ++x) higher += warp_tot[x];
+    const uint32_t incl = v + higher, above = incl - mine;
+    if (above < need && incl >= need && per * t < nb) {
+        uint32_t acc = above;
+        for (int e = per - 1; e >= 0; --e) {
+            const uint32_t c = hist[per * t + e];
+            if (acc + c >= need) {
+                *s_bin = per * t + e;
+                *s_above = acc;
+                *s_cnt = c;
+                break;
+            }
+            acc += c;
+        }
+    }
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(kFinishThreads)
 topk_finish(const float* __restrict__ scores, const __grid_constant__ RowMap m, int k, Workspace w,
             int32_t* __restrict__ idx, float* __restrict__ top_scores, unsigned int* status) {
     extern __shared__ uint64_t buf[];
+    __shared__ uint32_t hist[kBins];
+    __shared__ uint32_t warp_tot[32];
     __shared__ int warp_cnt[32];
-    __shared__ int s_got;
+    __shared__ int s_got, s_bin, s_fill;
+    __shared__ uint32_t s_above, s_cnt;
     const int row = blockIdx.x;
     const RowState st = w.state[row];
     int64_t off, n;
@@ -263,10 +346,40 @@ topk_finish(const float* __restrict__ scores, const __grid_constant__ RowMap m, 
     const int ns = min(st.count_above, k);
     int total;
     if (st.phase == 1) {
+        // the exact k-th key T among the candidates, by radix steps over the
+        // bits the row passes left unresolved
         const int nc = min(st.cand, kCap);
-        total = ns + nc;
-        for (int e = threadIdx.x; e < ns; e += blockDim.x) buf[e] = w.sure[(size_t)row * k + e];
-        for (int e = threadIdx.x; e < nc; e += blockDim.x) buf[ns + e] = w.cand[(size_t)row * kCap + e];
+        const uint64_t* cand = w.cand + (size_t)row * kCap;
+        uint32_t need = (uint32_t)(k - ns);
+        uint32_t prefix = st.prefix;
+        int shift = st.shift;
+        while (shift > 0) {
+            const int nbits = shift >= 12 ? 12 : shift, sh = shift - nbits;
+            const int nb = 1 << nbits;
+            for (int b = threadIdx.x; b < nb; b += kFinishThreads) hist[b] = 0;
+            __syncthreads();
+            for (int e = threadIdx.x; e < nc; e += kFinishThreads) {
+                const uint32_t key = (uint32_t)(cand[e] >> 32);
+                if (shift == 32 || (key >> shift) == prefix) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1u);
+            }
+            __syncthreads();
+            block_pick_bin(hist, nb, need, &s_bin, &s_above, &s_cnt, warp_tot);
+            need -= s_above;
+            prefix = (shift == 32 ? 0u : (prefix << nbits)) | (uint32_t)s_bin;
+            shift = sh;
+            __syncthreads();   // s_bin / s_above are rewritten by the next step
+        }
+        const uint32_t T = prefix;
+        // keep the sure keys, the candidates above T and the candidates at T
+        for (int e = threadIdx.x; e < ns; e += kFinishThreads) buf[e] = w.sure[(size_t)row * k + e];
+        if (threadIdx.x == 0) s_fill = ns;
+        __syncthreads();
+        for (int e = threadIdx.x; e < nc; e += kFinishThreads) {
+            const uint64_t c = cand[e];
+            if ((uint32_t)(c >> 32) >= T) buf[atomicAdd(&s_fill, 1)] = c;
+        }
+        __syncthreads();
+        total = s_fill;
     } else {
         // ties at the exact threshold key: take the lowest indices, in order
         if (st.phase != 2) atomicOr(status, (unsigned)FATHOM_DEV_TOPK_OVERFLOW);
@@ -282,12 +395,12 @@ topk_finish(const float* __restrict__ scores, const __grid_constant__ RowMap m, 
             if (got >= r) break;
             int64_t i = base + threadIdx.x;
             bool f = (i < n) && float_to_ordered(s[i]) == T;
-            unsigned m = __ballot_sync(0xffffffffu, f);
-            if (lane == 0) warp_cnt[wp] = __popc(m);
+            unsigned msk = __ballot_sync(0xffffffffu, f);
+            if (lane == 0) warp_cnt[wp] = __popc(msk);
             __syncthreads();
             int before = 0;
             for (int x = 0; x < wp; ++x) before += warp_cnt[x];
-            int rank = got + before + __popc(m & ((1u << lane) - 1u));
+            int rank = got + before + __popc(msk & ((1u << lane) - 1u));
             if (f && rank < r) buf[ns + rank] = composite(T, i);
             __syncthreads();
             if (threadIdx.x == 0) {
@@ -315,7 +428,8 @@ topk_finish(const float* __restrict__ scores, const __grid_constant__ RowMap m, 
 
 size_t topk_workspace_bytes(int64_t n, int rows, int k) {
     (void)n;
-    return align256(sizeof(RowState) * rows) + align256(sizeof(uint32_t) * 3 * (size_t)rows * kBins) +
+    return align256(sizeof(RowState) * rows) + align256(sizeof(int) * 4) +
+           align256(sizeof(uint32_t) * 3 * (size_t)rows * kBins) +
            align256(sizeof(uint64_t) * (size_t)rows * k) + align256(sizeof(uint64_t) * (size_t)rows * kCap);
 }
 
@@ -325,8 +439,14 @@ cudaError_t launch_topk_map(const float* scores, const RowMap& map, int rows, in
     unsigned int* status = device_status_ptr();
     const unsigned chunks = (unsigned)((map.max_n + kChunk - 1) / kChunk);
     topk_init<<<rows, 256, 0, stream>>>(w, map, rows);
-    for (int level = 0; level < 3; ++level) {
-        topk_hist<<<dim3(chunks, rows), kPassThreads, 0, stream>>>(scores, map, rows, w, level);
+    topk_hist<<<dim3(chunks, rows), kPassThreads, 0, stream>>>(scores, map, rows, w);
+    topk_select<<<rows, 1024, 0, stream>>>(w, rows, k, 0);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long items = (long long)chunks * rows;
+    const unsigned refine_grid = (unsigned)(items < 4LL * sms ? items : 4LL * sms);
+    for (int level = 1; level < 3; ++level) {
+        topk_hist_refine<<<refine_grid, kPassThreads, 0, stream>>>(scores, map, rows, (int)chunks, w, level);
         topk_select<<<rows, 1024, 0, stream>>>(w, rows, k, level);
     }
     topk_compact<<<dim3(chunks, rows), kPassThreads, 0, stream>>>(scores, map, k, w, status);

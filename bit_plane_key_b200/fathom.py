@@ -67,6 +67,8 @@ _sig("fathom_noalloc_scratch_bytes", _Z, [])
 _sig("fathom_scan_batched_workspace_bytes", _Z, [_SP, _I, _I, _I])
 _sig("fathom_scan_topk_batched", _I, [_SP, _I, _P, _I, _P, _I, _I, _P, _P, _P, _Z, _P])
 _sig("fathom_scan_topk_noalloc", _I, [_SP, _P, _I, _P, _I, _I, _P, _P, _P])
+_sig("fathom_decode_workspace_bytes", _Z, [_SP, _I, _I, _I])
+_sig("fathom_decode_step", _I, [_SP, _P, _I, _P, _I, _I, _I, _I, _P, _P, _L, _I, _I, _P, _P, _P, _P, _P, _Z, _P])
 
 
 def lib():
@@ -283,3 +285,35 @@ def scan_topk_noalloc(store, q, depths, k, idx, top_scores=None, stream=None):
     _check(_lib.fathom_scan_topk_noalloc(store.c, _ptr(q), _dtype_code(q), _ptr(depths), q.shape[0], int(k),
                                          _ptr(idx), _ptr(top_scores), _stream(stream)), "fathom_scan_topk_noalloc")
     return idx, top_scores
+
+
+def decode_workspace_bytes(store, n_q_heads, k, kv_groups):
+    return int(_lib.fathom_decode_workspace_bytes(store.c, int(n_q_heads), int(k), int(kv_groups)))
+
+
+def decode_step(store, q, sigma2, budget_bits, k, K_rows, V_rows, fixed_r=0, kv_groups=1, depths=None, idx=None,
+                top_scores=None, out=None, workspace=None, stream=None, want_top_scores=True):
+    """One decode step (depths, scan, top-k, attention) in one C-ABI call,
+    pipelined over kv_groups groups of KV heads.  Returns (depths, idx,
+    top_scores or None, out)."""
+    Hq, d = q.shape
+    dev = q.device
+    if K_rows.stride() != V_rows.stride() or K_rows.stride(2) != 1 or K_rows.stride(0) != store.n * K_rows.stride(1):
+        raise ValueError("K_rows and V_rows need strides (n*s, s, 1), the same for both")
+    if depths is None:
+        depths = torch.empty((Hq, d), dtype=torch.uint8, device=dev)
+    if idx is None:
+        idx = torch.empty((Hq, k), dtype=torch.int32, device=dev)
+    if top_scores is None and want_top_scores:
+        top_scores = torch.empty((Hq, k), dtype=torch.float32, device=dev)
+    if out is None:
+        out = torch.empty((Hq, d), dtype=torch.float32, device=dev)
+    need = decode_workspace_bytes(store, Hq, k, kv_groups)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check(_lib.fathom_decode_step(store.c, _ptr(q), _dtype_code(q), _ptr(sigma2), Hq, int(budget_bits), int(fixed_r),
+                                   int(k), _ptr(K_rows), _ptr(V_rows), int(K_rows.stride(1)),
+                                   int(not K_rows.is_cuda), int(kv_groups), _ptr(depths), _ptr(idx),
+                                   _ptr(top_scores), _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "fathom_decode_step")
+    return depths, idx, top_scores, out

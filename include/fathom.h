@@ -256,6 +256,41 @@ int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, con
                          int n_kv_heads, int64_t n, int d, int k, float* out, fathom_stream_t stream);
 
 /*
+ * One decode step of one layer in one call: per-query depths, the scan, top-k
+ * and exact attention over the selected rows.  [ai-feeds summary 方法: 输入,
+ * 关键模块 2-5, 输出]  The results equal fathom_alloc_depths, then
+ * fathom_scan_topk, then fathom_sparse_attend on the same arguments, bit for
+ * bit.
+ *
+ * The KV heads are split into kv_groups groups of equal size.  The scan of a
+ * group runs on `stream` while the top-k and attention of the previous group
+ * run on an auxiliary stream that the library creates per device on first
+ * use; the two are forked and joined with events, so all work is ordered on
+ * `stream` and the call may be captured into a CUDA graph.  kv_groups = 1
+ * runs the plain sequence.  Steps issued at the same time from several host
+ * threads on one device share the auxiliary stream (they stay correct; their
+ * top-k and attention serialise).
+ *   store        device- or host-resident store, as fathom_scan_topk.
+ *   q, q_dtype, sigma2, budget_bits, fixed_r  as fathom_alloc_depths.
+ *   k            as fathom_scan_topk (1 <= k <= min(n, 4096)).
+ *   K_rows, V_rows, row_stride, rows_host_resident  as fathom_sparse_attend.
+ *   kv_groups    1 <= kv_groups <= 64, dividing the store's n_kv_heads.
+ *   depths       device, u8 [Hq][d], written.
+ *   idx          device, i32 [Hq][k]; top_scores device f32 [Hq][k] or NULL.
+ *   out          device, f32 [Hq][d].
+ *   workspace    device, 256-byte aligned, at least
+ *                fathom_decode_workspace_bytes(store, Hq, k, kv_groups) bytes
+ *                (the scores of all heads and one top-k workspace).
+ * Errors: as the three separate calls; EINVAL for a bad kv_groups.
+ */
+size_t fathom_decode_workspace_bytes(const fathom_store* store, int n_q_heads, int k, int kv_groups);
+int fathom_decode_step(const fathom_store* store, const void* q, int q_dtype, const float* sigma2, int n_q_heads,
+                       int budget_bits, int fixed_r, int k, const uint16_t* K_rows, const uint16_t* V_rows,
+                       int64_t row_stride, int rows_host_resident, int kv_groups, uint8_t* depths, int32_t* idx,
+                       float* top_scores, float* out, void* workspace, size_t workspace_bytes,
+                       fathom_stream_t stream);
+
+/*
  * Reads and clears this device's status word (FATHOM_DEV_* bits) after
  * synchronising `stream`.  Returns the bits (>= 0), or -FATHOM_ECUDA.
  */

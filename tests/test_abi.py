@@ -28,7 +28,8 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for must in ("fathom_pack_bitplanes", "fathom_alloc_depths", "fathom_scan_topk", "fathom_sparse_attend",
                  "fathom_scan_scores", "fathom_topk", "fathom_planes_bytes", "fathom_scales_bytes",
-                 "fathom_scan_workspace_bytes", "fathom_last_device_status"):
+                 "fathom_scan_workspace_bytes", "fathom_last_device_status", "fathom_decode_step",
+                 "fathom_decode_workspace_bytes"):
         assert must in names
 
 
@@ -64,3 +65,17 @@ def test_null_arguments_rejected_before_any_cuda_call(libpath):
     assert L.fathom_topk(None, 10, 10, 1, 1, None, None, None, 0, None) == F.EINVAL
     assert L.fathom_scan_topk(None, None, 0, None, 1, 1, None, None, None, 0, None) == F.EINVAL
     assert L.fathom_sparse_attend(None, 0, None, None, 128, 0, None, 1, 1, 10, 128, 1, None, None) == F.EINVAL
+    assert L.fathom_decode_step(None, None, 0, None, 4, 92, 0, 16, None, None, 128, 0, 1, None, None, None, None,
+                                None, 0, None) == F.EINVAL
+
+
+def test_decode_workspace_sizes(libpath):
+    from bit_plane_key_b200 import fathom as F
+    st = F.fathom_store(8, 128, 1 << 20, F.n_pad(1 << 20), 1, 0, None, None)
+    one = F.lib().fathom_decode_workspace_bytes(ctypes.byref(st), 32, 2048, 1)
+    four = F.lib().fathom_decode_workspace_bytes(ctypes.byref(st), 32, 2048, 4)
+    assert one >= 4 * 32 * F.n_pad(1 << 20) and four >= 4 * 32 * F.n_pad(1 << 20)
+    assert four < one            # one top-k workspace, sized for a group's rows
+    assert F.lib().fathom_decode_workspace_bytes(ctypes.byref(st), 32, 2048, 3) == 0    # 3 does not divide 8
+    assert F.lib().fathom_decode_workspace_bytes(ctypes.byref(st), 32, 5000, 1) == 0    # k above the maximum
+    assert F.lib().fathom_decode_workspace_bytes(ctypes.byref(st), 30, 2048, 1) == 0    # Hq not a multiple of Hkv
