@@ -108,7 +108,53 @@ __global__ void topk_init(Workspace w, const __grid_constant__ RowMap m, int row
     }
 }
 
+// The kPer elements of a row chunk that thread t handles, all loads in
+// flight at once: with 16-byte aligned rows, four float4 loads (element
+// (q, e) at i0 + 4 (q * kPassThreads + t) + e), else kPer scalar loads
+// (element j at i0 + j * kPassThreads + t).  Out-of-range elements read 0.
+template <bool kVec>
+__device__ __forceinline__ int64_t chunk_index(int64_t i0, int j) {
+    return kVec ? i0 + 4 * ((int64_t)(j >> 2) * kPassThreads + threadIdx.x) + (j & 3)
+                : i0 + (int64_t)j * kPassThreads + threadIdx.x;
+}
+template <bool kVec>
+__device__ __forceinline__ void load_chunk(const float* __restrict__ s, int64_t i0, int64_t i1, float (&v)[kPer]) {
+    if constexpr (kVec) {
+#pragma unroll
+        for (int qd = 0; qd < kPer / 4; ++qd) {
+            const int64_t b = chunk_index<true>(i0, 4 * qd);
+            if (b + 3 < i1) {
+                const float4 x = *reinterpret_cast<const float4*>(s + b);
+                v[4 * qd] = x.x; v[4 * qd + 1] = x.y; v[4 * qd + 2] = x.z; v[4 * qd + 3] = x.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) v[4 * qd + e] = (b + e < i1) ? s[b + e] : 0.0f;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int64_t i = chunk_index<false>(i0, j);
+            v[j] = (i < i1) ? s[i] : 0.0f;
+        }
+    }
+}
+
 // Histogram of one chunk of one row into the row's level histogram.
+template <bool kVec>
+__device__ __forceinline__ void hist_body(const float* __restrict__ s, int64_t i0, int64_t i1, RowState st, int sh,
+                                          uint32_t mask, uint32_t* h) {
+    float v[kPer];
+    load_chunk<kVec>(s, i0, i1, v);
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int64_t i = chunk_index<kVec>(i0, j);
+        const uint32_t key = float_to_ordered(v[j]);
+        const bool in = (i < i1) && ((st.shift == 32) || ((key >> st.shift) == st.prefix));
+        if (in) atomicAdd(&h[(key >> sh) & mask], 1u);
+    }
+}
+
 __device__ __forceinline__ void hist_chunk(const float* __restrict__ scores, const RowMap& m, int rows, Workspace w,
                                            int level, int row, int chunk, uint32_t* h) {
     const RowState st = w.state[row];
@@ -124,19 +170,8 @@ __device__ __forceinline__ void hist_chunk(const float* __restrict__ scores, con
     const uint32_t mask = (uint32_t)nb - 1u;
     const int64_t i1 = min(n, i0 + kChunk);
     const float* s = scores + off;
-    float v[kPer];
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {   // all loads of the chunk in flight at once
-        const int64_t i = i0 + j * kPassThreads + threadIdx.x;
-        v[j] = (i < i1) ? s[i] : 0.0f;
-    }
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-        const int64_t i = i0 + j * kPassThreads + threadIdx.x;
-        const uint32_t key = float_to_ordered(v[j]);
-        const bool in = (i < i1) && ((st.shift == 32) || ((key >> st.shift) == st.prefix));
-        if (in) atomicAdd(&h[(key >> sh) & mask], 1u);
-    }
+    if ((reinterpret_cast<uintptr_t>(s + i0) & 15) == 0) hist_body<true>(s, i0, i1, st, sh, mask, h);
+    else hist_body<false>(s, i0, i1, st, sh, mask, h);
     __syncthreads();
     uint32_t* gh = w.hist + ((size_t)level * rows + row) * kBins;
     for (int b = threadIdx.x; b < nb; b += kPassThreads)
@@ -217,28 +252,24 @@ topk_select(Workspace w, int rows, int k, int level) {
     }
 }
 
-__global__ void __launch_bounds__(kPassThreads)
-topk_compact(const float* __restrict__ scores, const __grid_constant__ RowMap m, int k, Workspace w,
-             unsigned int* status) {
-    const int row = blockIdx.y;
-    const RowState st = w.state[row];
-    int64_t off, n;
-    row_span(m, row, &off, &n);
-    const int64_t i0 = (int64_t)blockIdx.x * kChunk;
-    if (i0 >= n) return;
-    const int64_t i1 = min(n, i0 + kChunk);
-    const float* s = scores + off;
-    const int lane = threadIdx.x & 31;
-    RowState* gst = w.state + row;
+// Keys above the row's bin go to the sure buffer, keys inside it to the
+// candidates.  A CTA counts its keepers, reserves its output ranges with one
+// atomic per buffer, then writes them: no warp waits on a contended counter.
+// The write pass reloads only the kept keys.
+template <bool kVec>
+__device__ __forceinline__ void compact_body(const float* __restrict__ s, int64_t i0, int64_t i1, RowState st, int row,
+                                             int k, Workspace w, unsigned int* status) {
+    constexpr int kWarpsPerCta = kPassThreads / 32;
+    __shared__ int s_na[kWarpsPerCta], s_nc[kWarpsPerCta];
+    __shared__ int s_base_a, s_base_c;
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     float v[kPer];
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {   // all loads of the chunk in flight at once
-        const int64_t i = i0 + j * kPassThreads + threadIdx.x;
-        v[j] = (i < i1) ? s[i] : 0.0f;
-    }
+    load_chunk<kVec>(s, i0, i1, v);
+    // classify: bit j of fa / fc = element j is sure / a candidate
+    uint32_t fa = 0, fc = 0;
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
-        const int64_t i = i0 + j * kPassThreads + threadIdx.x;
+        const int64_t i = chunk_index<kVec>(i0, j);
         const uint32_t key = float_to_ordered(v[j]);
         bool above = false, eq = false;
         if (i < i1) {
@@ -250,31 +281,77 @@ topk_compact(const float* __restrict__ scores, const __grid_constant__ RowMap m,
                 eq = hi == st.prefix;
             }
         }
-        const bool take_c = eq && st.phase == 1;
+        fa |= (above ? 1u : 0u) << j;
+        fc |= ((eq && st.phase == 1) ? 1u : 0u) << j;
+    }
+    const int na = (int)__reduce_add_sync(0xffffffffu, (unsigned)__popc(fa));   // this warp's keepers
+    const int nc = (int)__reduce_add_sync(0xffffffffu, (unsigned)__popc(fc));
+    if (lane == 0) {
+        s_na[wp] = na;
+        s_nc[wp] = nc;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int ta = 0, tc = 0;
+        for (int x = 0; x < kWarpsPerCta; ++x) {
+            ta += s_na[x];
+            tc += s_nc[x];
+        }
+        RowState* gst = w.state + row;
+        s_base_a = ta ? atomicAdd(&gst->n_sure, ta) : 0;
+        s_base_c = tc ? atomicAdd(&gst->n_cand, tc) : 0;
+    }
+    __syncthreads();
+    if (na + nc == 0) return;   // warp-uniform
+    int pa = s_base_a, pc = s_base_c;
+    for (int x = 0; x < wp; ++x) {
+        pa += s_na[x];
+        pc += s_nc[x];
+    }
+    const unsigned lower = (1u << lane) - 1u;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const bool above = (fa >> j) & 1u, take_c = (fc >> j) & 1u;
         const unsigned ma = __ballot_sync(0xffffffffu, above);
         const unsigned mc = __ballot_sync(0xffffffffu, take_c);
-        if (!(ma | mc)) continue;   // warp-uniform: nothing of this warp is kept
-        int base_a = 0, base_c = 0;
-        if (lane == 0) {
-            if (ma) base_a = atomicAdd(&gst->n_sure, __popc(ma));
-            if (mc) base_c = atomicAdd(&gst->n_cand, __popc(mc));
-        }
-        base_a = __shfl_sync(0xffffffffu, base_a, 0);
-        base_c = __shfl_sync(0xffffffffu, base_c, 0);
-        const unsigned lower = (1u << lane) - 1u;
+        if (!(ma | mc)) continue;   // warp-uniform
+        const int64_t i = chunk_index<kVec>(i0, j);
+        const uint32_t key = (above || take_c) ? float_to_ordered(s[i]) : 0u;
         if (above) {
-            const int slot = base_a + __popc(ma & lower);
+            const int slot = pa + __popc(ma & lower);
             if (slot < k) w.sure[(size_t)row * k + slot] = composite(key, i);
             else atomicOr(status, (unsigned)FATHOM_DEV_TOPK_OVERFLOW);
         }
         if (take_c) {
-            const int slot = base_c + __popc(mc & lower);
+            const int slot = pc + __popc(mc & lower);
             if (slot < kCap) w.cand[(size_t)row * kCap + slot] = composite(key, i);
             else atomicOr(status, (unsigned)FATHOM_DEV_TOPK_OVERFLOW);
         }
+        pa += __popc(ma);
+        pc += __popc(mc);
     }
 }
 
+__global__ void __launch_bounds__(kPassThreads)
+topk_compact(const float* __restrict__ scores, const __grid_constant__ RowMap m, int k, Workspace w,
+             unsigned int* status) {
+    const int row = blockIdx.y;
+    const RowState st = w.state[row];
+    int64_t off, n;
+    row_span(m, row, &off, &n);
+    const int64_t i0 = (int64_t)blockIdx.x * kChunk;
+    if (i0 >= n) return;
+    const int64_t i1 = min(n, i0 + kChunk);
+    const float* s = scores + off;
+    if ((reinterpret_cast<uintptr_t>(s + i0) & 15) == 0) compact_body<true>(s, i0, i1, st, row, k, w, status);
+    else compact_body<false>(s, i0, i1, st, row, k, w, status);
+}
+
+// Bitonic sort, descending, of buf[0..S), S a power of two.  Thread t
+// compares elements i = 2t - t % stride and i + stride, so while stride <= 32
+// a warp touches only its own 64-element ranges and a warp barrier suffices
+// between two such stages; the block barrier is taken before and after every
+// stage that crosses warps.
 __device__ void bitonic_desc(uint64_t* buf, int S) {
     for (int size = 2; size <= S; size <<= 1) {
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
@@ -288,7 +365,11 @@ __device__ void bitonic_desc(uint64_t* buf, int S) {
                     buf[j] = a;
                 }
             }
-            __syncthreads();
+            // a stage that crosses warps (stride > 32) needs the block barrier
+            // after it, and so does the stage before one
+            const int next = stride > 1 ? stride >> 1 : size;   // stride of the next stage
+            if (stride > 32 || next > 32 || (stride == 1 && size == S)) __syncthreads();
+            else __syncwarp();
         }
     }
 }

@@ -266,6 +266,28 @@ def test_topk_bit_exact(ref, n, rows, k, kind):
     assert F.last_device_status() == 0
 
 
+@pytest.mark.parametrize("kind", ["normal", "ties", "narrow"])
+def test_topk_repeatable_under_load(ref, kind):
+    """The same rows, 20 launches back to back with many rows in flight: every
+    launch must give the oracle's exact answer (a race in the selection or the
+    final sort shows up as a launch that differs)."""
+    rng = np.random.default_rng(7)
+    rows, n, k = 32, 65536, 2048
+    if kind == "normal":
+        s = rng.standard_normal((rows, n)).astype(np.float32)
+    elif kind == "ties":
+        s = np.round(rng.standard_normal((rows, n)), 1).astype(np.float32)
+    else:
+        s = (1.0 + rng.random((rows, n)) * 1e-3).astype(np.float32)
+    sd = dev(s)
+    ws = torch.empty(F.topk_workspace_bytes(n, rows, k), dtype=torch.uint8, device=DEV)
+    outs = [F.topk(sd, n, k, workspace=ws) for _ in range(20)]
+    want = np.stack([ref.topk(s[r], k) for r in range(rows)])
+    for idx, top in outs:
+        assert np.array_equal(host(idx), want)
+    assert F.last_device_status() == 0
+
+
 # --------------------------------------------------------------------------
 # a4 + a5 against the fp64 oracle
 # --------------------------------------------------------------------------
