@@ -34,32 +34,35 @@ constexpr int kUnroll = 8;     // rows in flight per warp
 constexpr int kSortCap = kMaxTopK;   // indices sorted in shared memory
 
 
+// A lane's V bf16 values of a row, kept as raw 32-bit words until used: the
+// loads of all rows in flight are issued before any value is converted.
 template <int V>
-__device__ __forceinline__ void load_row(const uint16_t* __restrict__ p, float* out) {
-    // V consecutive bf16 values
-    if constexpr (V == 4) {
-        uint2 u = *reinterpret_cast<const uint2*>(p);
-        out[0] = __uint_as_float(u.x << 16);
-        out[1] = __uint_as_float(u.x & 0xFFFF0000u);
-        out[2] = __uint_as_float(u.y << 16);
-        out[3] = __uint_as_float(u.y & 0xFFFF0000u);
-    } else if constexpr (V == 8) {
-        uint4 u = *reinterpret_cast<const uint4*>(p);
-        uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            out[2 * e] = __uint_as_float(w[e] << 16);
-            out[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+struct RowWords {
+    static constexpr int W = (V + 1) / 2;
+    uint32_t w[W];
+    __device__ __forceinline__ void load(const uint16_t* __restrict__ p) {
+        if constexpr (V == 8) {
+            const uint4 u = *reinterpret_cast<const uint4*>(p);
+            w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+        } else if constexpr (V == 4) {
+            const uint2 u = *reinterpret_cast<const uint2*>(p);
+            w[0] = u.x; w[1] = u.y;
+        } else if constexpr (V == 2) {
+            w[0] = *reinterpret_cast<const uint32_t*>(p);
+        } else {
+            w[0] = p[0];
         }
-    } else if constexpr (V == 2) {
-        uint32_t u = *reinterpret_cast<const uint32_t*>(p);
-        out[0] = __uint_as_float(u << 16);
-        out[1] = __uint_as_float(u & 0xFFFF0000u);
-    } else {
-#pragma unroll
-        for (int e = 0; e < V; ++e) out[e] = __uint_as_float((uint32_t)p[e] << 16);
     }
-}
+    __device__ __forceinline__ void clear() {
+#pragma unroll
+        for (int e = 0; e < W; ++e) w[e] = 0u;
+    }
+    __device__ __forceinline__ float at(int e) const {   // value e (bf16 -> f32 is a shift)
+        const uint32_t x = w[e >> 1];
+        return (V == 1) ? __uint_as_float(x << 16) : ((e & 1) ? __uint_as_float(x & 0xFFFF0000u)
+                                                              : __uint_as_float(x << 16));
+    }
+};
 
 template <int V>
 __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kThreads)
@@ -116,19 +119,21 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
     // so the head's 32 warps sweep the list together, in address order when sorted
     const int stride = kSplit * kWarps;
     for (int p0 = r + kSplit * wp; p0 < k; p0 += stride * kUnroll) {
-        float kv[kUnroll][V], vv[kUnroll][V];
+        RowWords<V> kw[kUnroll], vw[kUnroll];
         bool ok[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int p = p0 + u * stride;
             ok[u] = false;
+            kw[u].clear();
+            vw[u].clear();
             if (p < k) {
                 const int64_t i = ih[p];
                 if (i >= 0 && i < n) {
                     ok[u] = true;
                     const int64_t off = head_base + i * row_stride + lane * V;
-                    load_row<V>(Kr + off, kv[u]);
-                    load_row<V>(Vr + off, vv[u]);
+                    kw[u].load(Kr + off);
+                    vw[u].load(Vr + off);
                 } else if (lane == 0) {
                     atomicOr(status, (unsigned)FATHOM_DEV_BAD_INDEX);
                 }
@@ -138,7 +143,7 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
         for (int u = 0; u < kUnroll; ++u) {
             float dot = 0.0f;
 #pragma unroll
-            for (int e = 0; e < V; ++e) dot = fmaf(qv[e], kv[u][e], dot);
+            for (int e = 0; e < V; ++e) dot = fmaf(qv[e], kw[u].at(e), dot);
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
             if (!ok[u]) continue;   // warp-uniform
@@ -147,7 +152,7 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
             float p = exp2f(dot - mn);
             l = l * a + p;
 #pragma unroll
-            for (int e = 0; e < V; ++e) o[e] = fmaf(p, vv[u][e], o[e] * a);
+            for (int e = 0; e < V; ++e) o[e] = fmaf(p, vw[u].at(e), o[e] * a);
             m = mn;
         }
     }
