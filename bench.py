@@ -54,6 +54,8 @@ def parse():
                    help="KV-head groups of the pipelined decode step (1 = depths, scan, top-k, attention in turn)")
     p.add_argument("--no-extras", action="store_true", help="skip the HBM-resident and fixed-r comparison runs")
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    p.add_argument("--config", type=int, default=None, choices=[1, 2, 4, 5],
+                   help="measure another workload of the method (one JSON line per case; not the headline)")
     p.add_argument("--kernel", default=None, choices=["scan"],
                    help="time one kernel alone on this workload (a kernel benchmark, not the step metric)")
     return p.parse_args()
@@ -432,8 +434,161 @@ def kernel_bench(args):
                       "hbm_frac": gbs / hbm if args.resident == "hbm" else None}), flush=True)
 
 
+def _events_ms(torch, fn, steps, warmup, flush=None):
+    """Per-call device times (ms) of fn() with CUDA events on the current stream."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        if flush is not None:
+            flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return np.array(ts)
+
+
+def config_bench(args):
+    """The pages' other workloads, each timed through the one-call decode step
+    or the batched entry point (one JSON line per case):
+      1: one head, n = 4096, B = 64, k = 64, fp32 q, HBM: decode-step latency.
+      2: 8/32 heads, n = 131072, B in {46, 68, 92, 136} and fixed68/136, HBM.
+      4: 16 sessions, n ~ U[64k, 512k], host-resident, B = 68, k = 1024: one
+         batched scan + top-k.
+      5: 36 layers, n = 2^20, host-resident, B ~ U[46, 136]: one decode token
+         (all layers' steps); the layers share one K/V row buffer."""
+    import torch
+    import synth
+    import oracle
+    from bit_plane_key_b200 import fathom as F
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = []
+    if args.config in (1, 2):
+        cfg = synth.CONFIGS[args.config]
+        inp = synth.layer_inputs_cuda(args.config, device=dev)
+        Hkv, Hq, n, k = cfg["n_kv_heads"], cfg["n_q_heads"], cfg["n"], cfg["k"]
+        st = F.pack_bitplanes(inp["K"])
+        Kr, Vr = inp["K_rows"], inp["V_rows"]
+        ws = torch.empty(F.decode_workspace_bytes(st, Hq, k, 1), dtype=torch.uint8, device=dev)
+        bufs = dict(depths=torch.empty((Hq, 128), dtype=torch.uint8, device=dev),
+                    idx=torch.empty((Hq, k), dtype=torch.int32, device=dev),
+                    top_scores=torch.empty((Hq, k), dtype=torch.float32, device=dev),
+                    out=torch.empty((Hq, 128), dtype=torch.float32, device=dev), workspace=ws)
+        cases = [("B=%d" % b, b, 0) for b in cfg["budgets"]]
+        if args.config == 2:
+            cases += [("fixed68_r16", 0, 16), ("fixed136_r32", 0, 32)]
+        for name, b, fr in cases:
+            step = lambda: F.decode_step(st, inp["q_dev"], inp["sigma2_dev"], b, k, Kr, Vr, fixed_r=fr, **bufs)
+            t_flush = _events_ms(torch, step, args.steps, args.warmup, flush)
+            t_warm = _events_ms(torch, step, args.steps, args.warmup)
+            dep = F.alloc_depths(inp["q_dev"], inp["sigma2_dev"], b, fixed_r=fr)
+            scan = _events_ms(torch, lambda: F.scan_scores(st, inp["q_dev"], dep), args.steps, args.warmup, flush)
+            U = dep.view(Hkv, Hq // Hkv, 128).amax(dim=1)
+            nbytes = st.plane_bytes_read(U)
+            # the oracle on one KV group over all n keys (single thread)
+            g0 = 0
+            planes = st.planes[g0:g0 + 1].cpu().numpy().view(np.uint32)
+            scales = st.scales[g0:g0 + 1].cpu().numpy().view(np.uint16)
+            G = Hq // Hkv
+            qg = inp["q"][:G]
+            s2g = inp["sigma2"][g0:g0 + 1]
+            Krg = Kr[g0:g0 + 1].cpu().view(torch.int16).numpy().view(np.uint16)
+            Vrg = Vr[g0:g0 + 1].cpu().view(torch.int16).numpy().view(np.uint16)
+            t0 = time.perf_counter()
+            if fr:
+                oracle.decode(planes, scales, n, qg, s2g, 0, k, K_rows=Krg, V_rows=Vrg, fixed_r=fr)
+            else:
+                oracle.decode(planes, scales, n, qg, s2g, b, k, K_rows=Krg, V_rows=Vrg)
+            t_or = time.perf_counter() - t0
+            out.append({"config": args.config, "case": name, "workload": cfg["name"], "n": n, "n_kv_heads": Hkv,
+                        "n_q_heads": Hq, "k": k, "step_us_l2_flushed": float(np.median(t_flush)) * 1e3,
+                        "step_us_warm": float(np.median(t_warm)) * 1e3,
+                        "scan_us": float(np.median(scan)) * 1e3,
+                        "gkeys_per_s_step": n * Hkv / (float(np.median(t_flush)) * 1e-3) / 1e9,
+                        "scan_bytes_per_key_per_kv_head": nbytes / (n * Hkv),
+                        "scan_hbm_gbs": nbytes / (float(np.median(scan)) * 1e-3) / 1e9,
+                        "oracle_s_one_kv_group": t_or, "oracle_cores": 1,
+                        "gpu_vs_oracle_per_kv_group": t_or / (float(np.median(t_flush)) * 1e-3 / Hkv)})
+    elif args.config == 4:
+        cfg = synth.CONFIGS[4]
+        rng = synth.rng_for(4, 0, 9)
+        lengths = (rng.integers(cfg["n_lo"] // 64, cfg["n_hi"] // 64 + 1, cfg["sessions"]) * 64).tolist()
+        stores, qs, s2s = [], [], []
+        for sidx, n in enumerate(lengths):
+            inp = synth.layer_inputs_cuda(4, layer=sidx, n=n, device=dev, with_values=False)
+            stores.append(F.pack_bitplanes(inp["K"]).to_host())
+            qs.append(inp["q_dev"])
+            s2s.append(inp["sigma2_dev"])
+            del inp
+            torch.cuda.empty_cache()
+        q = torch.stack(qs)
+        s2 = torch.cat(s2s)
+        S, Hq, k, B = len(lengths), 32, cfg["k"], cfg["budgets"][0]
+        dep = torch.empty((S * Hq, 128), dtype=torch.uint8, device=dev)
+        ws = torch.empty(F.scan_batched_workspace_bytes(stores, Hq, k), dtype=torch.uint8, device=dev)
+        idx = torch.empty((S, Hq, k), dtype=torch.int32, device=dev)
+        top = torch.empty((S, Hq, k), dtype=torch.float32, device=dev)
+
+        def step():
+            F.alloc_depths(q.view(-1, 128), s2, B, out=dep)
+            F.scan_topk_batched(stores, q, dep.view(S, Hq, 128), k, idx=idx, top_scores=top, workspace=ws)
+        t = _events_ms(torch, step, args.steps, args.warmup, flush)
+        keys = sum(lengths) * 8
+        nbytes = 0
+        for sidx, st in enumerate(stores):
+            U = dep.view(S, 8, 4, 128)[sidx].amax(dim=1)
+            nbytes += st.plane_bytes_read(U)
+        ms = float(np.median(t))
+        out.append({"config": 4, "case": "16 sessions batched", "workload": cfg["name"], "sessions": S,
+                    "total_keys": sum(lengths), "step_ms": ms, "gkeys_per_s": keys / (ms * 1e-3) / 1e9,
+                    "scan_bytes_per_key_per_kv_head": nbytes / keys, "link_gbs": nbytes / (ms * 1e-3) / 1e9,
+                    "launches_per_step": 1 + 1 + 9})
+    elif args.config == 5:
+        cfg = synth.CONFIGS[5]
+        n, L = cfg["n"], cfg["layers"]
+        budgets = synth.rng_for(5, 0, 8).integers(cfg["b_lo"], cfg["b_hi"] + 1, L)
+        layers = []
+        Kr = Vr = None
+        for layer in range(L):
+            inp = synth.layer_inputs_cuda(5, layer=layer, n=n, device=dev, with_values=(layer == 0))
+            st = F.pack_bitplanes(inp["K"]).to_host()
+            if layer == 0:   # one shared interleaved K|V row buffer for all layers
+                Kr, Vr = F.kv_rows(8, n, 128, pin_memory=True)
+                Kr.copy_(inp["K_rows"])
+                Vr.copy_(inp["V_rows"])
+            layers.append((st, inp["q_dev"].clone(), inp["sigma2_dev"].clone(), int(budgets[layer])))
+            del inp
+            torch.cuda.empty_cache()
+        k = cfg["k"]
+        ws = torch.empty(F.decode_workspace_bytes(layers[0][0], 32, k, 1), dtype=torch.uint8, device=dev)
+        bufs = dict(depths=torch.empty((32, 128), dtype=torch.uint8, device=dev),
+                    idx=torch.empty((32, k), dtype=torch.int32, device=dev),
+                    top_scores=torch.empty((32, k), dtype=torch.float32, device=dev),
+                    out=torch.empty((32, 128), dtype=torch.float32, device=dev), workspace=ws)
+
+        def token():
+            for st, qd, s2d, b in layers:
+                F.decode_step(st, qd, s2d, b, k, Kr, Vr, **bufs)
+        t = _events_ms(torch, token, max(3, args.steps // 3), 1, flush)
+        ms = float(np.median(t))
+        out.append({"config": 5, "case": "36-layer decode token", "workload": cfg["name"], "layers": L, "n": n,
+                    "budgets_mean": float(np.mean(budgets)), "token_ms": ms, "per_layer_ms": ms / L,
+                    "gkeys_per_s": n * 8 * L / (ms * 1e-3) / 1e9, "kv_rows": "one buffer shared by all layers"})
+    for line in out:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.config:
+        config_bench(args)
+        return
     if args.impl == "reference":
         run_reference(args)
         return
