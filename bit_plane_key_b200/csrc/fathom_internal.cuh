@@ -11,7 +11,7 @@
 namespace fathom {
 
 constexpr int kBlock = 64;     // tokens per shared block scale
-constexpr int kPad = 128;      // key padding granule of the store
+constexpr int kPad = 1024;     // key padding granule of the store: plane rows start 128-byte aligned
 constexpr int kMaxD = 256;     // largest supported head dimension
 constexpr int kMaxTopK = 4096; // largest supported k
 constexpr size_t kMaxSmem = 227 * 1024;  // opt-in shared memory per CTA on sm_100

@@ -38,7 +38,9 @@
  *     Hkv = number of KV heads, Hq = number of query heads (a multiple of
  *     Hkv, query head h reads KV head h / (Hq/Hkv)), d = head dimension
  *     (a multiple of 32, at most 256), n = number of keys,
- *     n_pad = n rounded up to a multiple of 128.
+ *     n_pad = n rounded up to a multiple of 1024 (so that every plane row,
+ *     n_pad/8 bytes, starts on a 128-byte boundary and the 128-byte run
+ *     that a 1024-key tile reads from it is one aligned line).
  */
 #ifndef FATHOM_H
 #define FATHOM_H
@@ -95,7 +97,7 @@ typedef struct {
     const uint16_t* scales;
 } fathom_store;
 
-/* n rounded up to a multiple of 128; the padded key count of a store. */
+/* n rounded up to a multiple of 1024; the padded key count of a store. */
 int64_t fathom_n_pad(int64_t n);
 /* Bytes of the planes / scales arrays of a store; 0 for invalid sizes. */
 size_t fathom_planes_bytes(int n_kv_heads, int d, int64_t n);

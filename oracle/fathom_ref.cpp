@@ -50,7 +50,7 @@
 typedef int64_t i64;
 
 static const int BLOCK = 64;  /* tokens per shared block scale */
-static const int PAD = 128;   /* keys are padded to a multiple of this */
+static const int PAD = 1024;  /* keys are padded to a multiple of this (a layout convention of the store) */
 
 /* ------------------------------------------------------------------------ */
 /* fp16 / bf16 conversions written from the IEEE 754 binary16 definition.    */

@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(libpath):
 def test_host_only_functions(libpath):
     from bit_plane_key_b200 import fathom as F
     L = F.lib()
-    assert F.n_pad(1) == 128 and F.n_pad(128) == 128 and F.n_pad(4097) == 4224
+    assert F.n_pad(1) == 1024 and F.n_pad(1024) == 1024 and F.n_pad(4097) == 5120
     assert L.fathom_planes_bytes(8, 128, 131072) == 8 * 128 * 4 * 131072 // 8
     assert L.fathom_scales_bytes(8, 128, 131072) == 8 * 128 * (131072 // 64) * 2
     assert L.fathom_planes_bytes(8, 100, 1000) == 0      # d not a multiple of 32
