@@ -215,11 +215,14 @@ class Layer:
         h.copy_(t)
         return h
 
-    def step(self, budget, fixed_r=0, ev=None):
+    def step(self, budget, fixed_r=0, ev=None, pooled=False):
         F = self.F
         if ev:
             ev[0].record()
-        F.alloc_depths(self.q, self.s2, budget, fixed_r=fixed_r, out=self.depths)
+        if pooled:
+            F.alloc_depths_pooled(self.q, self.s2, budget, out=self.depths)
+        else:
+            F.alloc_depths(self.q, self.s2, budget, fixed_r=fixed_r, out=self.depths)
         if ev:
             ev[1].record()
         F.scan_scores(self.store, self.q, self.depths, out=self.scores)
@@ -306,9 +309,9 @@ def link_peak(F, torch, dev, nbytes=1 << 30, reps=10):
             "hbm_read_gbs": hbm}
 
 
-def timed_steps(torch, layer, budget, steps, warmup, fixed_r, flush, clocks_gpu=None):
+def timed_steps(torch, layer, budget, steps, warmup, fixed_r, flush, clocks_gpu=None, pooled=False):
     for _ in range(warmup):
-        layer.step(budget, fixed_r)
+        layer.step(budget, fixed_r, pooled=pooled)
     torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     sampler = ClockSampler(clocks_gpu) if clocks_gpu is not None else None
@@ -317,7 +320,7 @@ def timed_steps(torch, layer, budget, steps, warmup, fixed_r, flush, clocks_gpu=
     try:
         for s in range(steps):
             flush.zero_()
-            layer.step(budget, fixed_r, ev=evs[s])
+            layer.step(budget, fixed_r, ev=evs[s], pooled=pooled)
         torch.cuda.synchronize()
     finally:
         if sampler:
@@ -667,6 +670,15 @@ def main():
                             "scan_ms": float(r2["scan_ms"].mean()),
                             "gkeys_per_s": args.n * layer.Hkv / (float(p2["step_ms"].mean()) * 1e-3) / 1e9,
                             "scan_bytes_per_key_per_kv_head": b2 / (layer.n * layer.Hkv)}
+        # group-pooled depths (a variant, not the pages' per-query rule): one depth
+        # vector per KV head, so the scan reads exactly B plane bits per key
+        r4 = timed_steps(torch, layer, args.budget, args.steps, args.warmup, 0, flush, pooled=True)
+        b4, _ = layer.union_bytes()
+        idx_p = set(layer.idx[0].cpu().numpy().tolist())
+        extras["pooled_B%d" % args.budget] = {
+            "sequential_ms_per_step": float(r4["step_ms"].mean()), "scan_ms": float(r4["scan_ms"].mean()),
+            "scan_bytes_per_key_per_kv_head": b4 / (layer.n * layer.Hkv),
+            "needle_recall_head0": (len(needles & idx_p) / len(needles)) if needles else None}
         layer.step(args.budget)
         if args.resident == "host":
             # the same store in HBM (the pages' control condition)

@@ -52,7 +52,8 @@ int to_status(cudaError_t e) { return e == cudaSuccess ? FATHOM_OK : FATHOM_ECUD
 // Resolve a store's arrays to device-usable addresses, checking residency.
 int resolve_store(const fathom_store* s, const uint32_t** planes, const uint16_t** scales) {
     if (!s || !s->planes || !s->scales) return FATHOM_EINVAL;
-    if (!dims_ok(s->n_kv_heads, s->d) || s->n < 1 || s->n_pad != n_pad_of(s->n)) return FATHOM_EINVAL;
+    if (!dims_ok(s->n_kv_heads, s->d) || s->n < 1 || s->n_pad < n_pad_of(s->n) || s->n_pad % kPad)
+        return FATHOM_EINVAL;
     if ((reinterpret_cast<uintptr_t>(s->planes) & 15) || (reinterpret_cast<uintptr_t>(s->scales) & 1))
         return FATHOM_EINVAL;
     const void* dp = nullptr;
@@ -104,6 +105,30 @@ int fathom_pack_bitplanes(const void* K, int k_dtype, int n_kv_heads, int64_t n,
     return to_status(launch_pack(K, k_dtype, n_kv_heads, n, d, planes, scales, (cudaStream_t)stream));
 }
 
+int fathom_append_keys(fathom_store* store, const void* K_tail, int k_dtype, int64_t n_new, fathom_stream_t stream) {
+    if (!store || !K_tail || !store->planes || !store->scales) return FATHOM_EINVAL;
+    if (k_dtype != FATHOM_F32 && k_dtype != FATHOM_BF16) return FATHOM_EINVAL;
+    const int64_t n_old = store->n;
+    if (!dims_ok(store->n_kv_heads, store->d) || n_old < 0 || n_new <= n_old || store->n_pad % kPad ||
+        n_pad_of(n_new) > store->n_pad)
+        return FATHOM_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(store->planes) & 15) || (reinterpret_cast<uintptr_t>(store->scales) & 1))
+        return FATHOM_EINVAL;
+    const void* dp = nullptr;
+    const void* ds = nullptr;
+    Where want = store->host_resident ? Where::kHostPinned : Where::kDevice;
+    if (classify(store->planes, &dp) != want || classify(store->scales, &ds) != want) return FATHOM_EINVAL;
+    if (!is_device(K_tail)) return FATHOM_EINVAL;
+    const int64_t tail = (n_old / kBlock) * kBlock;   // first key of the last partial block
+    cudaError_t e = launch_pack_blocks(K_tail, k_dtype, store->n_kv_heads, n_new - tail, tail, tail / kBlock,
+                                       (n_new + kBlock - 1) / kBlock, n_new, store->d, store->n_pad,
+                                       const_cast<uint32_t*>(static_cast<const uint32_t*>(dp)),
+                                       const_cast<uint16_t*>(static_cast<const uint16_t*>(ds)), (cudaStream_t)stream);
+    if (e != cudaSuccess) return FATHOM_ECUDA;
+    store->n = n_new;
+    return FATHOM_OK;
+}
+
 int fathom_alloc_depths(const void* q, int q_dtype, const float* sigma2, int n_q_heads, int n_kv_heads, int d,
                         int budget_bits, int fixed_r, uint8_t* depths, fathom_stream_t stream) {
     if (!q || !sigma2 || !depths || !dims_ok(n_kv_heads, d) || n_q_heads < 1 || n_q_heads % n_kv_heads)
@@ -113,6 +138,17 @@ int fathom_alloc_depths(const void* q, int q_dtype, const float* sigma2, int n_q
     if (!is_device(q) || !is_device(sigma2) || !is_device(depths)) return FATHOM_EINVAL;
     return to_status(launch_depths(q, q_dtype, sigma2, n_q_heads, n_kv_heads, d, budget_bits, fixed_r, depths,
                                    (cudaStream_t)stream));
+}
+
+int fathom_alloc_depths_pooled(const void* q, int q_dtype, const float* sigma2, int n_q_heads, int n_kv_heads,
+                               int d, int budget_bits, uint8_t* depths, fathom_stream_t stream) {
+    if (!q || !sigma2 || !depths || !dims_ok(n_kv_heads, d) || n_q_heads < 1 || n_q_heads % n_kv_heads)
+        return FATHOM_EINVAL;
+    if (q_dtype != FATHOM_F32 && q_dtype != FATHOM_BF16) return FATHOM_EINVAL;
+    if (budget_bits < 0) return FATHOM_EINVAL;
+    if (!is_device(q) || !is_device(sigma2) || !is_device(depths)) return FATHOM_EINVAL;
+    return to_status(launch_depths(q, q_dtype, sigma2, n_q_heads, n_kv_heads, d, budget_bits, 0, depths,
+                                   (cudaStream_t)stream, 1));
 }
 
 int fathom_scan_scores(const fathom_store* store, const void* q, int q_dtype, const uint8_t* depths,
@@ -172,12 +208,13 @@ int fathom_scan_topk(const fathom_store* store, const void* q, int q_dtype, cons
         return FATHOM_EINVAL;
     if (!device_status_ptr()) return FATHOM_ECUDA;
     float* scores = static_cast<float*>(workspace);
-    size_t off = ((sizeof(float) * (size_t)n_q_heads * (size_t)store->n_pad) + 255) & ~size_t(255);
+    const int64_t ld = n_pad_of(store->n);   // score row stride
+    size_t off = ((sizeof(float) * (size_t)n_q_heads * (size_t)ld) + 255) & ~size_t(255);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = launch_scan(planes, scales, store->n_kv_heads, store->d, store->n, store->n_pad, q, q_dtype,
                                 depths, n_q_heads, scores, s);
     if (e != cudaSuccess) return FATHOM_ECUDA;
-    e = launch_topk(scores, store->n, store->n_pad, n_q_heads, k, idx, top_scores,
+    e = launch_topk(scores, store->n, ld, n_q_heads, k, idx, top_scores,
                     static_cast<char*>(workspace) + off, s);
     return to_status(e);
 }
@@ -236,14 +273,14 @@ int fathom_scan_topk_batched(const fathom_store* stores, int n_sessions, const v
         sm.n_pad[s] = st.n_pad;
         sm.score_base[s] = (int64_t)(off / sizeof(float));
         sm.tile0[s] = tiles;
-        const int64_t t = (st.n_pad + 1023) / 1024;
+        const int64_t t = n_pad_of(st.n) / 1024;
         if (t > INT32_MAX - tiles) return FATHOM_EINVAL;
         tiles += (int)t;
         rm.base[s] = sm.score_base[s];
-        rm.ld[s] = st.n_pad;
+        rm.ld[s] = n_pad_of(st.n);
         rm.n[s] = st.n;
         rm.max_n = st.n > rm.max_n ? st.n : rm.max_n;
-        off += a256(sizeof(float) * (size_t)n_q_heads * (size_t)st.n_pad);
+        off += a256(sizeof(float) * (size_t)n_q_heads * (size_t)n_pad_of(st.n));
     }
     sm.tile0[n_sessions] = tiles;
     if (!is_device(q) || !is_device(depths) || !is_device(idx) || !is_device(workspace) ||
@@ -290,8 +327,8 @@ size_t fathom_decode_workspace_bytes(const fathom_store* store, int n_q_heads, i
 
 int fathom_decode_step(const fathom_store* store, const void* q, int q_dtype, const float* sigma2, int n_q_heads,
                        int budget_bits, int fixed_r, int k, const uint16_t* K_rows, const uint16_t* V_rows,
-                       int64_t row_stride, int rows_host_resident, int kv_groups, uint8_t* depths, int32_t* idx,
-                       float* top_scores, float* out, void* workspace, size_t workspace_bytes,
+                       int64_t rows_n, int64_t row_stride, int rows_host_resident, int kv_groups, uint8_t* depths,
+                       int32_t* idx, float* top_scores, float* out, void* workspace, size_t workspace_bytes,
                        fathom_stream_t stream) {
     const uint32_t* planes;
     const uint16_t* scales;
@@ -305,7 +342,7 @@ int fathom_decode_step(const fathom_store* store, const void* q, int q_dtype, co
     if (budget_bits < 0 || fixed_r < 0 || fixed_r > d) return FATHOM_EINVAL;
     if (k < 1 || k > n || k > kMaxTopK || n > INT32_MAX) return FATHOM_EINVAL;
     if (d != 32 && d != 64 && d != 128 && d != 256) return FATHOM_EUNSUPPORTED;
-    if (row_stride < d || row_stride % 8) return FATHOM_EINVAL;
+    if (row_stride < d || row_stride % 8 || rows_n < n) return FATHOM_EINVAL;
     if ((reinterpret_cast<uintptr_t>(K_rows) & 15) || (reinterpret_cast<uintptr_t>(V_rows) & 15) ||
         (reinterpret_cast<uintptr_t>(workspace) & 255))
         return FATHOM_EINVAL;
@@ -321,8 +358,8 @@ int fathom_decode_step(const fathom_store* store, const void* q, int q_dtype, co
     if (!device_status_ptr()) return FATHOM_ECUDA;
     return to_status(launch_decode(planes, scales, Hkv, d, n, store->n_pad, q, q_dtype, sigma2, n_q_heads,
                                    budget_bits, fixed_r, k, static_cast<const uint16_t*>(kd),
-                                   static_cast<const uint16_t*>(vd), row_stride, rows_host_resident, kv_groups, depths,
-                                   idx, top_scores, out, workspace, (cudaStream_t)stream));
+                                   static_cast<const uint16_t*>(vd), row_stride, rows_n, rows_host_resident, kv_groups,
+                                   depths, idx, top_scores, out, workspace, (cudaStream_t)stream));
 }
 
 int fathom_last_device_status(fathom_stream_t stream) {

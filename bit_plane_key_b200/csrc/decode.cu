@@ -61,15 +61,16 @@ size_t decode_workspace_bytes(int64_t n, int Hq, int groups, int k) {
 
 cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n, int64_t n_pad,
                           const void* q, int q_dtype, const float* sigma2, int Hq, int budget, int fixed_r, int k,
-                          const uint16_t* K_rows, const uint16_t* V_rows, int64_t row_stride, int rows_host,
-                          int groups, uint8_t* depths, int32_t* idx, float* top_scores, float* out, void* workspace,
-                          cudaStream_t stream) {
+                          const uint16_t* K_rows, const uint16_t* V_rows, int64_t row_stride, int64_t rows_n,
+                          int rows_host, int groups, uint8_t* depths, int32_t* idx, float* top_scores, float* out,
+                          void* workspace, cudaStream_t stream) {
     Aux* aux = aux_for_device();
     if (!aux) return cudaErrorUnknown;
     const int hkv_g = Hkv / groups, hq_g = Hq / groups;
     const size_t q_elt = (q_dtype == FATHOM_BF16) ? 2 : 4;
     float* scores = static_cast<float*>(workspace);
-    void* topk_ws = static_cast<char*>(workspace) + a256(sizeof(float) * (size_t)Hq * (size_t)n_pad);
+    const int64_t ld = n_pad_of(n);   // score row stride; n_pad is the store's row stride
+    void* topk_ws = static_cast<char*>(workspace) + a256(sizeof(float) * (size_t)Hq * (size_t)ld);
 
     cudaError_t e = launch_depths(q, q_dtype, sigma2, Hq, Hkv, d, budget, fixed_r, depths, stream);
     if (e != cudaSuccess) return e;
@@ -77,18 +78,18 @@ cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hk
     for (int i = 0; i < groups; ++i) {
         const int g0 = i * hkv_g, h0 = i * hq_g;
         const void* qi = static_cast<const char*>(q) + q_elt * (size_t)h0 * d;
-        float* si = scores + (size_t)h0 * n_pad;
+        float* si = scores + (size_t)h0 * ld;
         e = launch_scan(planes + (size_t)g0 * d * 4 * (n_pad / 32), scales + (size_t)g0 * d * (n_pad / kBlock),
                         hkv_g, d, n, n_pad, qi, q_dtype, depths + (size_t)h0 * d, hq_g, si, stream);
         if (e == cudaSuccess) e = cudaEventRecord(aux->scanned[i], stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(aux->stream, aux->scanned[i], 0);
         int32_t* ii = idx + (size_t)h0 * k;
         float* ti = top_scores ? top_scores + (size_t)h0 * k : nullptr;
-        const size_t rows_off = (size_t)g0 * n * row_stride;
-        if (e == cudaSuccess) e = launch_topk(si, n, n_pad, hq_g, k, ii, ti, topk_ws, aux->stream);
+        const size_t rows_off = (size_t)g0 * rows_n * row_stride;
+        if (e == cudaSuccess) e = launch_topk(si, n, ld, hq_g, k, ii, ti, topk_ws, aux->stream);
         if (e == cudaSuccess)
-            e = launch_attend(qi, q_dtype, K_rows + rows_off, V_rows + rows_off, row_stride, ii, hq_g, hkv_g, n, d, k,
-                              rows_host, out + (size_t)h0 * d, aux->stream);
+            e = launch_attend(qi, q_dtype, K_rows + rows_off, V_rows + rows_off, row_stride, ii, hq_g, hkv_g, rows_n,
+                              d, k, rows_host, out + (size_t)h0 * d, aux->stream);
         if (e != cudaSuccess) {
             first = e;
             break;

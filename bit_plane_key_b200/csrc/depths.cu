@@ -18,6 +18,12 @@
 // t_c = #{t : key(c,t) >= theta}.  Because the keys are distinct exactly N
 // candidates pass, so sum_c t_c = N = min(B, 4d).
 //
+// Group-pooled variant (not in the pages, which decide per query: arXiv
+// abstract, "each query decides"): the importance of channel c for KV head g
+// is the fp32 sum, in head order, of the group's per-head w_{h,c}; one water
+// level per KV head; every head of the group gets the same depths, so the
+// scan reads exactly min(B, 4d) plane bits per key and KV head.
+//
 // Fixed-r comparison scans (ai-feeds.com summary, 与 Double Sparsity / Loki /
 // SparQ 的差异: a fixed 68 or 136 bits per key): depth 4 on the r channels with
 // the largest |q_c|, ties to the lower channel, by the same select on the
@@ -50,7 +56,7 @@ __device__ __forceinline__ uint64_t warp_select(const uint64_t* keys, int m, int
 
 __global__ void __launch_bounds__(kWarpsPerCta * 32)
 depths_kernel(const void* __restrict__ q, int q_dtype, const float* __restrict__ sigma2, int Hq, int Hkv,
-              int d, int budget, int fixed_r, uint8_t* __restrict__ depths) {
+              int d, int budget, int fixed_r, int pooled, uint8_t* __restrict__ depths) {
     const int lane = threadIdx.x & 31;
     const int h = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
     if (h >= Hq) return;
@@ -66,8 +72,19 @@ depths_kernel(const void* __restrict__ q, int q_dtype, const float* __restrict__
         for (int e = 0; e < kMaxChan; ++e) {
             if (e < per_lane) {
                 int c = lane + 32 * e;
-                float qc = load_q(q, q_dtype, (int64_t)h * d + c);
-                float w = __fmul_rn(__fmul_rn(qc, qc), sigma2[(int64_t)g * d + c]);
+                const float s2 = sigma2[(int64_t)g * d + c];
+                float w;
+                if (pooled) {   // sum of the group's per-head importances, in head order
+                    const int G = Hq / Hkv;
+                    w = 0.0f;
+                    for (int hh = g * G; hh < (g + 1) * G; ++hh) {
+                        const float qc = load_q(q, q_dtype, (int64_t)hh * d + c);
+                        w = __fadd_rn(w, __fmul_rn(__fmul_rn(qc, qc), s2));
+                    }
+                } else {
+                    const float qc = load_q(q, q_dtype, (int64_t)h * d + c);
+                    w = __fmul_rn(__fmul_rn(qc, qc), s2);
+                }
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
                     double v = (double)w * ((t == 0) ? 1.0 : (t == 1) ? 0.25 : (t == 2) ? 0.0625 : 0.015625);
@@ -110,10 +127,10 @@ depths_kernel(const void* __restrict__ q, int q_dtype, const float* __restrict__
 }  // namespace
 
 cudaError_t launch_depths(const void* q, int q_dtype, const float* sigma2, int Hq, int Hkv, int d,
-                          int budget, int fixed_r, uint8_t* depths, cudaStream_t stream) {
+                          int budget, int fixed_r, uint8_t* depths, cudaStream_t stream, int pooled) {
     dim3 grid((unsigned)((Hq + kWarpsPerCta - 1) / kWarpsPerCta));
     depths_kernel<<<grid, kWarpsPerCta * 32, 0, stream>>>(q, q_dtype, sigma2, Hq, Hkv, d, budget, fixed_r,
-                                                         depths);
+                                                         pooled, depths);
     return cudaGetLastError();
 }
 

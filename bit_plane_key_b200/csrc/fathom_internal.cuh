@@ -16,7 +16,7 @@ constexpr int kMaxD = 256;     // largest supported head dimension
 constexpr int kMaxTopK = 4096; // largest supported k
 constexpr size_t kMaxSmem = 227 * 1024;  // opt-in shared memory per CTA on sm_100
 
-inline int64_t n_pad_of(int64_t n) { return ((n + kPad - 1) / kPad) * kPad; }
+__host__ __device__ inline int64_t n_pad_of(int64_t n) { return ((n + kPad - 1) / kPad) * kPad; }
 
 // Per-device status word (FATHOM_DEV_* bits); its device address is passed
 // to every kernel that can set a bit.
@@ -35,8 +35,13 @@ int resolve_store(const fathom_store* s, const uint32_t** planes, const uint16_t
 // Host launchers (each enqueues on `stream`; arguments already validated).
 cudaError_t launch_pack(const void* K, int k_dtype, int Hkv, int64_t n, int d, uint32_t* planes,
                         uint16_t* scales, cudaStream_t stream);
+// (re)packs blocks [blk0, blk1) of a store of row stride n_pad holding n keys,
+// from K = keys [key0, key0 + rows) of every KV head
+cudaError_t launch_pack_blocks(const void* K, int k_dtype, int Hkv, int64_t rows, int64_t key0, int64_t blk0,
+                               int64_t blk1, int64_t n, int d, int64_t n_pad, uint32_t* planes, uint16_t* scales,
+                               cudaStream_t stream);
 cudaError_t launch_depths(const void* q, int q_dtype, const float* sigma2, int Hq, int Hkv, int d,
-                          int budget, int fixed_r, uint8_t* depths, cudaStream_t stream);
+                          int budget, int fixed_r, uint8_t* depths, cudaStream_t stream, int pooled = 0);
 size_t scan_smem_bytes(int d, int G);
 cudaError_t launch_scan(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n,
                         int64_t n_pad, const void* q, int q_dtype, const uint8_t* depths, int Hq,
@@ -76,9 +81,9 @@ cudaError_t launch_scan_batched(const SessionMap& map, int Hkv, int d, const voi
 size_t decode_workspace_bytes(int64_t n, int Hq, int groups, int k);
 cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n, int64_t n_pad,
                           const void* q, int q_dtype, const float* sigma2, int Hq, int budget, int fixed_r, int k,
-                          const uint16_t* K_rows, const uint16_t* V_rows, int64_t row_stride, int rows_host,
-                          int groups, uint8_t* depths, int32_t* idx, float* top_scores, float* out, void* workspace,
-                          cudaStream_t stream);
+                          const uint16_t* K_rows, const uint16_t* V_rows, int64_t row_stride, int64_t rows_n,
+                          int rows_host, int groups, uint8_t* depths, int32_t* idx, float* top_scores, float* out,
+                          void* workspace, cudaStream_t stream);
 cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
                           int64_t row_stride, const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k, int sort_rows, float* out,
                           cudaStream_t stream);

@@ -76,14 +76,15 @@ int fathom_scan_topk_noalloc(const fathom_store* store, const void* q, int q_dty
     if (!device_status_ptr()) return FATHOM_ECUDA;
     char* scratch = static_cast<char*>(scratch_address());
     if (!scratch) return FATHOM_ECUDA;
-    // same split as fathom_scan_topk: scores [Hq][n_pad], then the top-k buffers
+    // same split as fathom_scan_topk: scores [Hq][n_pad_of(n)], then the top-k buffers
     float* scores = reinterpret_cast<float*>(scratch);
-    const size_t off = ((sizeof(float) * (size_t)n_q_heads * (size_t)store->n_pad) + 255) & ~size_t(255);
+    const int64_t ld = n_pad_of(store->n);
+    const size_t off = ((sizeof(float) * (size_t)n_q_heads * (size_t)ld) + 255) & ~size_t(255);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = launch_scan(planes, scales, store->n_kv_heads, store->d, store->n, store->n_pad, q, q_dtype,
                                 depths, n_q_heads, scores, s);
     if (e != cudaSuccess) return FATHOM_ECUDA;
-    return to_status(launch_topk(scores, store->n, store->n_pad, n_q_heads, k, idx, top_scores, scratch + off, s));
+    return to_status(launch_topk(scores, store->n, ld, n_q_heads, k, idx, top_scores, scratch + off, s));
 }
 
 }  // extern "C"

@@ -12,6 +12,12 @@
 // in shared memory with coalesced loads; each warp then owns channels
 // c = warp, warp + 4, ...: lane l quantizes keys l and 32 + l, and a warp
 // ballot per plane yields the two 32-key plane words directly.
+//
+// A block is self-contained (its scale, its two words per plane row), so the
+// same kernel packs a whole store or re-packs a range of blocks: decode-time
+// append re-packs the last partial block (its scale changes when keys join
+// it) and the blocks after it, from a buffer holding the keys from that
+// block's first key on.
 #include "fathom_internal.cuh"
 
 namespace fathom {
@@ -20,18 +26,20 @@ namespace {
 constexpr int kWarps = 4;
 
 __global__ void __launch_bounds__(kWarps * 32)
-pack_kernel(const void* __restrict__ K, int k_dtype, int64_t n, int d, int64_t n_pad,
-            uint32_t* __restrict__ planes, uint16_t* __restrict__ scales) {
+pack_kernel(const void* __restrict__ K, int k_dtype, int64_t rows, int64_t key0, int64_t blk0, int64_t n, int d,
+            int64_t n_pad, uint32_t* __restrict__ planes, uint16_t* __restrict__ scales) {
+    // K holds keys [key0, key0 + rows) of every KV head: [Hkv][rows][d];
+    // n = keys of the store after this pack; n_pad = the store's row stride
     extern __shared__ float tile[];  // [64][d + 1]
     const int g = blockIdx.y;
-    const int64_t blk = blockIdx.x;
+    const int64_t blk = blk0 + blockIdx.x;
     const int64_t i0 = blk * kBlock;
     const int ld = d + 1;
     const int64_t rem = n - i0;
     const int keys = rem <= 0 ? 0 : (rem < kBlock ? (int)rem : kBlock);  // real keys in this block
 
     // Stage the tile: rows [i0, i0 + keys) are contiguous in K.
-    const int64_t base = ((int64_t)g * n + i0) * d;
+    const int64_t base = ((int64_t)g * rows + (i0 - key0)) * d;
     for (int e = threadIdx.x; e < kBlock * d; e += blockDim.x) {
         int r = e / d, c = e - r * d;
         float x = 0.0f;
@@ -85,17 +93,24 @@ pack_kernel(const void* __restrict__ K, int k_dtype, int64_t n, int d, int64_t n
 
 }  // namespace
 
-cudaError_t launch_pack(const void* K, int k_dtype, int Hkv, int64_t n, int d, uint32_t* planes,
-                        uint16_t* scales, cudaStream_t stream) {
-    const int64_t n_pad = n_pad_of(n);
-    dim3 grid((unsigned)(n_pad / kBlock), (unsigned)Hkv);
+cudaError_t launch_pack_blocks(const void* K, int k_dtype, int Hkv, int64_t rows, int64_t key0, int64_t blk0,
+                               int64_t blk1, int64_t n, int d, int64_t n_pad, uint32_t* planes, uint16_t* scales,
+                               cudaStream_t stream) {
+    if (blk1 <= blk0) return cudaSuccess;
+    dim3 grid((unsigned)(blk1 - blk0), (unsigned)Hkv);
     size_t smem = sizeof(float) * kBlock * (d + 1);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    pack_kernel<<<grid, kWarps * 32, smem, stream>>>(K, k_dtype, n, d, n_pad, planes, scales);
+    pack_kernel<<<grid, kWarps * 32, smem, stream>>>(K, k_dtype, rows, key0, blk0, n, d, n_pad, planes, scales);
     return cudaGetLastError();
+}
+
+cudaError_t launch_pack(const void* K, int k_dtype, int Hkv, int64_t n, int d, uint32_t* planes,
+                        uint16_t* scales, cudaStream_t stream) {
+    const int64_t n_pad = n_pad_of(n);
+    return launch_pack_blocks(K, k_dtype, Hkv, n, 0, 0, n_pad / kBlock, n, d, n_pad, planes, scales, stream);
 }
 
 }  // namespace fathom

@@ -103,7 +103,8 @@ __device__ __forceinline__ void load_g(const float* p, bool ok, float (&v)[G]) {
 }
 
 // One (tile of 1024 keys, KV head g) of one store; q, depths and scores are
-// the store's own [Hq][d], [Hq][d] and [Hq][n_pad] arrays.
+// the store's own [Hq][d], [Hq][d] and [Hq][n_pad_of(n)] arrays; n_pad is the
+// store's row stride (its capacity, >= n_pad_of(n)).
 template <int G>
 __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ scales,
                                           int d, int64_t n, int64_t n_pad, int tile, int g,
@@ -348,7 +349,7 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
     // ---- epilogue ----
     if (b < nblocks) {
         const int64_t k0 = tile0 + 64 * b + sv0;   // key of acc[0][0][0]
-        float* out = scores + ((int64_t)g * G + h) * n_pad + k0;
+        float* out = scores + ((int64_t)g * G + h) * n_pad_of(n) + k0;
         const float cst = s_cst[h * 16 + b];
         const bool whole = tile0 + kTileKeys <= n;
 #pragma unroll
@@ -401,7 +402,7 @@ cudaError_t launch_scan_g(const uint32_t* planes, const uint16_t* scales, int Hk
     auto kern = scan_kernel<G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((n_pad + kTileKeys - 1) / kTileKeys), (unsigned)Hkv);
+    dim3 grid((unsigned)(n_pad_of(n) / kTileKeys), (unsigned)Hkv);   // the tiles holding keys; n_pad is the stride
     kern<<<grid, Geo<G>::T, smem, stream>>>(planes, scales, d, n, n_pad, q, q_dtype, depths, scores,
                                             device_status_ptr());
     return cudaGetLastError();

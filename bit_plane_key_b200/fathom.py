@@ -54,6 +54,8 @@ _sig("fathom_planes_bytes", _Z, [_I, _I, _L])
 _sig("fathom_scales_bytes", _Z, [_I, _I, _L])
 _sig("fathom_pack_bitplanes", _I, [_P, _I, _I, _L, _I, _P, _P, _P])
 _sig("fathom_alloc_depths", _I, [_P, _I, _P, _I, _I, _I, _I, _I, _P, _P])
+_sig("fathom_alloc_depths_pooled", _I, [_P, _I, _P, _I, _I, _I, _I, _P, _P])
+_sig("fathom_append_keys", _I, [_SP, _P, _I, _L, _P])
 _sig("fathom_scan_scores", _I, [_SP, _P, _I, _P, _I, _P, _P])
 _sig("fathom_topk_workspace_bytes", _Z, [_L, _I, _I])
 _sig("fathom_topk", _I, [_P, _L, _L, _I, _I, _P, _P, _P, _Z, _P])
@@ -68,7 +70,7 @@ _sig("fathom_scan_batched_workspace_bytes", _Z, [_SP, _I, _I, _I])
 _sig("fathom_scan_topk_batched", _I, [_SP, _I, _P, _I, _P, _I, _I, _P, _P, _P, _Z, _P])
 _sig("fathom_scan_topk_noalloc", _I, [_SP, _P, _I, _P, _I, _I, _P, _P, _P])
 _sig("fathom_decode_workspace_bytes", _Z, [_SP, _I, _I, _I])
-_sig("fathom_decode_step", _I, [_SP, _P, _I, _P, _I, _I, _I, _I, _P, _P, _L, _I, _I, _P, _P, _P, _P, _P, _Z, _P])
+_sig("fathom_decode_step", _I, [_SP, _P, _I, _P, _I, _I, _I, _I, _P, _P, _L, _L, _I, _I, _P, _P, _P, _P, _P, _Z, _P])
 
 
 def lib():
@@ -104,12 +106,13 @@ def n_pad(n):
 
 
 class Store:
-    """A packed bit-plane store: planes u32 [Hkv][d][4][n_pad/32], scales u16 [Hkv][d][n_pad/64]."""
+    """A packed bit-plane store: planes u32 [Hkv][d][4][n_pad/32], scales u16 [Hkv][d][n_pad/64].
+    n = keys held; n_pad = capacity (the row stride, from the arrays' shape)."""
 
     def __init__(self, planes, scales, n, host_resident=None):
         self.planes, self.scales, self.n = planes, scales, int(n)
         self.n_kv_heads, self.d = int(planes.shape[0]), int(planes.shape[1])
-        self.n_pad = n_pad(n)
+        self.n_pad = int(planes.shape[-1]) * 32
         self.host_resident = (not planes.is_cuda) if host_resident is None else bool(host_resident)
         self._c = fathom_store(self.n_kv_heads, self.d, self.n, self.n_pad, int(self.host_resident), 0,
                                planes.data_ptr(), scales.data_ptr())
@@ -118,14 +121,26 @@ class Store:
     def c(self):
         return ctypes.byref(self._c)
 
+    @classmethod
+    def empty(cls, n_kv_heads, d, capacity, device=None, host_resident=False):
+        """An empty store (n = 0) with room for `capacity` keys, zero-filled,
+        in device memory or page-locked host memory; grow it with append_keys."""
+        cap = n_pad(capacity)
+        kw = dict(pin_memory=True) if host_resident else dict(device=device)
+        planes = torch.zeros((n_kv_heads, d, 4, cap // 32), dtype=torch.int32, **kw)
+        scales = torch.zeros((n_kv_heads, d, cap // 64), dtype=torch.int16, **kw)
+        return cls(planes, scales, 0, host_resident=host_resident)
+
     def to_host(self):
         """Copy of this store in page-locked host memory (host-resident)."""
         return Store(self.planes.cpu().pin_memory(), self.scales.cpu().pin_memory(), self.n, host_resident=True)
 
     def plane_bytes_read(self, union_depths):
-        """Plane + scale bytes a scan reads for union depths U [Hkv][d]."""
+        """Plane + scale bytes a scan reads for union depths U [Hkv][d] (over the
+        first n_pad(n) keys, the range a scan covers)."""
         U = union_depths.to(torch.int64)
-        return int(U.sum()) * self.n_pad // 8 + int((U > 0).sum()) * (self.n_pad // 64) * 2
+        npad = n_pad(self.n)
+        return int(U.sum()) * npad // 8 + int((U > 0).sum()) * (npad // 64) * 2
 
 
 def pack_bitplanes(K, planes=None, scales=None, stream=None):
@@ -141,6 +156,16 @@ def pack_bitplanes(K, planes=None, scales=None, stream=None):
     return Store(planes, scales, n, host_resident=False)
 
 
+def append_keys(store, K_tail, n_new, stream=None):
+    """Decode-time append: keys [store.n, n_new) into a store with the capacity.
+    K_tail [Hkv][n_new - t][d] (cuda, float32 or bfloat16) holds the keys from
+    t = (store.n // 64) * 64 on.  Updates store.n."""
+    _check(_lib.fathom_append_keys(store.c, _ptr(K_tail), _dtype_code(K_tail), int(n_new), _stream(stream)),
+           "fathom_append_keys")
+    store.n = int(store._c.n)
+    return store
+
+
 def alloc_depths(q, sigma2, budget_bits, fixed_r=0, out=None, stream=None):
     """q [Hq][d], sigma2 f32 [Hkv][d] -> depths u8 [Hq][d]."""
     Hq, d = q.shape
@@ -152,11 +177,23 @@ def alloc_depths(q, sigma2, budget_bits, fixed_r=0, out=None, stream=None):
     return out
 
 
+def alloc_depths_pooled(q, sigma2, budget_bits, out=None, stream=None):
+    """Group-pooled depths (one depth vector per KV head, repeated for its query
+    heads): q [Hq][d], sigma2 f32 [Hkv][d] -> depths u8 [Hq][d]."""
+    Hq, d = q.shape
+    Hkv = sigma2.shape[0]
+    if out is None:
+        out = torch.empty((Hq, d), dtype=torch.uint8, device=q.device)
+    _check(_lib.fathom_alloc_depths_pooled(_ptr(q), _dtype_code(q), _ptr(sigma2), Hq, Hkv, d, int(budget_bits),
+                                           _ptr(out), _stream(stream)), "fathom_alloc_depths_pooled")
+    return out
+
+
 def scan_scores(store, q, depths, out=None, stream=None):
     """Scores f32 [Hq][n_pad] (padding keys -inf)."""
     Hq = q.shape[0]
     if out is None:
-        out = torch.empty((Hq, store.n_pad), dtype=torch.float32, device=q.device)
+        out = torch.empty((Hq, n_pad(store.n)), dtype=torch.float32, device=q.device)
     _check(_lib.fathom_scan_scores(store.c, _ptr(q), _dtype_code(q), _ptr(depths), Hq, _ptr(out),
                                    _stream(stream)), "fathom_scan_scores")
     return out
@@ -298,8 +335,9 @@ def decode_step(store, q, sigma2, budget_bits, k, K_rows, V_rows, fixed_r=0, kv_
     top_scores or None, out)."""
     Hq, d = q.shape
     dev = q.device
-    if K_rows.stride() != V_rows.stride() or K_rows.stride(2) != 1 or K_rows.stride(0) != store.n * K_rows.stride(1):
-        raise ValueError("K_rows and V_rows need strides (n*s, s, 1), the same for both")
+    rows_n = K_rows.shape[1]
+    if K_rows.stride() != V_rows.stride() or K_rows.stride(2) != 1 or K_rows.stride(0) != rows_n * K_rows.stride(1):
+        raise ValueError("K_rows and V_rows need strides (rows*s, s, 1), the same for both")
     if depths is None:
         depths = torch.empty((Hq, d), dtype=torch.uint8, device=dev)
     if idx is None:
@@ -312,7 +350,7 @@ def decode_step(store, q, sigma2, budget_bits, k, K_rows, V_rows, fixed_r=0, kv_
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     _check(_lib.fathom_decode_step(store.c, _ptr(q), _dtype_code(q), _ptr(sigma2), Hq, int(budget_bits), int(fixed_r),
-                                   int(k), _ptr(K_rows), _ptr(V_rows), int(K_rows.stride(1)),
+                                   int(k), _ptr(K_rows), _ptr(V_rows), int(rows_n), int(K_rows.stride(1)),
                                    int(not K_rows.is_cuda), int(kv_groups), _ptr(depths), _ptr(idx),
                                    _ptr(top_scores), _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
            "fathom_decode_step")

@@ -85,6 +85,11 @@ enum {
  *   host_resident: 0 = both arrays in device memory, 1 = both in page-locked
  *           host memory (the scan then streams only the budgeted planes over
  *           the host link).
+ *   n       keys in the store; n_pad = its capacity and row stride in keys:
+ *           a multiple of 1024, at least fathom_n_pad(n) (equal for a store
+ *           packed once; larger for a cache that grows by fathom_append_keys).
+ *           Scans cover the keys [0, fathom_n_pad(n)) only, and score rows
+ *           have length fathom_n_pad(n) whatever the capacity.
  */
 typedef struct {
     int32_t n_kv_heads;
@@ -122,6 +127,26 @@ int fathom_pack_bitplanes(const void* K, int k_dtype, int n_kv_heads, int64_t n,
                           uint32_t* planes, uint16_t* scales, fathom_stream_t stream);
 
 /*
+ * Decode-time append: adds keys [store->n, n_new) to a store that has the
+ * capacity for them (not on the pages, which pack a cache once; a serving
+ * cache grows by a key per decoded token).  The block scale of the last
+ * partial 64-token block changes when keys join it, so that block is packed
+ * again, from its first key on, together with the new blocks; blocks before
+ * it are untouched.  The result equals fathom_pack_bitplanes of all n_new keys
+ * (bit for bit, over the first fathom_n_pad(n_new) keys of every row).
+ *   store   its planes/scales (device, or page-locked host memory written
+ *           through the mapping) sized for capacity store->n_pad; n may be 0
+ *           (an empty store).  On success store->n becomes n_new.
+ *   K_tail  device, [Hkv][n_new - t][d] with t = (store->n / 64) * 64: the keys
+ *           from the first key of the last partial block to n_new - 1 (keys
+ *           before n keep their values), dtype FATHOM_F32 or FATHOM_BF16.
+ *   Capacity outside [0, n_new] beyond fathom_n_pad(n_new) is never read.
+ * Errors: EINVAL for null pointers, n_new <= store->n, n_pad not a multiple of
+ * 1024 or below fathom_n_pad(n_new), arrays not where host_resident says.
+ */
+int fathom_append_keys(fathom_store* store, const void* K_tail, int k_dtype, int64_t n_new, fathom_stream_t stream);
+
+/*
  * Per-query read depths.
  * [arXiv abstract; ai-feeds summary 关键模块 2-3; evolve.pub Strengths (Sec 3.3)]
  * fixed_r == 0: reverse water-filling.  w_c = fl32(fl32(q_c*q_c)*sigma2_c)
@@ -141,6 +166,19 @@ int fathom_pack_bitplanes(const void* K, int k_dtype, int n_kv_heads, int64_t n,
 int fathom_alloc_depths(const void* q, int q_dtype, const float* sigma2, int n_q_heads,
                         int n_kv_heads, int d, int budget_bits, int fixed_r, uint8_t* depths,
                         fathom_stream_t stream);
+
+/*
+ * Group-pooled depths: a variant for comparison, not the pages' rule (which
+ * decides per query: arXiv abstract, "each query decides").  For KV head g
+ * the importance of channel c is the fp32 sum, in head order, of the group's
+ * per-head importances q_{h,c}^2 sigma2_{g,c} (each product rounded as in
+ * fathom_alloc_depths); one reverse water-filling over it with budget B; every
+ * query head of the group receives the same depths, so the scan reads exactly
+ * min(B, 4d) plane bits per key and KV head.
+ * Arguments and errors as fathom_alloc_depths (no fixed_r).
+ */
+int fathom_alloc_depths_pooled(const void* q, int q_dtype, const float* sigma2, int n_q_heads, int n_kv_heads,
+                               int d, int budget_bits, uint8_t* depths, fathom_stream_t stream);
 
 /*
  * Variable-depth scan: approximate scores of every key for every query head.
@@ -275,7 +313,10 @@ int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, con
  *   store        device- or host-resident store, as fathom_scan_topk.
  *   q, q_dtype, sigma2, budget_bits, fixed_r  as fathom_alloc_depths.
  *   k            as fathom_scan_topk (1 <= k <= min(n, 4096)).
- *   K_rows, V_rows, row_stride, rows_host_resident  as fathom_sparse_attend.
+ *   K_rows, V_rows, row_stride, rows_host_resident  as fathom_sparse_attend;
+ *   rows_n       keys per KV head in the row arrays (>= store->n; a growing
+ *                cache keeps its rows at a capacity: the head stride is
+ *                rows_n * row_stride).
  *   kv_groups    1 <= kv_groups <= 64, dividing the store's n_kv_heads.
  *   depths       device, u8 [Hq][d], written.
  *   idx          device, i32 [Hq][k]; top_scores device f32 [Hq][k] or NULL.
@@ -288,8 +329,8 @@ int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, con
 size_t fathom_decode_workspace_bytes(const fathom_store* store, int n_q_heads, int k, int kv_groups);
 int fathom_decode_step(const fathom_store* store, const void* q, int q_dtype, const float* sigma2, int n_q_heads,
                        int budget_bits, int fixed_r, int k, const uint16_t* K_rows, const uint16_t* V_rows,
-                       int64_t row_stride, int rows_host_resident, int kv_groups, uint8_t* depths, int32_t* idx,
-                       float* top_scores, float* out, void* workspace, size_t workspace_bytes,
+                       int64_t rows_n, int64_t row_stride, int rows_host_resident, int kv_groups, uint8_t* depths,
+                       int32_t* idx, float* top_scores, float* out, void* workspace, size_t workspace_bytes,
                        fathom_stream_t stream);
 
 /*

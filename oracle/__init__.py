@@ -71,6 +71,8 @@ def _declare(L):
     L.oref_fixed_depths.argtypes = [_P, _I, _I, _P]
     L.oref_alloc_depths.restype = _I
     L.oref_alloc_depths.argtypes = [_P, _P, _I, _I, _I, _I, _I, _P]
+    L.oref_alloc_depths_pooled.restype = _I
+    L.oref_alloc_depths_pooled.argtypes = [_P, _P, _I, _I, _I, _I, _P]
     L.oref_reconstruct.argtypes = [_P, _P, _I, _L, _I, _I, _P, _P]
     L.oref_scores_head.restype = _I
     L.oref_scores_head.argtypes = [_P, _P, _I, _L, _I, _I, _P, _P, _L, _L, _P, _P]
@@ -163,6 +165,17 @@ def fixed_depths(q, r):
     t = np.empty(q.size, np.uint8)
     _check(lib().oref_fixed_depths(_ptr(q), q.size, int(r), _ptr(t)), "fixed_depths")
     return t
+
+
+def alloc_depths_pooled(q, sigma2, B):
+    """Group-pooled depths (a variant, not the pages' per-query rule)."""
+    q = _c(q, np.float32)
+    s = _c(sigma2, np.float32)
+    Hq, d = q.shape
+    Hkv = s.shape[0]
+    out = np.empty((Hq, d), np.uint8)
+    _check(lib().oref_alloc_depths_pooled(_ptr(q), _ptr(s), Hq, Hkv, d, int(B), _ptr(out)), "alloc_depths_pooled")
+    return out
 
 
 def alloc_depths(q, sigma2, B, fixed_r=0):

@@ -277,6 +277,32 @@ extern "C" int oref_alloc_depths(const float* q, const float* sigma2, int Hq, in
     return 0;
 }
 
+/* Group-pooled variant (not the pages' per-query rule): the importance of
+ * channel c for KV head g is the fp32 sum, heads in order, of the group's
+ * per-head importances; one water-filling per KV head, copied to every
+ * query head of the group. */
+extern "C" int oref_alloc_depths_pooled(const float* q, const float* sigma2, int Hq, int Hkv, int d, int B,
+                                        uint8_t* depths) {
+    if (Hkv <= 0 || Hq % Hkv) return -1;
+    int G = Hq / Hkv;
+    std::vector<float> w(d), wh(d);
+    for (int g = 0; g < Hkv; ++g) {
+        for (int c = 0; c < d; ++c) w[c] = 0.0f;
+        for (int h = g * G; h < (g + 1) * G; ++h) {
+            oref_importance(q + (i64)h * d, sigma2 + (i64)g * d, d, wh.data());
+            for (int c = 0; c < d; ++c) {
+                volatile float acc = w[c] + wh[c];
+                w[c] = acc;
+            }
+        }
+        int rc = oref_depths(w.data(), d, B, depths + (i64)g * G * d);
+        if (rc) return rc;
+        for (int h = g * G + 1; h < (g + 1) * G; ++h)
+            for (int c = 0; c < d; ++c) depths[(i64)h * d + c] = depths[(i64)g * G * d + c];
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* (5) Basis rule on a read prefix [AIF 关键模块 4, paper Sec 3.5; ABS;       */
 /*     EVO Strengths, paper Sec 3.2]: khat = Delta * sum_{j<t}(2b_j-1)2^(2-j) */

@@ -152,6 +152,23 @@ def test_depths_extreme_importance(ref):
         assert np.array_equal(got, ref.alloc_depths(q, s2, B)), B
 
 
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_pooled_depths_bit_exact(ref, G):
+    """Group-pooled depths (the comparison variant) equal the oracle's, and the
+    scan over them reads exactly min(B, 4d) plane bits per key."""
+    rng = np.random.default_rng(50 + G)
+    Hkv, d = 2, 128
+    sig = synth.channel_sigma(rng, Hkv, d)
+    s2 = (sig * sig).astype(np.float32)
+    qb = synth.f32_to_bf16_bits(rng.standard_normal((Hkv * G, d)).astype(np.float32))
+    qd, qf = bf16(qb), synth.bf16_bits_to_f32(qb)
+    for B in (0, 5, 46, 92, 136, 4 * d, 4 * d + 9):
+        got = host(F.alloc_depths_pooled(qd, dev(s2), B))
+        assert np.array_equal(got, ref.alloc_depths_pooled(qf, s2, B)), B
+        assert np.all(got.reshape(Hkv, G, d) == got.reshape(Hkv, G, d)[:, :1])
+        assert np.all(got.sum(1) == min(B, 4 * d))
+
+
 # --------------------------------------------------------------------------
 # a4: scan scores within tolerance (+ the basis rule at every depth)
 # --------------------------------------------------------------------------

@@ -195,6 +195,54 @@ def test_depths_powers_of_four_closed_form(ref):
         assert ref.depths(w, B).tolist() == t_closed.tolist()
 
 
+# --------------------------------------------------------------------------
+# Group-pooled depths (a variant for comparison): reductions to the per-query
+# rule and optimality of the pooled objective
+# --------------------------------------------------------------------------
+def test_pooled_depths_reduce_to_per_query_rule(ref):
+    rng = np.random.default_rng(11)
+    d = 64
+    s2 = np.exp(rng.uniform(-3, 2, (2, d))).astype(np.float32)
+    q = rng.standard_normal((2, d)).astype(np.float32)
+    for B in (0, 17, 92, 256, 300):
+        # one query head per KV head: pooling changes nothing
+        assert np.array_equal(ref.alloc_depths_pooled(q, s2, B), ref.alloc_depths(q, s2, B))
+        # two identical query heads: the pooled weight is exactly 2w, which orders as w
+        q2 = np.repeat(q, 2, axis=0)
+        want = np.repeat(ref.alloc_depths(q, s2, B), 2, axis=0)
+        assert np.array_equal(ref.alloc_depths_pooled(q2, s2, B), want)
+
+
+@pytest.mark.parametrize("d", [1, 2, 3])
+def test_pooled_depths_minimise_the_group_distortion(ref, d):
+    """For G = 2 the pooled depths minimise sum_c (w_0c + w_1c) 4^-t_c over all
+    depth vectors with sum t = min(B, 4d) (brute force), and both heads get them."""
+    rng = np.random.default_rng(40 + d)
+    for trial in range(20):
+        q = rng.standard_normal((2, d)).astype(np.float32)
+        s2 = np.exp(rng.uniform(-2, 2, (1, d))).astype(np.float32)
+        wsum = np.asarray(q[0], np.float64) ** 2 * s2[0] + np.asarray(q[1], np.float64) ** 2 * s2[0]
+        for B in range(0, 4 * d + 2):
+            t = ref.alloc_depths_pooled(q, s2, B)
+            assert np.array_equal(t[0], t[1])
+            N = min(B, 4 * d)
+            assert int(t[0].sum()) == N
+            best = min(_objective(wsum, tt) for tt in itertools.product(range(5), repeat=d) if sum(tt) == N)
+            assert _objective(wsum, t[0]) == pytest.approx(best, rel=1e-6, abs=0.0)
+
+
+def test_pooled_depths_hand_example(ref):
+    """Two heads that each care about a different channel: per query each reads
+    its own channel; pooled, the group splits the budget by the summed weight."""
+    q = np.array([[2.0, 0.0, 1.0, 0.0], [0.0, 2.0, 1.0, 0.0]], np.float32)
+    s2 = np.ones((1, 4), np.float32)
+    # pooled w = (4, 4, 2, 0): candidates 4,4,1,1,2,0.5,0.5,0.25,... in (v desc, c asc, t asc)
+    # B = 3 takes (c0,t0), (c1,t0), (c2,t0)
+    assert ref.alloc_depths_pooled(q, s2, 3).tolist() == [[1, 1, 1, 0], [1, 1, 1, 0]]
+    # per query: head 0 w = (4, 0, 1, 0) takes (c0,t0), (c0,t1), (c2,t0)
+    assert ref.alloc_depths(q, s2, 3).tolist() == [[2, 0, 1, 0], [0, 2, 1, 0]]
+
+
 def test_depths_tie_rule(ref):
     w = np.ones(4, np.float32)
     assert ref.depths(w, 5).tolist() == [2, 1, 1, 1]
