@@ -56,6 +56,9 @@ def parse():
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     p.add_argument("--config", type=int, default=None, choices=[1, 2, 4, 5],
                    help="measure another workload of the method (one JSON line per case; not the headline)")
+    p.add_argument("--fidelity", type=int, default=None, choices=[2, 3],
+                   help="fidelity of the sparse step against exact dense attention on config 2 or 3 (a measurement "
+                        "harness: attention error, recall of the exact top-k, needle recall, bytes per key)")
     p.add_argument("--kernel", default=None, choices=["scan"],
                    help="time one kernel alone on this workload (a kernel benchmark, not the step metric)")
     return p.parse_args()
@@ -587,8 +590,78 @@ def config_bench(args):
         print(json.dumps(line), flush=True)
 
 
+def fidelity_bench(args):
+    """Per read policy (B in {46, 68, 92, 136}, fixed68, fixed136, pooled B=92):
+    the one-call decode step's attention output against exact dense attention
+    over all n keys (a plain fp32 torch reference, measurement only), the
+    recall of the exact top-k (top-k of q.k over the bf16 keys), the needles
+    found (config 3) and the plane + scale bytes the scan reads."""
+    import torch
+    import synth
+    from bit_plane_key_b200 import fathom as F
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = synth.CONFIGS[args.fidelity]
+    inp = synth.layer_inputs_cuda(args.fidelity, device=dev)
+    Hkv, Hq, d, n, k = cfg["n_kv_heads"], cfg["n_q_heads"], cfg["d"], cfg["n"], cfg["k"]
+    G = Hq // Hkv
+    st = F.pack_bitplanes(inp["K"])
+    del inp["K"]
+    Kr, Vr = inp["K_rows"], inp["V_rows"]
+    q = inp["q_dev"]
+    qf = q.float()
+    # exact dense attention, the exact top-k and the dense softmax, per KV head
+    dense = torch.empty((Hq, d), dtype=torch.float32, device=dev)
+    exact_idx = torch.empty((Hq, k), dtype=torch.int64, device=dev)
+    probs = torch.empty((Hq, n), dtype=torch.float32, device=dev)
+    for g in range(Hkv):
+        Kg = Kr[g].float()
+        s = qf[g * G:(g + 1) * G] @ Kg.T                       # [G][n]
+        exact_idx[g * G:(g + 1) * G] = torch.topk(s, k, dim=1).indices
+        p = torch.softmax(s / d ** 0.5, dim=1)
+        probs[g * G:(g + 1) * G] = p
+        dense[g * G:(g + 1) * G] = p @ Vr[g].float()
+        del Kg, s, p
+    # attention restricted to the exact top-k: the best any k-row selection can do
+    exact_sparse = F.sparse_attend(q, Kr, Vr, exact_idx.to(torch.int32).contiguous())
+    mass_exact = torch.gather(probs, 1, exact_idx).sum(1)
+    needles = set(inp.get("needles", np.array([], np.int64)).tolist())
+    policies = [("B=%d" % b, b, 0, False) for b in (46, 68, 92, 136)]
+    policies += [("fixed68_r16", 0, 16, False), ("fixed136_r32", 0, 32, False), ("pooled_B92", 92, 0, True)]
+    for name, b, fr, pooled in policies:
+        if pooled:
+            dep = F.alloc_depths_pooled(q, inp["sigma2_dev"], b)
+            idx, _ = F.scan_topk(st, q, dep, k)
+            out = F.sparse_attend(q, Kr, Vr, idx)
+        else:
+            dep, idx, _, out = F.decode_step(st, q, inp["sigma2_dev"], b, k, Kr, Vr, fixed_r=fr)
+        U = dep.view(Hkv, G, d).amax(dim=1)
+        nbytes = st.plane_bytes_read(U)
+        err = ((out - dense).norm(dim=1) / dense.norm(dim=1)).cpu().numpy()
+        err_x = ((out - exact_sparse).norm(dim=1) / exact_sparse.norm(dim=1)).cpu().numpy()
+        mass = torch.gather(probs, 1, idx.long()).sum(1)
+        rec = []
+        for h in range(Hq):
+            a = set(idx[h].cpu().numpy().tolist())
+            e = set(exact_idx[h].cpu().numpy().tolist())
+            rec.append(len(a & e) / k)
+        found = len(needles & set(idx[0].cpu().numpy().tolist())) / len(needles) if needles else None
+        print(json.dumps({"fidelity": args.fidelity, "policy": name, "n": n, "k": k,
+                          "scan_bytes_per_key_per_kv_head": nbytes / (n * Hkv),
+                          "softmax_mass_captured_mean": float(mass.mean()),
+                          "softmax_mass_exact_topk_mean": float(mass_exact.mean()),
+                          "attn_rel_err_vs_exact_topk_mean": float(err_x.mean()),
+                          "attn_rel_err_vs_exact_topk_max": float(err_x.max()),
+                          "attn_rel_err_vs_dense_mean": float(err.mean()),
+                          "exact_topk_recall_mean": float(np.mean(rec)), "exact_topk_recall_min": float(np.min(rec)),
+                          "needle_recall_head0": found}), flush=True)
+
+
 def main():
     args = parse()
+    if args.fidelity:
+        fidelity_bench(args)
+        return
     if args.config:
         config_bench(args)
         return
