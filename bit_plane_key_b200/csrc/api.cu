@@ -184,6 +184,21 @@ int fathom_topk(const float* scores, int64_t n, int64_t ld, int n_rows, int k, i
     return to_status(launch_topk(scores, n, ld, n_rows, k, idx, top_scores, workspace, (cudaStream_t)stream));
 }
 
+int fathom_topk_merge(const float* cand_scores, const int32_t* cand_idx, int n_rows, int n_cand, int k, int32_t* idx,
+                      float* top_scores, void* workspace, size_t workspace_bytes, fathom_stream_t stream) {
+    if (!cand_scores || !cand_idx || !idx || !workspace || n_rows < 1 || n_cand < 1 || k < 1 || k > n_cand ||
+        k > kMaxTopK)
+        return FATHOM_EINVAL;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return FATHOM_EINVAL;
+    if (workspace_bytes < topk_workspace_bytes(n_cand, n_rows, k)) return FATHOM_ENOMEM;
+    if (!is_device(cand_scores) || !is_device(cand_idx) || !is_device(idx) || !is_device(workspace) ||
+        (top_scores && !is_device(top_scores)))
+        return FATHOM_EINVAL;
+    if (!device_status_ptr()) return FATHOM_ECUDA;
+    return to_status(launch_topk_merge(cand_scores, cand_idx, n_rows, n_cand, k, idx, top_scores, workspace,
+                                       (cudaStream_t)stream));
+}
+
 size_t fathom_scan_workspace_bytes(const fathom_store* store, int n_q_heads, int k) {
     if (!store || n_q_heads < 1 || k < 1 || k > kMaxTopK || store->n < 1) return 0;
     size_t scores = ((sizeof(float) * (size_t)n_q_heads * (size_t)n_pad_of(store->n)) + 255) & ~size_t(255);

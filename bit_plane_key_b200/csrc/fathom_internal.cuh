@@ -62,6 +62,8 @@ struct RowMap {
 };
 cudaError_t launch_topk(const float* scores, int64_t n, int64_t ld, int rows, int k, int32_t* idx,
                         float* top_scores, void* ws, cudaStream_t stream);
+cudaError_t launch_topk_merge(const float* cand_scores, const int32_t* cand_idx, int rows, int n_cand, int k,
+                              int32_t* idx, float* top_scores, void* ws, cudaStream_t stream);
 cudaError_t launch_topk_map(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
                             float* top_scores, void* ws, cudaStream_t stream);
 

@@ -505,7 +505,25 @@ topk_finish(const float* __restrict__ scores, const __grid_constant__ RowMap m, 
     }
 }
 
+// positions into the gathered candidate lists -> the candidates' global indices
+__global__ void topk_map_positions(const int32_t* __restrict__ cand_idx, int n_cand, int k, int32_t* idx) {
+    const int row = blockIdx.y;
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= k) return;
+    const int32_t p = idx[(int64_t)row * k + e];
+    idx[(int64_t)row * k + e] = (p >= 0 && p < n_cand) ? cand_idx[(int64_t)row * n_cand + p] : -1;
+}
+
 }  // namespace
+
+cudaError_t launch_topk_merge(const float* cand_scores, const int32_t* cand_idx, int rows, int n_cand, int k,
+                              int32_t* idx, float* top_scores, void* ws, cudaStream_t stream) {
+    cudaError_t e = launch_topk(cand_scores, n_cand, n_cand, rows, k, idx, top_scores, ws, stream);
+    if (e != cudaSuccess) return e;
+    topk_map_positions<<<dim3((unsigned)((k + 255) / 256), (unsigned)rows), 256, 0, stream>>>(cand_idx, n_cand, k,
+                                                                                             idx);
+    return cudaGetLastError();
+}
 
 size_t topk_workspace_bytes(int64_t n, int rows, int k) {
     (void)n;

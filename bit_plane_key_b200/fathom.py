@@ -56,6 +56,7 @@ _sig("fathom_pack_bitplanes", _I, [_P, _I, _I, _L, _I, _P, _P, _P])
 _sig("fathom_alloc_depths", _I, [_P, _I, _P, _I, _I, _I, _I, _I, _P, _P])
 _sig("fathom_alloc_depths_pooled", _I, [_P, _I, _P, _I, _I, _I, _I, _P, _P])
 _sig("fathom_append_keys", _I, [_SP, _P, _I, _L, _P])
+_sig("fathom_topk_merge", _I, [_P, _P, _I, _I, _I, _P, _P, _P, _Z, _P])
 _sig("fathom_scan_scores", _I, [_SP, _P, _I, _P, _I, _P, _P])
 _sig("fathom_topk_workspace_bytes", _Z, [_L, _I, _I])
 _sig("fathom_topk", _I, [_P, _L, _L, _I, _I, _P, _P, _P, _Z, _P])
@@ -215,6 +216,23 @@ def topk(scores, n, k, idx=None, top_scores=None, workspace=None, stream=None):
         workspace = torch.empty(max(nb, 1), dtype=torch.uint8, device=scores.device)
     _check(_lib.fathom_topk(_ptr(scores), int(n), int(ld), rows, int(k), _ptr(idx), _ptr(top_scores),
                             _ptr(workspace), workspace.numel(), _stream(stream)), "fathom_topk")
+    return idx, top_scores
+
+
+def topk_merge(cand_scores, cand_idx, k, idx=None, top_scores=None, workspace=None, stream=None):
+    """Top-k of gathered per-shard lists: cand_scores f32 / cand_idx i32 [rows][n_cand]
+    (shards in ascending key-range order, each list in top-k order) -> idx, scores [rows][k]."""
+    rows, n_cand = cand_scores.shape
+    if idx is None:
+        idx = torch.empty((rows, k), dtype=torch.int32, device=cand_scores.device)
+    if top_scores is None:
+        top_scores = torch.empty((rows, k), dtype=torch.float32, device=cand_scores.device)
+    nb = topk_workspace_bytes(n_cand, rows, k)
+    if workspace is None:
+        workspace = torch.empty(max(nb, 1), dtype=torch.uint8, device=cand_scores.device)
+    _check(_lib.fathom_topk_merge(_ptr(cand_scores), _ptr(cand_idx), rows, n_cand, int(k), _ptr(idx),
+                                  _ptr(top_scores), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "fathom_topk_merge")
     return idx, top_scores
 
 

@@ -189,7 +189,7 @@ int fathom_alloc_depths_pooled(const void* q, int q_dtype, const float* sigma2, 
  *   store   a packed store (device or host-resident).
  *   q       device, [Hq][d], FATHOM_F32 or FATHOM_BF16.
  *   depths  device, u8 [Hq][d], values 0..4.
- *   scores  device, f32 [Hq][store->n_pad]; keys >= n are written -inf.
+ *   scores  device, f32 [Hq][fathom_n_pad(store->n)]; keys >= n are written -inf.
  * Errors: EINVAL as above, or a host-resident store whose pointers are not
  * page-locked, or a device store whose pointers are not device memory.
  */
@@ -210,6 +210,26 @@ int fathom_scan_scores(const fathom_store* store, const void* q, int q_dtype, co
 size_t fathom_topk_workspace_bytes(int64_t n, int n_rows, int k);
 int fathom_topk(const float* scores, int64_t n, int64_t ld, int n_rows, int k, int32_t* idx,
                 float* top_scores, void* workspace, size_t workspace_bytes, fathom_stream_t stream);
+
+/*
+ * Merge of per-shard top-k lists, for a key range split across GPUs (not on
+ * the pages, whose system runs on one GPU): every GPU scans a contiguous,
+ * 1024-aligned key range and takes its local top-k; the lists are gathered
+ * (one all-gather of (score, index) pairs per query head) and merged here
+ * into the top-k of all keys.
+ *   cand_scores  device, f32 [n_rows][n_cand]: the gathered lists, shard by
+ *                shard in ascending key-range order, each list in (score
+ *                descending, index ascending) order; padding entries -inf.
+ *   cand_idx     device, i32 [n_rows][n_cand]: the candidates' global key
+ *                indices.
+ *   idx, top_scores (or NULL), workspace (fathom_topk_workspace_bytes(n_cand,
+ *                n_rows, k) bytes)  as fathom_topk.
+ * Equal scores go to the candidate listed first, which is the lower global
+ * index under the ordering above, so the result equals the top-k of the
+ * unsplit scores.  Errors as fathom_topk with n = n_cand.
+ */
+int fathom_topk_merge(const float* cand_scores, const int32_t* cand_idx, int n_rows, int n_cand, int k, int32_t* idx,
+                      float* top_scores, void* workspace, size_t workspace_bytes, fathom_stream_t stream);
 
 /*
  * Scan + top-k of one decode step of one layer (fathom_scan_scores followed

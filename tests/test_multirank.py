@@ -77,3 +77,66 @@ def test_single_process_needs_no_group():
         os.environ.update(env)
     v, ms = throughput(1 << 20, 1, 50.0, 10)
     assert ms == 5.0 and v == pytest.approx((1 << 20) / 5e-3 / 1e9)
+
+
+def _shard_rank_main(rank, world, port, outdir, scores_path):
+    """Key-range sharding on CPU: local top-k of the rank's range (the oracle),
+    the gloo all-gather of (score, global index) lists, then a merge."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    import oracle
+    from bit_plane_key_b200.ranks import Ranks
+    from bit_plane_key_b200.shard import gather_candidates, shard_range
+    ranks = Ranks("gloo", device=torch.device("cpu"), timeout_s=60)
+    s = np.load(scores_path)
+    rows, n = s.shape
+    k = 300
+    k0, k1 = shard_range(n, world, rank)
+    top = np.full((rows, k), -np.inf, np.float32)
+    idx = np.full((rows, k), -1, np.int32)
+    for r in range(rows):
+        loc = oracle.topk(s[r, k0:k1], min(k, k1 - k0))
+        top[r, :len(loc)] = s[r, k0 + loc]
+        idx[r, :len(loc)] = loc + k0
+    cs, ci = gather_candidates(torch.from_numpy(top), torch.from_numpy(idx))
+    merged = []
+    for r in range(rows):
+        pos = oracle.topk(cs[r].numpy(), k)   # ties -> the candidate listed first
+        merged.append(ci[r].numpy()[pos].tolist())
+    ranks.close()
+    with open(os.path.join(outdir, "shard%d.json" % rank), "w") as f:
+        json.dump({"range": [k0, k1], "merged": merged}, f)
+
+
+@pytest.mark.timeout(180)
+def test_key_range_sharding_merge_on_two_gloo_ranks(tmp_path, ref):
+    """Two ranks each take the top-k of their key range; after the all-gather
+    and the merge both hold the top-k of the whole rows, ties (planted across
+    the range boundary) resolved to the lower global index."""
+    rng = np.random.default_rng(3)
+    rows, n = 3, 5000
+    s = np.round(rng.standard_normal((rows, n)), 1).astype(np.float32)   # many exact ties
+    s[:, 2040:2060] = 9.0                                                 # equal top scores on both sides of 2048
+    path = tmp_path / "scores.npy"
+    np.save(path, s)
+    world = 2
+    mp.start_processes(_shard_rank_main, args=(world, _free_port(), str(tmp_path), str(path)), nprocs=world,
+                       join=True, start_method="spawn")
+    out = [json.load(open(tmp_path / ("shard%d.json" % i))) for i in range(world)]
+    assert out[0]["range"] == [0, 3072] and out[1]["range"] == [3072, 5000]
+    for r in range(rows):
+        want = ref.topk(s[r], 300).tolist()
+        assert out[0]["merged"][r] == want and out[1]["merged"][r] == want
+
+
+def test_shard_ranges_cover_the_keys_on_aligned_cuts():
+    from bit_plane_key_b200.shard import shard_range
+    for n in (1, 1000, 1024, 5000, 1 << 20, (1 << 20) + 17):
+        for world in (1, 2, 3, 8):
+            cuts = [shard_range(n, world, r) for r in range(world)]
+            assert cuts[0][0] == 0 and cuts[-1][1] == n
+            for (a0, a1), (b0, b1) in zip(cuts, cuts[1:]):
+                assert a1 == b0
+            for a0, a1 in cuts:   # every non-empty range starts on a 1024-key cut; empty ones sit at n
+                assert (a0 % 1024 == 0) if a0 < a1 else (a0 == n)
