@@ -211,6 +211,7 @@ class Layer:
         self.top = torch.empty((self.Hq, args.k), dtype=torch.float32, device=dev)
         self.out = torch.empty((self.Hq, self.d), dtype=torch.float32, device=dev)
         self.ws = torch.empty(F.topk_workspace_bytes(self.n, self.Hq, args.k), dtype=torch.uint8, device=dev)
+        self.bmax = F.block_max_buffer(self.Hq, self.n, dev)
         self.dws = None
 
     def _pin(self, t):
@@ -228,10 +229,11 @@ class Layer:
             F.alloc_depths(self.q, self.s2, budget, fixed_r=fixed_r, out=self.depths)
         if ev:
             ev[1].record()
-        F.scan_scores(self.store, self.q, self.depths, out=self.scores)
+        F.scan_scores(self.store, self.q, self.depths, out=self.scores, block_max=self.bmax)
         if ev:
             ev[2].record()
-        F.topk(self.scores, self.n, self.args.k, idx=self.idx, top_scores=self.top, workspace=self.ws)
+        F.topk(self.scores, self.n, self.args.k, idx=self.idx, top_scores=self.top, workspace=self.ws,
+               block_max=self.bmax)
         if ev:
             ev[3].record()
         F.sparse_attend(self.q, self.K_rows, self.V_rows, self.idx, out=self.out)

@@ -152,36 +152,43 @@ int fathom_alloc_depths_pooled(const void* q, int q_dtype, const float* sigma2, 
 }
 
 int fathom_scan_scores(const fathom_store* store, const void* q, int q_dtype, const uint8_t* depths,
-                       int n_q_heads, float* scores, fathom_stream_t stream) {
+                       int n_q_heads, float* scores, uint32_t* block_max, fathom_stream_t stream) {
     const uint32_t* planes;
     const uint16_t* scales;
     int rc = resolve_store(store, &planes, &scales);
     if (rc) return rc;
     if (!q || !depths || !scores || !heads_ok(n_q_heads, store->n_kv_heads)) return FATHOM_EINVAL;
     if (q_dtype != FATHOM_F32 && q_dtype != FATHOM_BF16) return FATHOM_EINVAL;
-    if (!is_device(q) || !is_device(depths) || !is_device(scores)) return FATHOM_EINVAL;
+    if (!is_device(q) || !is_device(depths) || !is_device(scores) || (block_max && !is_device(block_max)))
+        return FATHOM_EINVAL;
     if (!scan_fits(store->d, n_q_heads, store->n_kv_heads)) return FATHOM_EUNSUPPORTED;
     if (!device_status_ptr()) return FATHOM_ECUDA;
     return to_status(launch_scan(planes, scales, store->n_kv_heads, store->d, store->n, store->n_pad, q, q_dtype,
-                                 depths, n_q_heads, scores, (cudaStream_t)stream));
+                                 depths, n_q_heads, scores, (cudaStream_t)stream, block_max));
 }
 
 size_t fathom_topk_workspace_bytes(int64_t n, int n_rows, int k) {
     if (n < 1 || n_rows < 1 || k < 1 || k > kMaxTopK) return 0;
-    return topk_workspace_bytes(n, n_rows, k);
+    const size_t a = topk_workspace_bytes(n, n_rows, k), b = topk_blocks_workspace_bytes(n_rows);
+    return a > b ? a : b;   // either path
 }
 
-int fathom_topk(const float* scores, int64_t n, int64_t ld, int n_rows, int k, int32_t* idx, float* top_scores,
-                void* workspace, size_t workspace_bytes, fathom_stream_t stream) {
+int fathom_topk(const float* scores, const uint32_t* block_max, int64_t n, int64_t ld, int n_rows, int k,
+                int32_t* idx, float* top_scores, void* workspace, size_t workspace_bytes, fathom_stream_t stream) {
     if (!scores || !idx || !workspace || n < 1 || ld < n || n_rows < 1 || k < 1 || k > n || k > kMaxTopK ||
         n > INT32_MAX)
         return FATHOM_EINVAL;
+    if (block_max && ld % kBlock) return FATHOM_EINVAL;
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return FATHOM_EINVAL;
-    if (workspace_bytes < topk_workspace_bytes(n, n_rows, k)) return FATHOM_ENOMEM;
-    if (!is_device(scores) || !is_device(idx) || !is_device(workspace) || (top_scores && !is_device(top_scores)))
+    if (workspace_bytes < fathom_topk_workspace_bytes(n, n_rows, k)) return FATHOM_ENOMEM;
+    if (!is_device(scores) || !is_device(idx) || !is_device(workspace) || (top_scores && !is_device(top_scores)) ||
+        (block_max && !is_device(block_max)))
         return FATHOM_EINVAL;
     if (!device_status_ptr()) return FATHOM_ECUDA;
-    return to_status(launch_topk(scores, n, ld, n_rows, k, idx, top_scores, workspace, (cudaStream_t)stream));
+    cudaStream_t s = (cudaStream_t)stream;
+    if (block_max)
+        return to_status(launch_topk_blocks(scores, block_max, n, ld, n_rows, k, idx, top_scores, workspace, s));
+    return to_status(launch_topk(scores, n, ld, n_rows, k, idx, top_scores, workspace, s));
 }
 
 int fathom_topk_merge(const float* cand_scores, const int32_t* cand_idx, int n_rows, int n_cand, int k, int32_t* idx,
@@ -201,8 +208,7 @@ int fathom_topk_merge(const float* cand_scores, const int32_t* cand_idx, int n_r
 
 size_t fathom_scan_workspace_bytes(const fathom_store* store, int n_q_heads, int k) {
     if (!store || n_q_heads < 1 || k < 1 || k > kMaxTopK || store->n < 1) return 0;
-    size_t scores = ((sizeof(float) * (size_t)n_q_heads * (size_t)n_pad_of(store->n)) + 255) & ~size_t(255);
-    return scores + topk_workspace_bytes(store->n, n_q_heads, k);
+    return scan_topk_layout(store->n, n_q_heads, n_q_heads).total;
 }
 
 int fathom_scan_topk(const fathom_store* store, const void* q, int q_dtype, const uint8_t* depths, int n_q_heads,
@@ -224,13 +230,14 @@ int fathom_scan_topk(const fathom_store* store, const void* q, int q_dtype, cons
     if (!device_status_ptr()) return FATHOM_ECUDA;
     float* scores = static_cast<float*>(workspace);
     const int64_t ld = n_pad_of(store->n);   // score row stride
-    size_t off = ((sizeof(float) * (size_t)n_q_heads * (size_t)ld) + 255) & ~size_t(255);
+    const ScanTopkLayout lay = scan_topk_layout(store->n, n_q_heads, n_q_heads);
+    uint32_t* bmax = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + lay.bmax_off);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = launch_scan(planes, scales, store->n_kv_heads, store->d, store->n, store->n_pad, q, q_dtype,
-                                depths, n_q_heads, scores, s);
+                                depths, n_q_heads, scores, s, bmax);
     if (e != cudaSuccess) return FATHOM_ECUDA;
-    e = launch_topk(scores, store->n, ld, n_q_heads, k, idx, top_scores,
-                    static_cast<char*>(workspace) + off, s);
+    e = launch_topk_blocks(scores, bmax, store->n, ld, n_q_heads, k, idx, top_scores,
+                           static_cast<char*>(workspace) + lay.topk_off, s);
     return to_status(e);
 }
 
@@ -255,9 +262,7 @@ size_t fathom_scan_batched_workspace_bytes(const fathom_store* stores, int n_ses
     if (n_q_heads < 1 || k < 1 || k > kMaxTopK) return 0;
     const size_t sb = batched_score_bytes(stores, n_sessions, n_q_heads);
     if (sb == 0) return 0;
-    int64_t max_n = 0;
-    for (int s = 0; s < n_sessions; ++s) max_n = stores[s].n > max_n ? stores[s].n : max_n;
-    return sb + topk_workspace_bytes(max_n, n_sessions * n_q_heads, k);
+    return sb + a256(sb / kBlock) + topk_blocks_workspace_bytes(n_sessions * n_q_heads);
 }
 
 int fathom_scan_topk_batched(const fathom_store* stores, int n_sessions, const void* q, int q_dtype,
@@ -304,11 +309,14 @@ int fathom_scan_topk_batched(const fathom_store* stores, int n_sessions, const v
     if (!scan_fits(stores[0].d, n_q_heads, stores[0].n_kv_heads)) return FATHOM_EUNSUPPORTED;
     if (!device_status_ptr()) return FATHOM_ECUDA;
     float* scores = static_cast<float*>(workspace);
+    // block maxima after all sessions' scores: session s's rows at score_base[s] / 64
+    uint32_t* bmax = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + off);
     cudaStream_t cs = (cudaStream_t)stream;
-    cudaError_t e = launch_scan_batched(sm, stores[0].n_kv_heads, stores[0].d, q, q_dtype, depths, n_q_heads, scores, cs);
+    cudaError_t e = launch_scan_batched(sm, stores[0].n_kv_heads, stores[0].d, q, q_dtype, depths, n_q_heads, scores,
+                                        cs, bmax);
     if (e != cudaSuccess) return FATHOM_ECUDA;
-    return to_status(launch_topk_map(scores, rm, n_sessions * n_q_heads, k, idx, top_scores,
-                                     static_cast<char*>(workspace) + off, cs));
+    return to_status(launch_topk_blocks_map(scores, bmax, rm, n_sessions * n_q_heads, k, idx, top_scores,
+                                            static_cast<char*>(workspace) + off + a256(off / kBlock), cs));
 }
 
 int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,

@@ -51,12 +51,11 @@ Aux* aux_for_device() {
     return &a;
 }
 
-inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
-
 }  // namespace
 
 size_t decode_workspace_bytes(int64_t n, int Hq, int groups, int k) {
-    return a256(sizeof(float) * (size_t)Hq * (size_t)n_pad_of(n)) + topk_workspace_bytes(n, Hq / groups, k);
+    (void)k;
+    return scan_topk_layout(n, Hq, Hq / groups).total;
 }
 
 cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n, int64_t n_pad,
@@ -70,7 +69,9 @@ cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hk
     const size_t q_elt = (q_dtype == FATHOM_BF16) ? 2 : 4;
     float* scores = static_cast<float*>(workspace);
     const int64_t ld = n_pad_of(n);   // score row stride; n_pad is the store's row stride
-    void* topk_ws = static_cast<char*>(workspace) + a256(sizeof(float) * (size_t)Hq * (size_t)ld);
+    const ScanTopkLayout lay = scan_topk_layout(n, Hq, hq_g);
+    uint32_t* bmax = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + lay.bmax_off);
+    void* topk_ws = static_cast<char*>(workspace) + lay.topk_off;
 
     cudaError_t e = launch_depths(q, q_dtype, sigma2, Hq, Hkv, d, budget, fixed_r, depths, stream);
     if (e != cudaSuccess) return e;
@@ -79,14 +80,15 @@ cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hk
         const int g0 = i * hkv_g, h0 = i * hq_g;
         const void* qi = static_cast<const char*>(q) + q_elt * (size_t)h0 * d;
         float* si = scores + (size_t)h0 * ld;
+        uint32_t* bi = bmax + (size_t)h0 * (ld / kBlock);
         e = launch_scan(planes + (size_t)g0 * d * 4 * (n_pad / 32), scales + (size_t)g0 * d * (n_pad / kBlock),
-                        hkv_g, d, n, n_pad, qi, q_dtype, depths + (size_t)h0 * d, hq_g, si, stream);
+                        hkv_g, d, n, n_pad, qi, q_dtype, depths + (size_t)h0 * d, hq_g, si, stream, bi);
         if (e == cudaSuccess) e = cudaEventRecord(aux->scanned[i], stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(aux->stream, aux->scanned[i], 0);
         int32_t* ii = idx + (size_t)h0 * k;
         float* ti = top_scores ? top_scores + (size_t)h0 * k : nullptr;
         const size_t rows_off = (size_t)g0 * rows_n * row_stride;
-        if (e == cudaSuccess) e = launch_topk(si, n, ld, hq_g, k, ii, ti, topk_ws, aux->stream);
+        if (e == cudaSuccess) e = launch_topk_blocks(si, bi, n, ld, hq_g, k, ii, ti, topk_ws, aux->stream);
         if (e == cudaSuccess)
             e = launch_attend(qi, q_dtype, K_rows + rows_off, V_rows + rows_off, row_stride, ii, hq_g, hkv_g, rows_n,
                               d, k, rows_host, out + (size_t)h0 * d, aux->stream);

@@ -43,9 +43,11 @@ cudaError_t launch_pack_blocks(const void* K, int k_dtype, int Hkv, int64_t rows
 cudaError_t launch_depths(const void* q, int q_dtype, const float* sigma2, int Hq, int Hkv, int d,
                           int budget, int fixed_r, uint8_t* depths, cudaStream_t stream, int pooled = 0);
 size_t scan_smem_bytes(int d, int G);
+// bmax (optional): the max score of every 64-key block as an ordered key,
+// [Hq][n_pad_of(n)/64], for launch_topk_blocks
 cudaError_t launch_scan(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n,
                         int64_t n_pad, const void* q, int q_dtype, const uint8_t* depths, int Hq,
-                        float* scores, cudaStream_t stream);
+                        float* scores, cudaStream_t stream, uint32_t* bmax = nullptr);
 size_t topk_workspace_bytes(int64_t n, int rows, int k);
 
 // Where the score rows are: rows are grouped in sets of `rows_per_set`
@@ -62,6 +64,26 @@ struct RowMap {
 };
 cudaError_t launch_topk(const float* scores, int64_t n, int64_t ld, int rows, int k, int32_t* idx,
                         float* top_scores, void* ws, cudaStream_t stream);
+// top-k of score rows whose 64-key block maxima (ordered keys, [row][ld/64])
+// the scan wrote alongside; ld a multiple of 64 and base offsets too
+size_t topk_blocks_workspace_bytes(int rows);
+
+// Workspace of a scan followed by the block-maximum top-k: scores
+// f32 [Hq][n_pad_of(n)], block maxima u32 [Hq][n_pad_of(n)/64], the top-k
+// buffers for `topk_rows` rows; each part 256-byte aligned.
+struct ScanTopkLayout {
+    size_t bmax_off, topk_off, total;
+};
+inline ScanTopkLayout scan_topk_layout(int64_t n, int Hq, int topk_rows) {
+    const size_t ld = (size_t)n_pad_of(n);
+    const size_t sb = (sizeof(float) * (size_t)Hq * ld + 255) & ~size_t(255);
+    const size_t bb = (sizeof(uint32_t) * (size_t)Hq * (ld / kBlock) + 255) & ~size_t(255);
+    return {sb, sb + bb, sb + bb + topk_blocks_workspace_bytes(topk_rows)};
+}
+cudaError_t launch_topk_blocks(const float* scores, const uint32_t* bmax, int64_t n, int64_t ld, int rows, int k,
+                               int32_t* idx, float* top_scores, void* ws, cudaStream_t stream);
+cudaError_t launch_topk_blocks_map(const float* scores, const uint32_t* bmax, const RowMap& map, int rows, int k,
+                                   int32_t* idx, float* top_scores, void* ws, cudaStream_t stream);
 cudaError_t launch_topk_merge(const float* cand_scores, const int32_t* cand_idx, int rows, int n_cand, int k,
                               int32_t* idx, float* top_scores, void* ws, cudaStream_t stream);
 cudaError_t launch_topk_map(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
@@ -79,7 +101,8 @@ struct SessionMap {
     int tile0[kMaxSets + 1];
 };
 cudaError_t launch_scan_batched(const SessionMap& map, int Hkv, int d, const void* q, int q_dtype,
-                                const uint8_t* depths, int Hq, float* scores, cudaStream_t stream);
+                                const uint8_t* depths, int Hq, float* scores, cudaStream_t stream,
+                                uint32_t* bmax = nullptr);
 size_t decode_workspace_bytes(int64_t n, int Hq, int groups, int k);
 cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n, int64_t n_pad,
                           const void* q, int q_dtype, const float* sigma2, int Hq, int budget, int fixed_r, int k,

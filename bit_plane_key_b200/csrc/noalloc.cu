@@ -76,15 +76,17 @@ int fathom_scan_topk_noalloc(const fathom_store* store, const void* q, int q_dty
     if (!device_status_ptr()) return FATHOM_ECUDA;
     char* scratch = static_cast<char*>(scratch_address());
     if (!scratch) return FATHOM_ECUDA;
-    // same split as fathom_scan_topk: scores [Hq][n_pad_of(n)], then the top-k buffers
+    // same split as fathom_scan_topk: scores [Hq][n_pad_of(n)], block maxima, then the top-k buffers
     float* scores = reinterpret_cast<float*>(scratch);
     const int64_t ld = n_pad_of(store->n);
-    const size_t off = ((sizeof(float) * (size_t)n_q_heads * (size_t)ld) + 255) & ~size_t(255);
+    const ScanTopkLayout lay = scan_topk_layout(store->n, n_q_heads, n_q_heads);
+    uint32_t* bmax = reinterpret_cast<uint32_t*>(scratch + lay.bmax_off);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = launch_scan(planes, scales, store->n_kv_heads, store->d, store->n, store->n_pad, q, q_dtype,
-                                depths, n_q_heads, scores, s);
+                                depths, n_q_heads, scores, s, bmax);
     if (e != cudaSuccess) return FATHOM_ECUDA;
-    return to_status(launch_topk(scores, store->n, ld, n_q_heads, k, idx, top_scores, scratch + off, s));
+    return to_status(launch_topk_blocks(scores, bmax, store->n, ld, n_q_heads, k, idx, top_scores,
+                                        scratch + lay.topk_off, s));
 }
 
 }  // extern "C"

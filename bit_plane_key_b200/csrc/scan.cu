@@ -110,7 +110,7 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
                                           int d, int64_t n, int64_t n_pad, int tile, int g,
                                           const void* __restrict__ q, int q_dtype,
                                           const uint8_t* __restrict__ depths, float* __restrict__ scores,
-                                          unsigned int* status) {
+                                          uint32_t* __restrict__ bmax, unsigned int* status) {
     using Z = Geo<G>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const ScanSmem lay{d, G};
@@ -126,6 +126,7 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
     uint8_t* s_U = smem_raw + lay.uni();
     uint8_t* s_t = smem_raw + lay.tdep();
     __shared__ int s_L;
+    __shared__ uint32_t s_bmax[8 * kTileBlocks];   // per (head, block) max score as an ordered key; G <= 8
     const int off_stride = d / 8 + 4;
 
     const int64_t tile0 = (int64_t)tile * kTileKeys;
@@ -138,6 +139,7 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     // ---- plan: depths, union list, row pointers, per-head item lists, per-(channel, head) factors ----
+    for (int e = tid; e < G * kTileBlocks; e += Z::T) s_bmax[e] = 0u;   // below every ordered key
     for (int e = tid; e < G * d; e += Z::T) {
         int t = depths[(int64_t)g * G * d + e];
         if (t > 4) {
@@ -352,6 +354,7 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
         float* out = scores + ((int64_t)g * G + h) * n_pad_of(n) + k0;
         const float cst = s_cst[h * 16 + b];
         const bool whole = tile0 + kTileKeys <= n;
+        uint32_t kmax = 0u;
 #pragma unroll
         for (int i = 0; i < Z::NSV; ++i)
 #pragma unroll
@@ -359,9 +362,18 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int o = 32 * wd + i + 8 * k;
-                    const float v = acc[i][wd][k] + cst;
-                    out[o] = (whole || k0 + o < n) ? v : -INFINITY;
+                    const float v = (whole || k0 + o < n) ? acc[i][wd][k] + cst : -INFINITY;
+                    out[o] = v;
+                    kmax = max(kmax, float_to_ordered(v));
                 }
+        atomicMax(&s_bmax[h * kTileBlocks + b], kmax);
+    }
+    // the maximum of every 64-key block, for the top-k that reads only the
+    // blocks that can hold a selected key
+    __syncthreads();
+    if (bmax && tid < G * kTileBlocks) {
+        const int hh = tid / kTileBlocks, bb = tid % kTileBlocks;
+        bmax[((int64_t)g * G + hh) * (n_pad_of(n) / kBlock) + tile0 / kBlock + bb] = s_bmax[tid];
     }
 }
 
@@ -369,15 +381,17 @@ template <int G>
 __global__ void __launch_bounds__(Geo<G>::T, Geo<G>::MinBlocks)
 scan_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ scales, int d, int64_t n,
             int64_t n_pad, const void* __restrict__ q, int q_dtype, const uint8_t* __restrict__ depths,
-            float* __restrict__ scores, unsigned int* status) {
-    scan_tile<G>(planes, scales, d, n, n_pad, (int)blockIdx.x, (int)blockIdx.y, q, q_dtype, depths, scores, status);
+            float* __restrict__ scores, uint32_t* __restrict__ bmax, unsigned int* status) {
+    scan_tile<G>(planes, scales, d, n, n_pad, (int)blockIdx.x, (int)blockIdx.y, q, q_dtype, depths, scores, bmax,
+                 status);
 }
 
 // Batched sessions: blockIdx.x runs over the tiles of all sessions.
 template <int G>
 __global__ void __launch_bounds__(Geo<G>::T, Geo<G>::MinBlocks)
 scan_batched_kernel(const __grid_constant__ SessionMap map, int d, int Hq, const void* __restrict__ q, int q_dtype,
-                    const uint8_t* __restrict__ depths, float* __restrict__ scores, unsigned int* status) {
+                    const uint8_t* __restrict__ depths, float* __restrict__ scores, uint32_t* __restrict__ bmax,
+                    unsigned int* status) {
     const int t = (int)blockIdx.x;
     int lo = 0, hi = map.nsess - 1;   // last session with tile0 <= t
     while (lo < hi) {
@@ -391,32 +405,33 @@ scan_batched_kernel(const __grid_constant__ SessionMap map, int d, int Hq, const
                          ? static_cast<const void*>(static_cast<const uint16_t*>(q) + sidx * qstride)
                          : static_cast<const void*>(static_cast<const float*>(q) + sidx * qstride);
     scan_tile<G>(map.planes[sidx], map.scales[sidx], d, map.n[sidx], map.n_pad[sidx], t - map.tile0[sidx],
-                 (int)blockIdx.y, qs, q_dtype, depths + sidx * qstride, scores + map.score_base[sidx], status);
+                 (int)blockIdx.y, qs, q_dtype, depths + sidx * qstride, scores + map.score_base[sidx],
+                 bmax ? bmax + map.score_base[sidx] / kBlock : nullptr, status);
 }
 
 template <int G>
 cudaError_t launch_scan_g(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n,
                           int64_t n_pad, const void* q, int q_dtype, const uint8_t* depths, float* scores,
-                          cudaStream_t stream) {
+                          uint32_t* bmax, cudaStream_t stream) {
     const size_t smem = ScanSmem{d, G}.bytes();
     auto kern = scan_kernel<G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)(n_pad_of(n) / kTileKeys), (unsigned)Hkv);   // the tiles holding keys; n_pad is the stride
-    kern<<<grid, Geo<G>::T, smem, stream>>>(planes, scales, d, n, n_pad, q, q_dtype, depths, scores,
+    kern<<<grid, Geo<G>::T, smem, stream>>>(planes, scales, d, n, n_pad, q, q_dtype, depths, scores, bmax,
                                             device_status_ptr());
     return cudaGetLastError();
 }
 
 template <int G>
 cudaError_t launch_scan_batched_g(const SessionMap& map, int Hkv, int d, const void* q, int q_dtype,
-                                  const uint8_t* depths, int Hq, float* scores, cudaStream_t stream) {
+                                  const uint8_t* depths, int Hq, float* scores, uint32_t* bmax, cudaStream_t stream) {
     const size_t smem = ScanSmem{d, G}.bytes();
     auto kern = scan_batched_kernel<G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)map.tile0[map.nsess], (unsigned)Hkv);
-    kern<<<grid, Geo<G>::T, smem, stream>>>(map, d, Hq, q, q_dtype, depths, scores, device_status_ptr());
+    kern<<<grid, Geo<G>::T, smem, stream>>>(map, d, Hq, q, q_dtype, depths, scores, bmax, device_status_ptr());
     return cudaGetLastError();
 }
 
@@ -426,23 +441,23 @@ size_t scan_smem_bytes(int d, int G) { return ScanSmem{d, G}.bytes(); }
 
 cudaError_t launch_scan(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n, int64_t n_pad,
                         const void* q, int q_dtype, const uint8_t* depths, int Hq, float* scores,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, uint32_t* bmax) {
     switch (Hq / Hkv) {
-        case 1: return launch_scan_g<1>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, stream);
-        case 2: return launch_scan_g<2>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, stream);
-        case 4: return launch_scan_g<4>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, stream);
-        case 8: return launch_scan_g<8>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, stream);
+        case 1: return launch_scan_g<1>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
+        case 2: return launch_scan_g<2>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
+        case 4: return launch_scan_g<4>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
+        case 8: return launch_scan_g<8>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_scan_batched(const SessionMap& map, int Hkv, int d, const void* q, int q_dtype,
-                                const uint8_t* depths, int Hq, float* scores, cudaStream_t stream) {
+                                const uint8_t* depths, int Hq, float* scores, cudaStream_t stream, uint32_t* bmax) {
     switch (Hq / Hkv) {
-        case 1: return launch_scan_batched_g<1>(map, Hkv, d, q, q_dtype, depths, Hq, scores, stream);
-        case 2: return launch_scan_batched_g<2>(map, Hkv, d, q, q_dtype, depths, Hq, scores, stream);
-        case 4: return launch_scan_batched_g<4>(map, Hkv, d, q, q_dtype, depths, Hq, scores, stream);
-        case 8: return launch_scan_batched_g<8>(map, Hkv, d, q, q_dtype, depths, Hq, scores, stream);
+        case 1: return launch_scan_batched_g<1>(map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream);
+        case 2: return launch_scan_batched_g<2>(map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream);
+        case 4: return launch_scan_batched_g<4>(map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream);
+        case 8: return launch_scan_batched_g<8>(map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -505,6 +505,207 @@ topk_finish(const float* __restrict__ scores, const __grid_constant__ RowMap m, 
     }
 }
 
+// ---------------------------------------------------------------------------
+// Top-k from block maxima.  The scan also writes, for every 64-key block, the
+// largest score of the block (as an ordered key).  With m = the k-th largest
+// block maximum of a row, k distinct keys (each block's maximum) score at
+// least m, so the k-th largest score T >= m, and every key at or above T lies
+// in a block whose maximum is >= m: only those blocks (about k of them) are
+// read.  Kernels: threshold (m per row), compact (the keys >= m of the
+// surviving blocks), finish (the exact T among them, the sure keys and ties,
+// sorted).  A row whose candidates overflow the buffer (e.g. all scores
+// equal) is finished from its full row instead, with the same exact rules.
+// ---------------------------------------------------------------------------
+constexpr int kCapB = 16384;   // candidates per row on the block path
+
+struct BlkWs {
+    RowState* state;   // [rows]: prefix = m, n_cand, pad bit 0 = candidate overflow
+    uint64_t* cand;    // [rows][kCapB]
+};
+
+BlkWs carve_blk(void* ws, int rows) {
+    BlkWs w;
+    char* p = static_cast<char*>(ws);
+    w.state = reinterpret_cast<RowState*>(p);
+    p += align256(sizeof(RowState) * rows);
+    w.cand = reinterpret_cast<uint64_t*>(p);
+    return w;
+}
+
+// The exact need-th largest of cnt ordered keys key_at(0..cnt) (1 <= need <=
+// cnt): radix steps of 12, 12 and 8 bits with a shared-memory histogram.
+// Returns T; *gt = keys above T, *eq = keys equal to T.  All threads of a
+// kFinishThreads block call it and get the result.
+template <class KeyAt>
+__device__ uint32_t block_kth_key(KeyAt key_at, int64_t cnt, uint32_t need, uint32_t* hist, int* s_bin,
+                                  uint32_t* s_above, uint32_t* s_cnt, uint32_t* warp_tot, uint32_t* gt, uint32_t* eq) {
+    uint32_t prefix = 0, above = 0;
+    int shift = 32;
+    while (shift > 0) {
+        const int nbits = shift >= 12 ? 12 : shift, sh = shift - nbits, nb = 1 << nbits;
+        for (int b = threadIdx.x; b < nb; b += blockDim.x) hist[b] = 0;
+        __syncthreads();
+        for (int64_t e = threadIdx.x; e < cnt; e += blockDim.x) {
+            const uint32_t key = key_at(e);
+            if (shift == 32 || (key >> shift) == prefix) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1u);
+        }
+        __syncthreads();
+        block_pick_bin(hist, nb, need, s_bin, s_above, s_cnt, warp_tot);
+        need -= *s_above;
+        above += *s_above;
+        prefix = (shift == 32 ? 0u : (prefix << nbits)) | (uint32_t)*s_bin;
+        shift = sh;
+        __syncthreads();   // s_bin / s_above are rewritten by the next step
+    }
+    *gt = above;
+    *eq = *s_cnt;
+    return prefix;
+}
+
+__global__ void __launch_bounds__(kFinishThreads)
+topk_blk_threshold(const uint32_t* __restrict__ bmax, const __grid_constant__ RowMap m, int k, BlkWs w) {
+    __shared__ uint32_t hist[kBins];
+    __shared__ uint32_t warp_tot[32];
+    __shared__ int s_bin;
+    __shared__ uint32_t s_above, s_cnt;
+    const int row = blockIdx.x;
+    int64_t off, n;
+    row_span(m, row, &off, &n);
+    const uint32_t* bm = bmax + off / kBlock;
+    const int64_t nreal = (n + kBlock - 1) / kBlock;
+    uint32_t mkey = 0;   // fewer blocks than k: every key is a candidate
+    if (k <= nreal) {
+        uint32_t gt, eq;
+        mkey = block_kth_key([&](int64_t e) { return bm[e]; }, nreal, (uint32_t)k, hist, &s_bin, &s_above, &s_cnt,
+                             warp_tot, &gt, &eq);
+    }
+    if (threadIdx.x == 0) {
+        RowState s;
+        s.prefix = mkey;
+        s.shift = 0;
+        s.count_above = 0;
+        s.cand = 0;
+        s.phase = 1;
+        s.n_sure = 0;
+        s.n_cand = 0;
+        s.pad = 0;
+        w.state[row] = s;
+    }
+}
+
+// Thread t of CTA x looks at block j = 256 x + t; a warp then reads each of
+// its surviving blocks (64 scores, two per lane) and keeps the keys >= m.
+__global__ void __launch_bounds__(kPassThreads)
+topk_blk_compact(const float* __restrict__ scores, const uint32_t* __restrict__ bmax, const __grid_constant__ RowMap m,
+                 BlkWs w) {
+    const int row = blockIdx.y;
+    int64_t off, n;
+    row_span(m, row, &off, &n);
+    const int64_t nreal = (n + kBlock - 1) / kBlock;
+    const uint32_t mkey = w.state[row].prefix;
+    const uint32_t* bm = bmax + off / kBlock;
+    const float* s = scores + off;
+    RowState* gst = w.state + row;
+    const int lane = threadIdx.x & 31;
+    const int64_t j = (int64_t)blockIdx.x * kPassThreads + threadIdx.x;
+    const bool surv = j < nreal && bm[j] >= mkey;
+    unsigned sm = __ballot_sync(0xffffffffu, surv);
+    const unsigned lower = (1u << lane) - 1u;
+    const int64_t j0 = j - lane;
+    while (sm) {   // warp-uniform
+        const int src = __ffs(sm) - 1;
+        sm &= sm - 1;
+        const int64_t i0 = (j0 + src) * kBlock;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int64_t i = i0 + half * 32 + lane;
+            const uint32_t key = (i < n) ? float_to_ordered(s[i]) : 0u;
+            const bool keep = i < n && key >= mkey;
+            const unsigned km = __ballot_sync(0xffffffffu, keep);
+            if (!km) continue;
+            int base = 0;
+            if (lane == 0) base = atomicAdd(&gst->n_cand, __popc(km));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (keep) {
+                const int slot = base + __popc(km & lower);
+                if (slot < kCapB) w.cand[(size_t)row * kCapB + slot] = composite(key, i);
+                else atomicOr(&gst->pad, 1);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kFinishThreads)
+topk_blk_finish(const float* __restrict__ scores, const __grid_constant__ RowMap m, int k, BlkWs w,
+                int32_t* __restrict__ idx, float* __restrict__ top_scores) {
+    extern __shared__ uint64_t buf[];
+    __shared__ uint32_t hist[kBins];
+    __shared__ uint32_t warp_tot[32];
+    __shared__ int warp_cnt[32];
+    __shared__ int s_bin, s_fill, s_got;
+    __shared__ uint32_t s_above, s_cnt;
+    const int row = blockIdx.x;
+    const RowState st = w.state[row];
+    int64_t off, n;
+    row_span(m, row, &off, &n);
+    const float* s = scores + off;
+    const uint64_t* cand = w.cand + (size_t)row * kCapB;
+    const bool use_cand = !(st.pad & 1);   // else the candidates overflowed: use the full row
+    const int64_t cnt = use_cand ? (int64_t)min(st.n_cand, kCapB) : n;
+    auto key_at = [&](int64_t e) -> uint32_t {
+        return use_cand ? (uint32_t)(cand[e] >> 32) : float_to_ordered(s[e]);
+    };
+    uint32_t gt, eq;
+    const uint32_t T = block_kth_key(key_at, cnt, (uint32_t)k, hist, &s_bin, &s_above, &s_cnt, warp_tot, &gt, &eq);
+    const bool ties_fit = gt + eq <= (uint32_t)kSortMax;
+    if (threadIdx.x == 0) s_fill = 0;
+    __syncthreads();
+    for (int64_t e = threadIdx.x; e < cnt; e += blockDim.x) {
+        const uint32_t key = key_at(e);
+        if (key > T || (ties_fit && key == T)) buf[atomicAdd(&s_fill, 1)] = use_cand ? cand[e] : composite(key, e);
+    }
+    __syncthreads();
+    int total = s_fill;
+    if (!ties_fit) {
+        // more keys tie at T than the sort holds: take the lowest indices, in order
+        const int ns = (int)gt, r = k - ns;
+        if (threadIdx.x == 0) s_got = 0;
+        __syncthreads();
+        const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+        for (int64_t base = 0; base < n; base += blockDim.x) {
+            const int got = s_got;
+            if (got >= r) break;
+            const int64_t i = base + threadIdx.x;
+            const bool f = (i < n) && float_to_ordered(s[i]) == T;
+            const unsigned msk = __ballot_sync(0xffffffffu, f);
+            if (lane == 0) warp_cnt[wp] = __popc(msk);
+            __syncthreads();
+            int before = 0;
+            for (int x = 0; x < wp; ++x) before += warp_cnt[x];
+            const int rank = got + before + __popc(msk & ((1u << lane) - 1u));
+            if (f && rank < r) buf[ns + rank] = composite(T, i);
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                int add = 0;
+                for (int x = 0; x < (int)(blockDim.x >> 5); ++x) add += warp_cnt[x];
+                s_got = got + add;
+            }
+            __syncthreads();
+        }
+        total = k;
+    }
+    int S = 1;
+    while (S < total) S <<= 1;
+    for (int e = total + threadIdx.x; e < S; e += blockDim.x) buf[e] = 0ull;
+    __syncthreads();
+    bitonic_desc(buf, S);
+    for (int e = threadIdx.x; e < k; e += blockDim.x) {
+        const uint64_t c = buf[e];
+        idx[(int64_t)row * k + e] = (int32_t)(0xFFFFFFFFu - (uint32_t)c);
+        if (top_scores) top_scores[(int64_t)row * k + e] = ordered_to_float((uint32_t)(c >> 32));
+    }
+}
+
 // positions into the gathered candidate lists -> the candidates' global indices
 __global__ void topk_map_positions(const int32_t* __restrict__ cand_idx, int n_cand, int k, int32_t* idx) {
     const int row = blockIdx.y;
@@ -523,6 +724,36 @@ cudaError_t launch_topk_merge(const float* cand_scores, const int32_t* cand_idx,
     topk_map_positions<<<dim3((unsigned)((k + 255) / 256), (unsigned)rows), 256, 0, stream>>>(cand_idx, n_cand, k,
                                                                                              idx);
     return cudaGetLastError();
+}
+
+size_t topk_blocks_workspace_bytes(int rows) {
+    return align256(sizeof(RowState) * rows) + align256(sizeof(uint64_t) * (size_t)rows * kCapB);
+}
+
+cudaError_t launch_topk_blocks_map(const float* scores, const uint32_t* bmax, const RowMap& map, int rows, int k,
+                                   int32_t* idx, float* top_scores, void* ws, cudaStream_t stream) {
+    BlkWs w = carve_blk(ws, rows);
+    topk_blk_threshold<<<rows, kFinishThreads, 0, stream>>>(bmax, map, k, w);
+    const int64_t nbk = (map.max_n + kBlock - 1) / kBlock;
+    topk_blk_compact<<<dim3((unsigned)((nbk + kPassThreads - 1) / kPassThreads), rows), kPassThreads, 0, stream>>>(
+        scores, bmax, map, w);
+    const size_t smem = sizeof(uint64_t) * kSortMax;
+    cudaError_t e = cudaFuncSetAttribute(topk_blk_finish, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    topk_blk_finish<<<rows, kFinishThreads, smem, stream>>>(scores, map, k, w, idx, top_scores);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk_blocks(const float* scores, const uint32_t* bmax, int64_t n, int64_t ld, int rows, int k,
+                               int32_t* idx, float* top_scores, void* ws, cudaStream_t stream) {
+    RowMap m;
+    m.rows_per_set = rows;
+    m.nsets = 1;
+    m.max_n = n;
+    m.base[0] = 0;
+    m.ld[0] = ld;
+    m.n[0] = n;
+    return launch_topk_blocks_map(scores, bmax, m, rows, k, idx, top_scores, ws, stream);
 }
 
 size_t topk_workspace_bytes(int64_t n, int rows, int k) {

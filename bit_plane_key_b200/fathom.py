@@ -57,9 +57,9 @@ _sig("fathom_alloc_depths", _I, [_P, _I, _P, _I, _I, _I, _I, _I, _P, _P])
 _sig("fathom_alloc_depths_pooled", _I, [_P, _I, _P, _I, _I, _I, _I, _P, _P])
 _sig("fathom_append_keys", _I, [_SP, _P, _I, _L, _P])
 _sig("fathom_topk_merge", _I, [_P, _P, _I, _I, _I, _P, _P, _P, _Z, _P])
-_sig("fathom_scan_scores", _I, [_SP, _P, _I, _P, _I, _P, _P])
+_sig("fathom_scan_scores", _I, [_SP, _P, _I, _P, _I, _P, _P, _P])
 _sig("fathom_topk_workspace_bytes", _Z, [_L, _I, _I])
-_sig("fathom_topk", _I, [_P, _L, _L, _I, _I, _P, _P, _P, _Z, _P])
+_sig("fathom_topk", _I, [_P, _P, _L, _L, _I, _I, _P, _P, _P, _Z, _P])
 _sig("fathom_scan_workspace_bytes", _Z, [_SP, _I, _I])
 _sig("fathom_scan_topk", _I, [_SP, _P, _I, _P, _I, _I, _P, _P, _P, _Z, _P])
 _sig("fathom_sparse_attend", _I, [_P, _I, _P, _P, _L, _I, _P, _I, _I, _L, _I, _I, _P, _P])
@@ -190,22 +190,29 @@ def alloc_depths_pooled(q, sigma2, budget_bits, out=None, stream=None):
     return out
 
 
-def scan_scores(store, q, depths, out=None, stream=None):
-    """Scores f32 [Hq][n_pad] (padding keys -inf)."""
+def scan_scores(store, q, depths, out=None, block_max=None, stream=None):
+    """Scores f32 [Hq][n_pad(n)] (padding keys -inf); block_max (optional) u32
+    [Hq][n_pad(n)/64] receives the block maxima that topk() can use."""
     Hq = q.shape[0]
     if out is None:
         out = torch.empty((Hq, n_pad(store.n)), dtype=torch.float32, device=q.device)
-    _check(_lib.fathom_scan_scores(store.c, _ptr(q), _dtype_code(q), _ptr(depths), Hq, _ptr(out),
+    _check(_lib.fathom_scan_scores(store.c, _ptr(q), _dtype_code(q), _ptr(depths), Hq, _ptr(out), _ptr(block_max),
                                    _stream(stream)), "fathom_scan_scores")
     return out
+
+
+def block_max_buffer(n_rows, n, device):
+    """A block-maxima buffer for scan_scores / topk: u32 (as int32) [rows][n_pad(n)/64]."""
+    return torch.empty((n_rows, n_pad(n) // 64), dtype=torch.int32, device=device)
 
 
 def topk_workspace_bytes(n, rows, k):
     return int(_lib.fathom_topk_workspace_bytes(int(n), int(rows), int(k)))
 
 
-def topk(scores, n, k, idx=None, top_scores=None, workspace=None, stream=None):
-    """Top-k of score rows [rows][ld] over the first n columns."""
+def topk(scores, n, k, idx=None, top_scores=None, workspace=None, block_max=None, stream=None):
+    """Top-k of score rows [rows][ld] over the first n columns (block_max: the
+    block maxima the scan wrote with these scores, or None)."""
     rows, ld = scores.shape
     if idx is None:
         idx = torch.empty((rows, k), dtype=torch.int32, device=scores.device)
@@ -214,8 +221,8 @@ def topk(scores, n, k, idx=None, top_scores=None, workspace=None, stream=None):
     nb = topk_workspace_bytes(n, rows, k)
     if workspace is None:
         workspace = torch.empty(max(nb, 1), dtype=torch.uint8, device=scores.device)
-    _check(_lib.fathom_topk(_ptr(scores), int(n), int(ld), rows, int(k), _ptr(idx), _ptr(top_scores),
-                            _ptr(workspace), workspace.numel(), _stream(stream)), "fathom_topk")
+    _check(_lib.fathom_topk(_ptr(scores), _ptr(block_max), int(n), int(ld), rows, int(k), _ptr(idx),
+                            _ptr(top_scores), _ptr(workspace), workspace.numel(), _stream(stream)), "fathom_topk")
     return idx, top_scores
 
 

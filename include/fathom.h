@@ -190,16 +190,24 @@ int fathom_alloc_depths_pooled(const void* q, int q_dtype, const float* sigma2, 
  *   q       device, [Hq][d], FATHOM_F32 or FATHOM_BF16.
  *   depths  device, u8 [Hq][d], values 0..4.
  *   scores  device, f32 [Hq][fathom_n_pad(store->n)]; keys >= n are written -inf.
+ *   block_max  NULL, or device u32 [Hq][fathom_n_pad(store->n)/64]: the largest
+ *           score of every 64-key block as an order-preserving key, for
+ *           fathom_topk to read only the blocks that can hold a selected key.
  * Errors: EINVAL as above, or a host-resident store whose pointers are not
  * page-locked, or a device store whose pointers are not device memory.
  */
 int fathom_scan_scores(const fathom_store* store, const void* q, int q_dtype, const uint8_t* depths,
-                       int n_q_heads, float* scores, fathom_stream_t stream);
+                       int n_q_heads, float* scores, uint32_t* block_max, fathom_stream_t stream);
 
 /*
  * Top-k of score rows: the k largest of scores[r][0..n), ties to the lower
  * index, listed in that order.  [ai-feeds summary 关键模块 5, 输出]
  *   scores      device, f32 [n_rows][ld] (ld >= n); NaN is not allowed.
+ *   block_max   NULL (select from the scores alone: histogram passes over
+ *               every row), or the block maxima that fathom_scan_scores wrote
+ *               with these scores (ld a multiple of 64): with m = the k-th
+ *               largest block maximum of a row, k keys score at least m, so
+ *               only the blocks whose maximum is >= m are read.
  *   idx         device, i32 [n_rows][k].
  *   top_scores  device, f32 [n_rows][k], or NULL.
  *   workspace   device, at least fathom_topk_workspace_bytes(n, n_rows, k) bytes,
@@ -208,8 +216,8 @@ int fathom_scan_scores(const fathom_store* store, const void* q, int q_dtype, co
  * workspace.
  */
 size_t fathom_topk_workspace_bytes(int64_t n, int n_rows, int k);
-int fathom_topk(const float* scores, int64_t n, int64_t ld, int n_rows, int k, int32_t* idx,
-                float* top_scores, void* workspace, size_t workspace_bytes, fathom_stream_t stream);
+int fathom_topk(const float* scores, const uint32_t* block_max, int64_t n, int64_t ld, int n_rows, int k,
+                int32_t* idx, float* top_scores, void* workspace, size_t workspace_bytes, fathom_stream_t stream);
 
 /*
  * Merge of per-shard top-k lists, for a key range split across GPUs (not on

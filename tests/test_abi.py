@@ -62,7 +62,7 @@ def test_null_arguments_rejected_before_any_cuda_call(libpath):
     L = F.lib()
     assert L.fathom_pack_bitplanes(None, 0, 1, 10, 32, None, None, None) == F.EINVAL
     assert L.fathom_alloc_depths(None, 0, None, 1, 1, 32, 10, 0, None, None) == F.EINVAL
-    assert L.fathom_topk(None, 10, 10, 1, 1, None, None, None, 0, None) == F.EINVAL
+    assert L.fathom_topk(None, None, 10, 10, 1, 1, None, None, None, 0, None) == F.EINVAL
     assert L.fathom_scan_topk(None, None, 0, None, 1, 1, None, None, None, 0, None) == F.EINVAL
     assert L.fathom_sparse_attend(None, 0, None, None, 128, 0, None, 1, 1, 10, 128, 1, None, None) == F.EINVAL
     assert L.fathom_decode_step(None, None, 0, None, 4, 92, 0, 16, None, None, 10, 128, 0, 1, None, None, None,

@@ -283,6 +283,28 @@ def test_topk_bit_exact(ref, n, rows, k, kind):
     assert F.last_device_status() == 0
 
 
+@pytest.mark.parametrize("n,B,k", [(20000, 92, 2048), (5000, 46, 700), (70000, 0, 1024), (131072, 136, 4096),
+                                    (3000, 92, 3000)])
+def test_topk_from_block_maxima_equals_full_selection(n, B, k):
+    """The scan's block maxima let top-k read only the blocks that can hold a
+    selected key; the result must equal the selection over the whole rows bit
+    for bit (B = 0: every score ties, the candidates overflow and the full-row
+    path takes the lowest indices)."""
+    inp = make(2, n=n, Hkv=2, Hq=8, layer=B)
+    st = F.pack_bitplanes(dev(inp["K"]))
+    dep = F.alloc_depths(q_dev(inp), dev(inp["sigma2"]), B)
+    bm = F.block_max_buffer(8, n, DEV)
+    sc = F.scan_scores(st, q_dev(inp), dep, block_max=bm)
+    i_blk, t_blk = F.topk(sc, n, k, block_max=bm)
+    i_all, t_all = F.topk(sc, n, k)
+    assert torch.equal(i_blk, i_all) and torch.equal(t_blk, t_all)
+    i_st, t_st = F.scan_topk(st, q_dev(inp), dep, k)
+    assert torch.equal(i_st, i_all) and torch.equal(t_st, t_all)
+    if B == 0:
+        assert np.array_equal(host(i_blk), np.tile(np.arange(k, dtype=np.int32), (8, 1)))
+    assert F.last_device_status() == 0
+
+
 @pytest.mark.parametrize("kind", ["normal", "ties", "narrow"])
 def test_topk_repeatable_under_load(ref, kind):
     """The same rows, 20 launches back to back with many rows in flight: every
