@@ -169,8 +169,7 @@ int fathom_scan_scores(const fathom_store* store, const void* q, int q_dtype, co
 
 size_t fathom_topk_workspace_bytes(int64_t n, int n_rows, int k) {
     if (n < 1 || n_rows < 1 || k < 1 || k > kMaxTopK) return 0;
-    const size_t a = topk_workspace_bytes(n, n_rows, k), b = topk_blocks_workspace_bytes(n_rows);
-    return a > b ? a : b;   // either path
+    return topk_any_workspace_bytes(n, n_rows, k);   // either path
 }
 
 int fathom_topk(const float* scores, const uint32_t* block_max, int64_t n, int64_t ld, int n_rows, int k,
@@ -208,7 +207,7 @@ int fathom_topk_merge(const float* cand_scores, const int32_t* cand_idx, int n_r
 
 size_t fathom_scan_workspace_bytes(const fathom_store* store, int n_q_heads, int k) {
     if (!store || n_q_heads < 1 || k < 1 || k > kMaxTopK || store->n < 1) return 0;
-    return scan_topk_layout(store->n, n_q_heads, n_q_heads).total;
+    return scan_topk_layout(store->n, n_q_heads, n_q_heads, k).total;
 }
 
 int fathom_scan_topk(const fathom_store* store, const void* q, int q_dtype, const uint8_t* depths, int n_q_heads,
@@ -230,7 +229,7 @@ int fathom_scan_topk(const fathom_store* store, const void* q, int q_dtype, cons
     if (!device_status_ptr()) return FATHOM_ECUDA;
     float* scores = static_cast<float*>(workspace);
     const int64_t ld = n_pad_of(store->n);   // score row stride
-    const ScanTopkLayout lay = scan_topk_layout(store->n, n_q_heads, n_q_heads);
+    const ScanTopkLayout lay = scan_topk_layout(store->n, n_q_heads, n_q_heads, k);
     uint32_t* bmax = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + lay.bmax_off);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = launch_scan(planes, scales, store->n_kv_heads, store->d, store->n, store->n_pad, q, q_dtype,
@@ -262,7 +261,9 @@ size_t fathom_scan_batched_workspace_bytes(const fathom_store* stores, int n_ses
     if (n_q_heads < 1 || k < 1 || k > kMaxTopK) return 0;
     const size_t sb = batched_score_bytes(stores, n_sessions, n_q_heads);
     if (sb == 0) return 0;
-    return sb + a256(sb / kBlock) + topk_blocks_workspace_bytes(n_sessions * n_q_heads);
+    int64_t max_n = 0;
+    for (int s = 0; s < n_sessions; ++s) max_n = stores[s].n > max_n ? stores[s].n : max_n;
+    return sb + a256(sb / kBlock) + topk_any_workspace_bytes(max_n, n_sessions * n_q_heads, k);
 }
 
 int fathom_scan_topk_batched(const fathom_store* stores, int n_sessions, const void* q, int q_dtype,

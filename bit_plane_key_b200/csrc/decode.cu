@@ -54,8 +54,7 @@ Aux* aux_for_device() {
 }  // namespace
 
 size_t decode_workspace_bytes(int64_t n, int Hq, int groups, int k) {
-    (void)k;
-    return scan_topk_layout(n, Hq, Hq / groups).total;
+    return scan_topk_layout(n, Hq, Hq / groups, k).total;
 }
 
 cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n, int64_t n_pad,
@@ -69,7 +68,7 @@ cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hk
     const size_t q_elt = (q_dtype == FATHOM_BF16) ? 2 : 4;
     float* scores = static_cast<float*>(workspace);
     const int64_t ld = n_pad_of(n);   // score row stride; n_pad is the store's row stride
-    const ScanTopkLayout lay = scan_topk_layout(n, Hq, hq_g);
+    const ScanTopkLayout lay = scan_topk_layout(n, Hq, hq_g, k);
     uint32_t* bmax = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + lay.bmax_off);
     void* topk_ws = static_cast<char*>(workspace) + lay.topk_off;
 

@@ -68,17 +68,23 @@ cudaError_t launch_topk(const float* scores, int64_t n, int64_t ld, int rows, in
 // the scan wrote alongside; ld a multiple of 64 and base offsets too
 size_t topk_blocks_workspace_bytes(int rows);
 
-// Workspace of a scan followed by the block-maximum top-k: scores
-// f32 [Hq][n_pad_of(n)], block maxima u32 [Hq][n_pad_of(n)/64], the top-k
-// buffers for `topk_rows` rows; each part 256-byte aligned.
+// top-k buffers for either path of launch_topk_blocks
+inline size_t topk_any_workspace_bytes(int64_t n, int rows, int k) {
+    const size_t a = topk_workspace_bytes(n, rows, k), b = topk_blocks_workspace_bytes(rows);
+    return a > b ? a : b;
+}
+
+// Workspace of a scan followed by top-k: scores f32 [Hq][n_pad_of(n)], block
+// maxima u32 [Hq][n_pad_of(n)/64], the top-k buffers for `topk_rows` rows;
+// each part 256-byte aligned.
 struct ScanTopkLayout {
     size_t bmax_off, topk_off, total;
 };
-inline ScanTopkLayout scan_topk_layout(int64_t n, int Hq, int topk_rows) {
+inline ScanTopkLayout scan_topk_layout(int64_t n, int Hq, int topk_rows, int k) {
     const size_t ld = (size_t)n_pad_of(n);
     const size_t sb = (sizeof(float) * (size_t)Hq * ld + 255) & ~size_t(255);
     const size_t bb = (sizeof(uint32_t) * (size_t)Hq * (ld / kBlock) + 255) & ~size_t(255);
-    return {sb, sb + bb, sb + bb + topk_blocks_workspace_bytes(topk_rows)};
+    return {sb, sb + bb, sb + bb + topk_any_workspace_bytes(n, topk_rows, k)};
 }
 cudaError_t launch_topk_blocks(const float* scores, const uint32_t* bmax, int64_t n, int64_t ld, int rows, int k,
                                int32_t* idx, float* top_scores, void* ws, cudaStream_t stream);

@@ -79,7 +79,7 @@ int fathom_scan_topk_noalloc(const fathom_store* store, const void* q, int q_dty
     // same split as fathom_scan_topk: scores [Hq][n_pad_of(n)], block maxima, then the top-k buffers
     float* scores = reinterpret_cast<float*>(scratch);
     const int64_t ld = n_pad_of(store->n);
-    const ScanTopkLayout lay = scan_topk_layout(store->n, n_q_heads, n_q_heads);
+    const ScanTopkLayout lay = scan_topk_layout(store->n, n_q_heads, n_q_heads, k);
     uint32_t* bmax = reinterpret_cast<uint32_t*>(scratch + lay.bmax_off);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = launch_scan(planes, scales, store->n_kv_heads, store->d, store->n, store->n_pad, q, q_dtype,

@@ -732,6 +732,13 @@ size_t topk_blocks_workspace_bytes(int rows) {
 
 cudaError_t launch_topk_blocks_map(const float* scores, const uint32_t* bmax, const RowMap& map, int rows, int k,
                                    int32_t* idx, float* top_scores, void* ws, cudaStream_t stream) {
+    // The bound m is tight only when a row has many more blocks than k: with
+    // at least 8k blocks, m lies in the top eighth of the block maxima and the
+    // surviving blocks hold about k candidates.  Shorter rows take the
+    // histogram path over the whole row.
+    int64_t min_n = map.max_n;
+    for (int s = 0; s < map.nsets; ++s) min_n = map.n[s] < min_n ? map.n[s] : min_n;
+    if (min_n / kBlock < 8 * (int64_t)k) return launch_topk_map(scores, map, rows, k, idx, top_scores, ws, stream);
     BlkWs w = carve_blk(ws, rows);
     topk_blk_threshold<<<rows, kFinishThreads, 0, stream>>>(bmax, map, k, w);
     const int64_t nbk = (map.max_n + kBlock - 1) / kBlock;
