@@ -28,10 +28,11 @@ namespace fathom {
 namespace {
 
 constexpr int kSplit = 8;      // CTAs per head (cluster size)
-constexpr int kWarps = 4;
+constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kUnroll = 8;     // rows in flight per warp
 constexpr int kSortCap = kMaxTopK;   // indices sorted in shared memory
+constexpr int kIdxRegs = (kMaxTopK + kSplit * kWarps * 32 - 1) / (kSplit * kWarps * 32);   // row indices per lane
 
 
 // A lane's V bf16 values of a row, kept as raw 32-bit words until used: the
@@ -116,22 +117,34 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
         ih = s_idx;
     }
     // rows of this warp: positions p = r + kSplit * (wp + kWarps * m) of the (sorted) list,
-    // so the head's 32 warps sweep the list together, in address order when sorted
+    // so the head's warps sweep the list together, in address order when sorted.
+    // The warp's row indices are read once, lane j holding those of m = j + 32 e,
+    // so every batch issues its row loads at once
     const int stride = kSplit * kWarps;
-    for (int p0 = r + kSplit * wp; p0 < k; p0 += stride * kUnroll) {
+    const int rows_w = (k - (r + kSplit * wp) + stride - 1) / stride;   // rows of this warp (may be <= 0)
+    int32_t my_idx[kIdxRegs];
+#pragma unroll
+    for (int e = 0; e < kIdxRegs; ++e) {
+        const int mm = lane + 32 * e;
+        my_idx[e] = (mm < rows_w) ? ih[r + kSplit * wp + stride * mm] : -1;
+    }
+    for (int m0 = 0; m0 < rows_w; m0 += kUnroll) {
         RowWords<V> kw[kUnroll], vw[kUnroll];
         bool ok[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int p = p0 + u * stride;
+            const int mm = m0 + u;
             ok[u] = false;
             kw[u].clear();
             vw[u].clear();
-            if (p < k) {
-                const int64_t i = ih[p];
+            int32_t i = -1;
+#pragma unroll
+            for (int e = 0; e < kIdxRegs; ++e)
+                if ((mm >> 5) == e) i = __shfl_sync(0xffffffffu, my_idx[e], mm & 31);
+            if (mm < rows_w) {
                 if (i >= 0 && i < n) {
                     ok[u] = true;
-                    const int64_t off = head_base + i * row_stride + lane * V;
+                    const int64_t off = head_base + (int64_t)i * row_stride + lane * V;
                     kw[u].load(Kr + off);
                     vw[u].load(Vr + off);
                 } else if (lane == 0) {

@@ -8,15 +8,16 @@
 // taking the B largest candidates v(c,t) = w_c 4^-t, t = 0..3.  The water
 // level theta is the value of the last candidate taken.
 //
-// One warp per query head.  Every candidate gets a distinct 64-bit key that
-// orders exactly as (v descending, c ascending, t ascending):
-//   the fp64 bit pattern of v = (double)w * 2^-2t (exact; a positive double's
-//   bits are monotone in its value, and an fp32 w leaves the low 29 bits of
-//   the pattern zero) OR-ed with ((255 - c) << 2 | (3 - t)).
-// theta is found by a bitwise radix select of the N-th largest key (bisection
-// on the threshold, 64 steps of one warp-wide count each); then
-// t_c = #{t : key(c,t) >= theta}.  Because the keys are distinct exactly N
-// candidates pass, so sum_c t_c = N = min(B, 4d).
+// One CTA per query head, one thread per candidate (c, t) = (tid / 4, tid % 4).
+// Each candidate gets a 32-bit key that orders exactly as v: v = (double)w 2^-2t
+// is exact in fp64 (a subnormal fp32 w included), its biased exponent lies in
+// [868, 1151] and its significand in the top 23 mantissa bits, so
+//   key = (exponent - 860) << 23 | significand   (0 for w = 0, ~0 for inf)
+// is monotone in v and equal only for equal v.  theta = the N-th largest key,
+// N = min(B, 4d), found bit by bit from the top (32 block-wide counts); the
+// candidates above theta are taken, and of those equal to theta the first
+// N - #{key > theta} in (c, t) order, which is the tie rule (c ascending, then
+// t ascending).  t_c = the number taken on channel c, so sum_c t_c = N.
 //
 // Group-pooled variant (not in the pages, which decide per query: arXiv
 // abstract, "each query decides"): the importance of channel c for KV head g
@@ -26,101 +27,74 @@
 //
 // Fixed-r comparison scans (ai-feeds.com summary, 与 Double Sparsity / Loki /
 // SparQ 的差异: a fixed 68 or 136 bits per key): depth 4 on the r channels with
-// the largest |q_c|, ties to the lower channel, by the same select on the
-// keys (bits(|q_c|) << 8 | (255 - c)).
+// the largest |q_c|, ties to the lower channel, by the same select with one
+// candidate per channel and key bits(|q_c|).
 #include "fathom_internal.cuh"
 
 namespace fathom {
 namespace {
 
-constexpr int kWarpsPerCta = 4;
-constexpr int kMaxChan = kMaxD / 32;  // channels per lane
-
-__device__ __forceinline__ int warp_count_ge(const uint64_t* keys, int m, uint64_t thr) {
-    int cnt = 0;
-#pragma unroll
-    for (int e = 0; e < 4 * kMaxChan; ++e)
-        if (e < m && keys[e] >= thr) ++cnt;
-    return __reduce_add_sync(0xffffffffu, cnt);
+// key of v = w 2^-2t (w >= 0): monotone in v, equal only for equal v
+__device__ __forceinline__ uint32_t cand_key(float w, int t) {
+    if (!(w > 0.0f)) return 0u;
+    if (isinf(w)) return 0xFFFFFFFFu;
+    const uint64_t b = (uint64_t)__double_as_longlong((double)w);   // normal, exponent >= 874
+    const uint32_t e = (uint32_t)(b >> 52) - 2u * (uint32_t)t;          // times 2^-2t, exactly
+    return (e - 860u) << 23 | ((uint32_t)(b >> 29) & 0x7FFFFFu);
 }
 
-// Largest T with #{keys >= T} >= N (1 <= N <= total); exact N-th largest.
-__device__ __forceinline__ uint64_t warp_select(const uint64_t* keys, int m, int N) {
-    uint64_t T = 0;
-    for (int bit = 63; bit >= 0; --bit) {
-        uint64_t cand = T | (1ull << bit);
-        if (warp_count_ge(keys, m, cand) >= N) T = cand;
-    }
-    return T;
-}
-
-__global__ void __launch_bounds__(kWarpsPerCta * 32)
+// blockDim = 4d: thread (c, t) = (tid / 4, tid % 4)
+__global__ void __launch_bounds__(4 * kMaxD)
 depths_kernel(const void* __restrict__ q, int q_dtype, const float* __restrict__ sigma2, int Hq, int Hkv,
               int d, int budget, int fixed_r, int pooled, uint8_t* __restrict__ depths) {
-    const int lane = threadIdx.x & 31;
-    const int h = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
-    if (h >= Hq) return;
+    __shared__ int s_ties[4 * kMaxD / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int h = blockIdx.x;
     const int g = h / (Hq / Hkv);
-    const int per_lane = d / 32;  // channel c = lane + 32 * e
-    uint64_t keys[4 * kMaxChan];
-    int m;
+    const int c = tid >> 2, t = tid & 3;
+    uint32_t key;
+    bool valid;
     int N;
     if (fixed_r == 0) {
-        m = 4 * per_lane;
+        const float s2 = sigma2[(int64_t)g * d + c];
+        float w;
+        if (pooled) {   // sum of the group's per-head importances, in head order
+            const int G = Hq / Hkv;
+            w = 0.0f;
+            for (int hh = g * G; hh < (g + 1) * G; ++hh) {
+                const float qc = load_q(q, q_dtype, (int64_t)hh * d + c);
+                w = __fadd_rn(w, __fmul_rn(__fmul_rn(qc, qc), s2));
+            }
+        } else {
+            const float qc = load_q(q, q_dtype, (int64_t)h * d + c);
+            w = __fmul_rn(__fmul_rn(qc, qc), s2);
+        }
+        key = cand_key(w, t);
+        valid = true;
         N = min(budget, 4 * d);
-#pragma unroll
-        for (int e = 0; e < kMaxChan; ++e) {
-            if (e < per_lane) {
-                int c = lane + 32 * e;
-                const float s2 = sigma2[(int64_t)g * d + c];
-                float w;
-                if (pooled) {   // sum of the group's per-head importances, in head order
-                    const int G = Hq / Hkv;
-                    w = 0.0f;
-                    for (int hh = g * G; hh < (g + 1) * G; ++hh) {
-                        const float qc = load_q(q, q_dtype, (int64_t)hh * d + c);
-                        w = __fadd_rn(w, __fmul_rn(__fmul_rn(qc, qc), s2));
-                    }
-                } else {
-                    const float qc = load_q(q, q_dtype, (int64_t)h * d + c);
-                    w = __fmul_rn(__fmul_rn(qc, qc), s2);
-                }
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    double v = (double)w * ((t == 0) ? 1.0 : (t == 1) ? 0.25 : (t == 2) ? 0.0625 : 0.015625);
-                    keys[4 * e + t] = (uint64_t)__double_as_longlong(v) |
-                                      ((uint64_t)(255 - c) << 2) | (uint64_t)(3 - t);
-                }
-            }
-        }
-    } else {
-        m = per_lane;
+    } else {   // one candidate per channel: |q_c|
+        key = __float_as_uint(fabsf(load_q(q, q_dtype, (int64_t)h * d + c)));
+        valid = t == 0;
         N = min(fixed_r, d);
-#pragma unroll
-        for (int e = 0; e < kMaxChan; ++e) {
-            if (e < per_lane) {
-                int c = lane + 32 * e;
-                float qa = fabsf(load_q(q, q_dtype, (int64_t)h * d + c));
-                keys[e] = ((uint64_t)__float_as_uint(qa) << 8) | (uint64_t)(255 - c);
-            }
-        }
     }
-    uint64_t theta = ~0ull;  // N == 0: nothing passes
-    if (N > 0) theta = warp_select(keys, m, N);
-#pragma unroll
-    for (int e = 0; e < kMaxChan; ++e) {
-        if (e < per_lane) {
-            int c = lane + 32 * e;
-            int t;
-            if (fixed_r == 0) {
-                t = 0;
-#pragma unroll
-                for (int s = 0; s < 4; ++s) t += (N > 0 && keys[4 * e + s] >= theta) ? 1 : 0;
-            } else {
-                t = (N > 0 && keys[e] >= theta) ? 4 : 0;
-            }
-            depths[(int64_t)h * d + c] = (uint8_t)t;
-        }
+    // theta: the largest T with #{key >= T} >= N
+    uint32_t T = 0;
+    for (int bit = 31; bit >= 0 && N > 0; --bit) {
+        const uint32_t cand = T | (1u << bit);
+        if (__syncthreads_count(valid && key >= cand) >= N) T = cand;
+    }
+    const int above = __syncthreads_count(valid && key > T);
+    const bool tie = valid && key == T;
+    const unsigned tb = __ballot_sync(0xffffffffu, tie);
+    if (lane == 0) s_ties[warp] = __popc(tb);
+    __syncthreads();
+    int rank = __popc(tb & ((1u << lane) - 1u));   // ties before this one, in (c, t) order
+    for (int x = 0; x < warp; ++x) rank += s_ties[x];
+    const bool take = N > 0 && valid && (key > T || (tie && rank < N - above));
+    const unsigned taken = __ballot_sync(0xffffffffu, take);
+    if (t == 0) {
+        const int dep = (fixed_r == 0) ? __popc((taken >> (lane & ~3)) & 0xFu) : (take ? 4 : 0);
+        depths[(int64_t)h * d + c] = (uint8_t)dep;
     }
 }
 
@@ -128,8 +102,7 @@ depths_kernel(const void* __restrict__ q, int q_dtype, const float* __restrict__
 
 cudaError_t launch_depths(const void* q, int q_dtype, const float* sigma2, int Hq, int Hkv, int d,
                           int budget, int fixed_r, uint8_t* depths, cudaStream_t stream, int pooled) {
-    dim3 grid((unsigned)((Hq + kWarpsPerCta - 1) / kWarpsPerCta));
-    depths_kernel<<<grid, kWarpsPerCta * 32, 0, stream>>>(q, q_dtype, sigma2, Hq, Hkv, d, budget, fixed_r,
+    depths_kernel<<<(unsigned)Hq, 4 * d, 0, stream>>>(q, q_dtype, sigma2, Hq, Hkv, d, budget, fixed_r,
                                                          pooled, depths);
     return cudaGetLastError();
 }

@@ -20,8 +20,15 @@
 //
 // Kernels: init, (hist, select) x 3 levels, compact, finish.  Level 0 always
 // runs over every row; levels 1 and 2 run as small grid-stride launches that
-// leave at once when no row is still refining (the common case).
+// leave at once when no row is still refining (the common case).  Rows of at
+// most kRowsMax keys skip all of this: one cluster kernel per launch holds a
+// row in the shared memory of 1 to 8 CTAs and selects there (topk_rows).
+// Rows with at least 8k blocks of 64 keys take the block-maximum path.
+#include <cooperative_groups.h>
+
 #include "fathom_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace fathom {
 namespace {
@@ -376,11 +383,12 @@ __device__ void bitonic_desc(uint64_t* buf, int S) {
 
 // With hist[0..nb) filled, finds the bin b holding the need-th largest key
 // (bins ordered high to low): *above = keys in bins above b, *cnt = keys in b.
-// Called by every thread of a kFinishThreads block; all get the result.
+// Called by every thread of the block (a multiple of 32 threads, at most
+// 1024); all get the result.
 __device__ void block_pick_bin(const uint32_t* hist, int nb, uint32_t need, int* s_bin, uint32_t* s_above,
                                uint32_t* s_cnt, uint32_t* warp_tot) {
-    const int t = threadIdx.x, lane = t & 31, wp = t >> 5;
-    const int per = nb / kFinishThreads > 0 ? nb / kFinishThreads : 1;   // bins per thread
+    const int t = threadIdx.x, lane = t & 31, wp = t >> 5, nt = (int)blockDim.x;
+    const int per = nb / nt > 0 ? nb / nt : 1;   // bins per thread
     uint32_t mine = 0;
     if (per * t < nb)
         for (int e = 0; e < per; ++e) mine += hist[per * t + e];
@@ -393,7 +401,7 @@ __device__ void block_pick_bin(const uint32_t* hist, int nb, uint32_t need, int*
     if (lane == 0) warp_tot[wp] = v;
     __syncthreads();
     uint32_t higher = 0;
-    for (int x = wp + 1; x < kFinishThreads / 32; ++x) higher += warp_tot[x];
+    for (int x = wp + 1; x < nt / 32; ++x) higher += warp_tot[x];
     const uint32_t incl = v + higher, above = incl - mine;
     if (above < need && incl >= need && per * t < nb) {
         uint32_t acc = above;
@@ -706,6 +714,264 @@ topk_blk_finish(const float* __restrict__ scores, const __grid_constant__ RowMap
     }
 }
 
+// ---------------------------------------------------------------------------
+// Short rows (n <= kRowsMax keys): one kernel, no workspace.  A cluster of CL
+// CTAs takes a row; CTA x holds the ordered keys of its slice of the row in
+// shared memory.  Three radix steps (12, 12 and 8 bits) each combine the CTAs'
+// histograms through distributed shared memory (cluster_pick), so every CTA
+// finds the same exact k-th key T.  Each CTA then writes its keys above T, and its keys equal
+// to T whose rank among the row's ties (CTA order, then index order) is below
+// k - #{keys > T}, into CTA 0's shared memory; CTA 0 sorts the k entries as
+// 64-bit composites (key << 32 | ~index).
+// ---------------------------------------------------------------------------
+constexpr int kSliceKeys = 16384;   // keys per CTA
+constexpr int kRowThreads = 512;
+constexpr int kMaxCluster = 8;
+constexpr int64_t kRowsMax = (int64_t)kMaxCluster * kSliceKeys;
+constexpr size_t kRowSmem = sizeof(uint32_t) * (kSliceKeys + kBins) + sizeof(uint64_t) * kMaxTopK;
+
+__device__ __forceinline__ int block_sum_int(int v, int* warp_cnt) {
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    v = __reduce_add_sync(0xffffffffu, v);
+    if (lane == 0) warp_cnt[wp] = v;
+    __syncthreads();
+    int t = 0;
+    for (int x = 0; x < (int)(blockDim.x >> 5); ++x) t += warp_cnt[x];
+    __syncthreads();
+    return t;
+}
+
+template <int CL>
+__device__ __forceinline__ void cluster_barrier() {
+    if constexpr (CL > 1) cg::this_cluster().sync();
+    else __syncthreads();
+}
+
+// With this CTA's keys added to hist[0..nb), picks the bin of the need-th
+// largest key of the whole cluster, as block_pick_bin (every CTA gets the
+// result).  The summed histogram is split: CTA x sums bins [x nb/CL,
+// (x+1) nb/CL) over the cluster and publishes their total; every CTA then
+// finds the range holding the need-th key from the totals and picks inside it
+// from that range's sums.  Each CTA reads about nb + nb/CL remote words.
+// hsum holds nb/CL words; hist is reused as scratch.
+template <int CL>
+__device__ __forceinline__ void cluster_pick(uint32_t* hist, uint32_t* hsum, int nb, uint32_t need, int* s_bin,
+                                             uint32_t* s_above, uint32_t* s_cnt, uint32_t* warp_tot, int* warp_cnt,
+                                             uint32_t* s_tot) {
+    if constexpr (CL > 1) {
+        cg::cluster_group cluster = cg::this_cluster();
+        const int x = (int)cluster.block_rank(), per = nb / CL, tid = threadIdx.x;
+        cluster.sync();   // every CTA's histogram is complete
+        int mine = 0;
+        for (int j = tid; j < per; j += kRowThreads) {
+            uint32_t t = 0;
+#pragma unroll
+            for (int y = 0; y < CL; ++y) t += cluster.map_shared_rank(hist, y)[x * per + j];
+            hsum[j] = t;
+            mine += (int)t;
+        }
+        mine = block_sum_int(mine, warp_cnt);
+        if (tid == 0) *s_tot = (uint32_t)mine;
+        cluster.sync();   // range sums and totals are published; nobody reads hist any more
+        uint32_t acc = 0;
+        int ys = 0;
+        for (int y = CL - 1; y >= 0; --y) {   // ranges from the highest bins down
+            const uint32_t t = *cluster.map_shared_rank(s_tot, y);
+            if (acc + t >= need) {
+                ys = y;
+                break;
+            }
+            acc += t;
+        }
+        const uint32_t* hy = cluster.map_shared_rank(hsum, ys);
+        for (int j = tid; j < per; j += kRowThreads) hist[j] = hy[j];
+        __syncthreads();
+        block_pick_bin(hist, per, need - acc, s_bin, s_above, s_cnt, warp_tot);
+        if (tid == 0) {
+            *s_bin += ys * per;
+            *s_above += acc;
+        }
+        cluster.sync();   // the picks are visible, and every CTA has read the range it needed
+    } else {
+        __syncthreads();
+        block_pick_bin(hist, nb, need, s_bin, s_above, s_cnt, warp_tot);
+    }
+}
+
+template <int CL>
+__global__ void __launch_bounds__(kRowThreads)
+topk_rows(const float* __restrict__ scores, const __grid_constant__ RowMap m, int k, int32_t* __restrict__ idx,
+          float* __restrict__ top_scores) {
+    extern __shared__ __align__(16) unsigned char row_smem[];
+    uint32_t* keys = reinterpret_cast<uint32_t*>(row_smem);                      // [kSliceKeys]
+    uint32_t* hist = keys + kSliceKeys;                                           // [kBins]
+    uint64_t* buf = reinterpret_cast<uint64_t*>(hist + kBins);                    // [kMaxTopK], CTA 0
+    uint32_t* hsum = (CL > 1) ? reinterpret_cast<uint32_t*>(buf) : hist;          // cluster histogram
+    __shared__ uint32_t warp_tot[32];
+    __shared__ int warp_cnt[32];
+    __shared__ int s_bin, s_fill, s_gt, s_eq;
+    __shared__ uint32_t s_above, s_cnt, s_tot;
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    int rank = 0;
+    if constexpr (CL > 1) rank = (int)cg::this_cluster().block_rank();
+    const int row = blockIdx.x / CL;
+    int64_t off, n;
+    row_span(m, row, &off, &n);
+    const int64_t L = ((n + CL - 1) / CL + 3) & ~int64_t(3);   // slice length, <= kSliceKeys
+    const int64_t start = rank * L;
+    const int cnt = (int)(n - start < 0 ? 0 : (n - start < L ? n - start : L));
+    const float* s = scores + off + start;
+
+    // the slice as ordered keys
+    if ((reinterpret_cast<uintptr_t>(s) & 15u) == 0) {
+        const int nv = cnt >> 2;
+        const float4* s4 = reinterpret_cast<const float4*>(s);
+        for (int v0 = tid; v0 < nv; v0 += 8 * kRowThreads) {
+            float4 x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (v0 + u * kRowThreads < nv) x[u] = __ldg(s4 + v0 + u * kRowThreads);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (v0 + u * kRowThreads < nv) {
+                    uint32_t* dk = keys + 4 * (v0 + u * kRowThreads);
+                    dk[0] = float_to_ordered(x[u].x);
+                    dk[1] = float_to_ordered(x[u].y);
+                    dk[2] = float_to_ordered(x[u].z);
+                    dk[3] = float_to_ordered(x[u].w);
+                }
+        }
+        for (int e = 4 * nv + tid; e < cnt; e += kRowThreads) keys[e] = float_to_ordered(s[e]);
+    } else {
+        for (int e = tid; e < cnt; e += kRowThreads) keys[e] = float_to_ordered(__ldg(s + e));
+    }
+    __syncthreads();
+
+    // the exact k-th largest key T of the row
+    uint32_t need = (uint32_t)k, prefix = 0, above = 0;
+    int shift = 32;
+    while (shift > 0) {
+        const int nbits = shift >= 12 ? 12 : shift, sh = shift - nbits, nb = 1 << nbits;
+        for (int b = tid; b < nb; b += kRowThreads) hist[b] = 0;
+        __syncthreads();
+        for (int e = tid; e < cnt; e += kRowThreads) {
+            const uint32_t key = keys[e];
+            if (shift == 32 || (key >> shift) == prefix) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1u);
+        }
+        cluster_pick<CL>(hist, hsum, nb, need, &s_bin, &s_above, &s_cnt, warp_tot, warp_cnt, &s_tot);
+        need -= s_above;
+        above += s_above;
+        prefix = (shift == 32 ? 0u : (prefix << nbits)) | (uint32_t)s_bin;
+        shift = sh;
+        __syncthreads();   // s_bin / s_above are rewritten by the next step
+    }
+    const uint32_t T = prefix;
+    const int gt_row = (int)above, take_eq = k - gt_row;   // keys above T; ties to take (>= 1)
+
+    // this CTA's keys above T and at T, and those of the CTAs before it
+    int my_gt = 0, my_eq = 0;
+    for (int e = tid; e < cnt; e += kRowThreads) {
+        my_gt += keys[e] > T;
+        my_eq += keys[e] == T;
+    }
+    my_gt = block_sum_int(my_gt, warp_cnt);
+    my_eq = block_sum_int(my_eq, warp_cnt);
+    if (tid == 0) {
+        s_gt = my_gt;
+        s_eq = my_eq;
+        s_fill = 0;
+    }
+    cluster_barrier<CL>();
+    int gt_before = 0, eq_before = 0;
+    uint64_t* dst = buf;
+    if constexpr (CL > 1) {
+        cg::cluster_group cluster = cg::this_cluster();
+        for (int x = 0; x < rank; ++x) {
+            gt_before += *cluster.map_shared_rank(&s_gt, x);
+            eq_before += *cluster.map_shared_rank(&s_eq, x);
+        }
+        dst = cluster.map_shared_rank(buf, 0);
+    }
+    // keys above T, in any order (the sort orders them)
+    for (int e = tid; e < cnt; e += kRowThreads)
+        if (keys[e] > T) dst[gt_before + atomicAdd(&s_fill, 1)] = composite(keys[e], start + e);
+    // keys at T with row tie rank < take_eq
+    if (my_eq > 0 && eq_before < take_eq) {
+        if (eq_before + my_eq <= take_eq) {   // all of this CTA's ties are taken: any order
+            __syncthreads();
+            if (tid == 0) s_fill = 0;
+            __syncthreads();
+            for (int e = tid; e < cnt; e += kRowThreads)
+                if (keys[e] == T) dst[gt_row + eq_before + atomicAdd(&s_fill, 1)] = composite(T, start + e);
+        } else {   // the cut falls inside this CTA: ordered scan
+            int got = eq_before;
+            for (int base = 0; base < cnt && got < take_eq; base += kRowThreads) {
+                const int e = base + tid;
+                const bool f = e < cnt && keys[e] == T;
+                const unsigned msk = __ballot_sync(0xffffffffu, f);
+                if (lane == 0) warp_cnt[wp] = __popc(msk);
+                __syncthreads();
+                int before = 0, all = 0;
+                for (int x = 0; x < kRowThreads / 32; ++x) {
+                    before += (x < wp) ? warp_cnt[x] : 0;
+                    all += warp_cnt[x];
+                }
+                const int r = got + before + __popc(msk & ((1u << lane) - 1u));
+                if (f && r < take_eq) dst[gt_row + r] = composite(T, start + e);
+                got += all;
+                __syncthreads();   // warp_cnt is rewritten by the next window
+            }
+        }
+    }
+    cluster_barrier<CL>();   // CTA 0 holds the row's k entries
+    if (rank != 0) return;
+    int S = 1;
+    while (S < k) S <<= 1;
+    for (int e = k + tid; e < S; e += kRowThreads) buf[e] = 0ull;
+    __syncthreads();
+    bitonic_desc(buf, S);
+    for (int e = tid; e < k; e += kRowThreads) {
+        const uint64_t c = buf[e];
+        idx[(int64_t)row * k + e] = (int32_t)(0xFFFFFFFFu - (uint32_t)c);
+        if (top_scores) top_scores[(int64_t)row * k + e] = ordered_to_float((uint32_t)(c >> 32));
+    }
+}
+
+template <int CL>
+cudaError_t launch_topk_rows_cl(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
+                                float* top_scores, cudaStream_t stream) {
+    auto kern = topk_rows<CL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRowSmem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * CL));
+    cfg.blockDim = dim3(kRowThreads);
+    cfg.dynamicSmemBytes = kRowSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = CL > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, scores, map, k, idx, top_scores);
+}
+
+// rows of at most kRowsMax keys and k <= kMaxTopK
+cudaError_t launch_topk_rows(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
+                             float* top_scores, cudaStream_t stream) {
+    int cl = 1;
+    while ((int64_t)cl * kSliceKeys < map.max_n) cl <<= 1;
+    switch (cl) {
+        case 1: return launch_topk_rows_cl<1>(scores, map, rows, k, idx, top_scores, stream);
+        case 2: return launch_topk_rows_cl<2>(scores, map, rows, k, idx, top_scores, stream);
+        case 4: return launch_topk_rows_cl<4>(scores, map, rows, k, idx, top_scores, stream);
+        case 8: return launch_topk_rows_cl<8>(scores, map, rows, k, idx, top_scores, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 // positions into the gathered candidate lists -> the candidates' global indices
 __global__ void topk_map_positions(const int32_t* __restrict__ cand_idx, int n_cand, int k, int32_t* idx) {
     const int row = blockIdx.y;
@@ -772,6 +1038,7 @@ size_t topk_workspace_bytes(int64_t n, int rows, int k) {
 
 cudaError_t launch_topk_map(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
                             float* top_scores, void* ws, cudaStream_t stream) {
+    if (map.max_n <= kRowsMax && k <= kMaxTopK) return launch_topk_rows(scores, map, rows, k, idx, top_scores, stream);
     Workspace w = carve(ws, rows, k);
     unsigned int* status = device_status_ptr();
     const unsigned chunks = (unsigned)((map.max_n + kChunk - 1) / kChunk);

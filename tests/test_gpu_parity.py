@@ -259,8 +259,11 @@ def test_six_key_example_on_gpu():
 @pytest.mark.parametrize("n,rows,k,kind", [
     (100, 3, 1, "normal"), (100, 3, 100, "normal"), (4096, 2, 64, "normal"), (20000, 4, 2048, "normal"),
     (131072, 2, 2048, "normal"), (200000, 2, 4096, "ties"), (50000, 2, 2048, "equal"),
-    (70000, 2, 1000, "narrow"), (4096, 1, 4096, "ties"), (9000, 1, 4096, "ties")])
+    (70000, 2, 1000, "narrow"), (4096, 1, 4096, "ties"), (9000, 1, 4096, "ties"),
+    (300000, 2, 2048, "normal"), (140000, 2, 1000, "narrow"), (140000, 1, 3000, "equal")])
 def test_topk_bit_exact(ref, n, rows, k, kind):
+    """Rows up to 131072 keys take the one-kernel cluster path (1, 2, 4 or 8
+    CTAs per row), longer rows the multi-pass histogram path."""
     rng = np.random.default_rng(n + k)
     if kind == "normal":
         s = rng.standard_normal((rows, n)).astype(np.float32)
@@ -306,12 +309,13 @@ def test_topk_from_block_maxima_equals_full_selection(n, B, k):
 
 
 @pytest.mark.parametrize("kind", ["normal", "ties", "narrow"])
-def test_topk_repeatable_under_load(ref, kind):
+@pytest.mark.parametrize("n", [65536, 262144])
+def test_topk_repeatable_under_load(ref, kind, n):
     """The same rows, 20 launches back to back with many rows in flight: every
     launch must give the oracle's exact answer (a race in the selection or the
     final sort shows up as a launch that differs)."""
     rng = np.random.default_rng(7)
-    rows, n, k = 32, 65536, 2048
+    rows, k = 32, 2048
     if kind == "normal":
         s = rng.standard_normal((rows, n)).astype(np.float32)
     elif kind == "ties":
