@@ -492,6 +492,21 @@ def _events_ms(torch, fn, steps, warmup, flush=None):
     return np.array(ts)
 
 
+def _graph_of(torch, fn, warmup=3):
+    """fn() captured once into a CUDA graph (after warm-up calls on a side
+    stream, as capture requires); returns the graph's replay."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(warmup):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
 def config_bench(args):
     """The pages' other workloads, each timed through the one-call decode step
     or the batched entry point (one JSON line per case):
@@ -527,6 +542,9 @@ def config_bench(args):
             step = lambda: F.decode_step(st, inp["q_dev"], inp["sigma2_dev"], b, k, Kr, Vr, fixed_r=fr, **bufs)
             t_flush = _events_ms(torch, step, args.steps, args.warmup, flush)
             t_warm = _events_ms(torch, step, args.steps, args.warmup)
+            graph = _graph_of(torch, step)   # the same call replayed from a CUDA graph: no host launch cost
+            t_graph = _events_ms(torch, graph.replay, args.steps, args.warmup, flush)
+            del graph
             dep = F.alloc_depths(inp["q_dev"], inp["sigma2_dev"], b, fixed_r=fr)
             scan = _events_ms(torch, lambda: F.scan_scores(st, inp["q_dev"], dep), args.steps, args.warmup, flush)
             U = dep.view(Hkv, Hq // Hkv, 128).amax(dim=1)
@@ -549,6 +567,7 @@ def config_bench(args):
             out.append({"config": args.config, "case": name, "workload": cfg["name"], "n": n, "n_kv_heads": Hkv,
                         "n_q_heads": Hq, "k": k, "step_us_l2_flushed": float(np.median(t_flush)) * 1e3,
                         "step_us_warm": float(np.median(t_warm)) * 1e3,
+                        "step_us_cuda_graph_l2_flushed": float(np.median(t_graph)) * 1e3,
                         "scan_us": float(np.median(scan)) * 1e3,
                         "gkeys_per_s_step": n * Hkv / (float(np.median(t_flush)) * 1e-3) / 1e9,
                         "scan_bytes_per_key_per_kv_head": nbytes / (n * Hkv),
@@ -802,6 +821,18 @@ def main():
                 "depths_ms": float(r3["depths_ms"].mean()),
                 "gkeys_per_s": args.n * layer.Hkv / (float(p3["step_ms"].mean()) * 1e-3) / 1e9,
                 "scan_gbs": b3 / (s3 * 1e-3) / 1e9, "scan_hbm_frac": b3 / (s3 * 1e-3) / 1e9 / hbm_peak}
+            # the same scan against the ALU roofline: the method's signed plane
+            # accumulates (sum over query heads and channels of t_hc, per key)
+            # over 148 SMs x 128 lanes x the SM clock sampled in the timed region
+            ops = float(layer.depths.sum().item()) * args.n
+            sms = torch.cuda.get_device_properties(dev).multi_processor_count
+            mhz = ((pipe.get("clocks") or {}).get("sm_mhz")) or 1965.0
+            alu_peak = sms * 128 * mhz * 1e6 / 1e12
+            extras["hbm_resident"]["roofline_alu"] = {
+                "bound": "alu", "achieved": ops / (s3 * 1e-3) / 1e12, "peak": alu_peak,
+                "unit": "T plane-accumulates/s", "frac": ops / (s3 * 1e-3) / 1e12 / alu_peak,
+                "ops_per_key_per_kv_head": ops / (args.n * layer.Hkv),
+                "peak_source": "%d SMs x 128 lanes x %.0f MHz (sampled)" % (sms, mhz)}
             layer.store, layer.K_rows, layer.V_rows = keep
 
     cpu = None

@@ -24,8 +24,8 @@
 // (U_c > 0) are streamed in chunks of 16:
 //   stage: thread (channel group, plane word w) loads the U_c plane words of
 //     its channels (row pointers prepared once per tile) and transposes them
-//     to the 8 code words (s, w) (rotate + mask per plane and word), stored
-//     with conflict-free 32-bit stores.  Thread (channel, block) pairs form
+//     to the 8 code words (s, w) (planes paired, then merged to nibbles, one
+//     rotate + mask per word), stored with conflict-free 32-bit stores.  Thread (channel, block) pairs form
 //     the coefficients 32 q Delta of every head and add Delta q (2^(3-t) - 24)
 //     into a per-(block, head) constant kept in registers.
 //   compute: warp (head h, key split) walks head h's item list of the chunk:
@@ -80,14 +80,49 @@ struct ScanSmem {
     __host__ __device__ size_t bytes() const { return (tdep() + (size_t)G * d + 15) & ~size_t(15); }
 };
 
+__device__ __forceinline__ uint32_t rotr(uint32_t x, int sft) { return __funnelshift_r(x, x, (uint32_t)sft & 31u); }
+
+// The 8 code words of 32 keys of one channel from its first U plane words p
+// (p[j] = 0 for j >= U): word sv holds keys sv + 8k, k = 0..3, plane j of key
+// sv + 8k at bit 8k + 6 - j.  Planes are first paired, and for U >= 3 the two
+// pairs merged into nibbles (key 4m + c in nibble m of a word per class c),
+// so that one rotate and one mask place several planes at once.
+__device__ __forceinline__ void codes_of(const uint32_t (&p)[4], int U, uint32_t (&x)[8]) {
+    if (U >= 2) {
+        // even keys 2m: bit 2m = plane 1, bit 2m+1 = plane 0; odd keys 2m+1 likewise
+        const uint32_t e01 = (p[1] & 0x55555555u) | ((p[0] << 1) & 0xAAAAAAAAu);
+        const uint32_t o01 = ((p[1] >> 1) & 0x55555555u) | (p[0] & 0xAAAAAAAAu);
+        if (U == 2) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                x[2 * r] = rotr(e01, 2 * r - 5) & 0x60606060u;
+                x[2 * r + 1] = rotr(o01, 2 * r - 5) & 0x60606060u;
+            }
+        } else {
+            const uint32_t e23 = (p[3] & 0x55555555u) | ((p[2] << 1) & 0xAAAAAAAAu);
+            const uint32_t o23 = ((p[3] >> 1) & 0x55555555u) | (p[2] & 0xAAAAAAAAu);
+            // key 4m + c: nibble m of q[c], planes 3..0 in its bits 0..3
+            const uint32_t q[4] = {(e23 & 0x33333333u) | ((e01 << 2) & 0xCCCCCCCCu),
+                                   (o23 & 0x33333333u) | ((o01 << 2) & 0xCCCCCCCCu),
+                                   ((e23 >> 2) & 0x33333333u) | (e01 & 0xCCCCCCCCu),
+                                   ((o23 >> 2) & 0x33333333u) | (o01 & 0xCCCCCCCCu)};
+#pragma unroll
+            for (int sv = 0; sv < 8; ++sv) x[sv] = rotr(q[sv & 3], 4 * (sv >> 2) - 3) & 0x78787878u;
+        }
+    } else {
+#pragma unroll
+        for (int sv = 0; sv < 8; ++sv) x[sv] = (U == 1) ? (rotr(p[0], sv - 6) & 0x40404040u) : 0u;
+    }
+}
+
 // F of byte k of a code word (he = kHalfExp)
 __device__ __forceinline__ float f_of(uint32_t x, uint32_t he, uint32_t k) {
     return __uint_as_float(__byte_perm(x, he, 0x7044u | (k << 8)));
 }
 
-// G consecutive floats of shared memory (16-byte aligned when G >= 4), or zeros
+// G consecutive floats of shared memory (16-byte aligned when G >= 4)
 template <int G>
-__device__ __forceinline__ void load_g(const float* p, bool ok, float (&v)[G]) {
+__device__ __forceinline__ void load_g(const float* p, float (&v)[G]) {
     if constexpr (G % 4 == 0) {
 #pragma unroll
         for (int i = 0; i < G; i += 4) {
@@ -98,8 +133,6 @@ __device__ __forceinline__ void load_g(const float* p, bool ok, float (&v)[G]) {
 #pragma unroll
         for (int i = 0; i < G; ++i) v[i] = p[i];
     }
-#pragma unroll
-    for (int i = 0; i < G; ++i) v[i] = ok ? v[i] : 0.0f;
 }
 
 // One (tile of 1024 keys, KV head g) of one store; q, depths and scores are
@@ -169,10 +202,12 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
     __syncthreads();
     const int L = s_L;
     const int nchunks = (L + kChunk - 1) / kChunk;
-    for (int a = tid; a < L; a += Z::T) {
-        const int64_t row = (int64_t)g * d + s_act[a];
+    for (int a = tid; a < nchunks * kChunk; a += Z::T) {   // slots past the list: nothing to read
+        const bool live = a < L;
+        const int64_t row = (int64_t)g * d + (live ? s_act[a] : 0);
         s_prow[a] = planes + row * 4 * words_total + tile0 / 32;
         s_srow[a] = scales + row * nblk_total + tile0 / kBlock;
+        if (!live) s_U[a] = 0;
     }
     for (int e = tid; e < L * G; e += Z::T) {
         const int a = e / G, hh = e - a * G;
@@ -181,6 +216,10 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
         const float qv = load_q(q, q_dtype, ((int64_t)g * G + hh) * d + c);
         s_q32[e] = (t > 0) ? 32.0f * qv : 0.0f;
         s_qk[e] = (t > 0) ? qv * (__uint_as_float((uint32_t)(130 - t) << 23) - 24.0f) : 0.0f;
+    }
+    for (int e = L * G + tid; e < nchunks * kChunk * G; e += Z::T) {   // the last chunk's unused slots
+        s_q32[e] = 0.0f;
+        s_qk[e] = 0.0f;
     }
     if (warp < G) {
         // item list of head h = warp, chunk by chunk: channels read to the
@@ -235,8 +274,8 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
 #pragma unroll
         for (int i = 0; i < Z::CPT; ++i) {
             const int a = ch * kChunk + cg * Z::CPT + i;   // warp-uniform
-            const int U = (a < L && wok) ? s_U[a] : 0;
-            const uint32_t* p = ((a < L) ? s_prow[a] : planes) + w;
+            const int U = wok ? s_U[a] : 0;
+            const uint32_t* p = s_prow[a] + w;
 #pragma unroll
             for (int j = 0; j < 4; ++j) pw[i][j] = (j < U) ? __ldg(p + j * words_total) : 0u;
         }
@@ -251,19 +290,9 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
 #pragma unroll
         for (int i = 0; i < Z::CPT; ++i) {
             const int al = cg * Z::CPT + i, a = ch * kChunk + al;
-            const int U = (a < L) ? s_U[a] : 0;   // warp-uniform
+            const int U = s_U[a];   // warp-uniform; 0 past the list
             uint32_t x[8];
-#pragma unroll
-            for (int sv = 0; sv < 8; ++sv) x[sv] = 0u;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if (j < U) {
-#pragma unroll
-                    for (int sv = 0; sv < 8; ++sv)
-                        x[sv] |= __funnelshift_r(pw[i][j], pw[i][j], (uint32_t)(sv + j - 6) & 31u) &
-                                 (0x01010101u << (6 - j));
-                }
-            }
+            codes_of(pw[i], U, x);
 #pragma unroll
             for (int sv = 0; sv < 8; ++sv) cbase[al * kChanWords + sv * kTileWords] = x[sv];
         }
@@ -272,8 +301,8 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
         for (int u = 0; u < Z::DPT; ++u) {
             const int al = (tid + u * Z::T) >> 4, a = ch * kChunk + al;   // a < d: nchunks * 16 <= d
             float qv[G], kv[G];
-            load_g<G>(s_q32 + a * G, a < L, qv);
-            load_g<G>(s_qk + a * G, a < L, kv);
+            load_g<G>(s_q32 + a * G, qv);   // zero past the union list
+            load_g<G>(s_qk + a * G, kv);
 #pragma unroll
             for (int hh = 0; hh < G; ++hh) {
                 cf[(hh * kChunk + al) * kTileBlocks + bb] = qv[hh] * pd[u];
