@@ -203,11 +203,14 @@ int fathom_scan_scores(const fathom_store* store, const void* q, int q_dtype, co
  * Top-k of score rows: the k largest of scores[r][0..n), ties to the lower
  * index, listed in that order.  [ai-feeds summary 关键模块 5, 输出]
  *   scores      device, f32 [n_rows][ld] (ld >= n); NaN is not allowed.
- *   block_max   NULL (select from the scores alone: histogram passes over
- *               every row), or the block maxima that fathom_scan_scores wrote
- *               with these scores (ld a multiple of 64): with m = the k-th
- *               largest block maximum of a row, k keys score at least m, so
- *               only the blocks whose maximum is >= m are read.
+ *   block_max   NULL (select from the scores alone), or the block maxima
+ *               that fathom_scan_scores wrote with these scores (ld a
+ *               multiple of 64): with m = the k-th largest block maximum of a
+ *               row, k keys score at least m, so only the blocks whose
+ *               maximum is >= m are read.  The bound is used for rows of at
+ *               least 8k blocks; rows of at most 131072 keys are selected in
+ *               on-chip memory by one kernel, longer ones by histogram passes
+ *               over the whole row.  The result is the same on every path.
  *   idx         device, i32 [n_rows][k].
  *   top_scores  device, f32 [n_rows][k], or NULL.
  *   workspace   device, at least fathom_topk_workspace_bytes(n, n_rows, k) bytes,
