@@ -342,6 +342,35 @@ int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, con
                                    (cudaStream_t)stream));
 }
 
+int fathom_sparse_attend_partial(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
+                                 int64_t row_stride, int rows_host_resident, int64_t key0, const int32_t* idx,
+                                 int n_q_heads, int n_kv_heads, int64_t n, int d, int k, float* parts,
+                                 fathom_stream_t stream) {
+    if (!q || !K_rows || !V_rows || !idx || !parts || n < 1 || key0 < 0 || k < 1 || !dims_ok(n_kv_heads, d) ||
+        !heads_ok(n_q_heads, n_kv_heads))
+        return FATHOM_EINVAL;
+    if (q_dtype != FATHOM_F32 && q_dtype != FATHOM_BF16) return FATHOM_EINVAL;
+    if (d != 32 && d != 64 && d != 128 && d != 256) return FATHOM_EUNSUPPORTED;
+    if (row_stride < d || row_stride % 8) return FATHOM_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(K_rows) & 15) || (reinterpret_cast<uintptr_t>(V_rows) & 15))
+        return FATHOM_EINVAL;
+    const void* kd = nullptr;
+    const void* vd = nullptr;
+    Where want = rows_host_resident ? Where::kHostPinned : Where::kDevice;
+    if (classify(K_rows, &kd) != want || classify(V_rows, &vd) != want) return FATHOM_EINVAL;
+    if (!is_device(q) || !is_device(idx) || !is_device(parts)) return FATHOM_EINVAL;
+    if (!device_status_ptr()) return FATHOM_ECUDA;
+    return to_status(launch_attend(q, q_dtype, static_cast<const uint16_t*>(kd), static_cast<const uint16_t*>(vd),
+                                   row_stride, idx, n_q_heads, n_kv_heads, n, d, k, rows_host_resident, nullptr,
+                                   (cudaStream_t)stream, key0, parts));
+}
+
+int fathom_attend_merge(const float* parts, int world, int n_q_heads, int d, float* out, fathom_stream_t stream) {
+    if (!parts || !out || world < 1 || n_q_heads < 1 || d < 1 || d > kMaxD) return FATHOM_EINVAL;
+    if (!is_device(parts) || !is_device(out)) return FATHOM_EINVAL;
+    return to_status(launch_attend_merge(parts, world, n_q_heads, d, out, (cudaStream_t)stream));
+}
+
 size_t fathom_decode_workspace_bytes(const fathom_store* store, int n_q_heads, int k, int kv_groups) {
     if (!store || store->n < 1 || n_q_heads < 1 || k < 1 || k > kMaxTopK || kv_groups < 1 || kv_groups > 64 ||
         store->n_kv_heads < 1 || store->n_kv_heads % kv_groups || n_q_heads % store->n_kv_heads)

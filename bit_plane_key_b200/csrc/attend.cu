@@ -11,6 +11,12 @@
 // [l*d/32, (l+1)*d/32)).  The warps' partial (max, sum, o) merge in shared
 // memory, then CTA 0 merges the kSplit CTA partials through distributed
 // shared memory and writes o_h.  No workspace and no second kernel.
+// With a key range split across GPUs, each rank runs the same kernel over
+// the rows it holds (global indices shifted by its first key; the other
+// ranks' indices skipped) and writes the CTA 0 merge unnormalised: o relative
+// to the running maximum m, m and the sum l (log2 units, as below);
+// attend_merge_kernel combines the ranks' partials the way CTA 0 combines
+// its cluster's.
 // Rows may live in device memory or in page-locked host memory.  Over the
 // host link, gathering rows in address order is faster than in score order,
 // so for host-resident rows every CTA first sorts the head's indices in
@@ -69,7 +75,8 @@ template <int V>
 __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kThreads)
 attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restrict__ Kr,
               const uint16_t* __restrict__ Vr, int64_t row_stride, const int32_t* __restrict__ idx, int Hq, int Hkv,
-              int64_t n, int k, int sort_rows, float* __restrict__ out, unsigned int* status) {
+              int64_t n, int64_t key0, int k, int sort_rows, float* __restrict__ out, float* __restrict__ parts,
+              unsigned int* status) {
     constexpr int d = V * 32;
     __shared__ int32_t s_idx[kSortCap];
     __shared__ float s_m[kWarps], s_l[kWarps];
@@ -142,12 +149,13 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
             for (int e = 0; e < kIdxRegs; ++e)
                 if ((mm >> 5) == e) i = __shfl_sync(0xffffffffu, my_idx[e], mm & 31);
             if (mm < rows_w) {
-                if (i >= 0 && i < n) {
+                const int64_t il = (int64_t)i - key0;   // row in this array
+                if (il >= 0 && il < n) {
                     ok[u] = true;
-                    const int64_t off = head_base + (int64_t)i * row_stride + lane * V;
+                    const int64_t off = head_base + il * row_stride + lane * V;
                     kw[u].load(Kr + off);
                     vw[u].load(Vr + off);
-                } else if (lane == 0) {
+                } else if (!parts && lane == 0) {   // a partial skips the other ranges' rows
                     atomicOr(status, (unsigned)FATHOM_DEV_BAD_INDEX);
                 }
             }
@@ -209,26 +217,63 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
             f[x] = (mx == -INFINITY) ? 0.0f : exp2f(mx - M);
             L = fmaf(*cluster.map_shared_rank(&c_l, x), f[x], L);
         }
+        float* ph = parts ? parts + (int64_t)h * (d + 2) : nullptr;
         for (int c = threadIdx.x; c < d; c += kThreads) {
             float O = 0.0f;
 #pragma unroll
             for (int x = 0; x < kSplit; ++x) O = fmaf(cluster.map_shared_rank(c_o, x)[c], f[x], O);
-            out[(int64_t)h * d + c] = (L > 0.0f) ? O / L : 0.0f;
+            if (ph) ph[c] = O;
+            else out[(int64_t)h * d + c] = (L > 0.0f) ? O / L : 0.0f;
+        }
+        if (ph && threadIdx.x == 0) {
+            ph[d] = M;
+            ph[d + 1] = L;
         }
     }
     cluster.sync();   // keep every CTA's shared memory alive until CTA 0 has read it
 }
 
+// Merge of per-range partials (o relative to m, m, l) of the same heads:
+// M = max_r m_r, L = sum_r l_r 2^(m_r - M), out = sum_r o_r 2^(m_r - M) / L,
+// ranges summed in order r = 0, 1, ...  One CTA per head.
+__global__ void __launch_bounds__(128)
+attend_merge_kernel(const float* __restrict__ parts, int world, int Hq, int d, float* __restrict__ out) {
+    const int h = blockIdx.x;
+    const int64_t rs = (int64_t)Hq * (d + 2);   // one range's partials
+    const float* p = parts + (int64_t)h * (d + 2);
+    float M = -INFINITY;
+    for (int r = 0; r < world; ++r) M = fmaxf(M, p[r * rs + d]);
+    float L = 0.0f;
+    for (int r = 0; r < world; ++r) {
+        const float mr = p[r * rs + d];
+        L = fmaf(p[r * rs + d + 1], (mr == -INFINITY) ? 0.0f : exp2f(mr - M), L);
+    }
+    for (int c = threadIdx.x; c < d; c += blockDim.x) {
+        float O = 0.0f;
+        for (int r = 0; r < world; ++r) {
+            const float mr = p[r * rs + d];
+            O = fmaf(p[r * rs + c], (mr == -INFINITY) ? 0.0f : exp2f(mr - M), O);
+        }
+        out[(int64_t)h * d + c] = (L > 0.0f) ? O / L : 0.0f;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_attend_merge(const float* parts, int world, int Hq, int d, float* out, cudaStream_t stream) {
+    attend_merge_kernel<<<(unsigned)Hq, 128, 0, stream>>>(parts, world, Hq, d, out);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
                           int64_t row_stride, const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k,
-                          int sort_rows, float* out, cudaStream_t stream) {
+                          int sort_rows, float* out, cudaStream_t stream, int64_t key0, float* parts) {
     dim3 grid((unsigned)(Hq * kSplit));
     unsigned int* st = device_status_ptr();
     const int sr = (sort_rows && k <= kSortCap) ? 1 : 0;
     auto go = [&](auto kern) {
-        kern<<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, row_stride, idx, Hq, Hkv, n, k, sr, out, st);
+        kern<<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, row_stride, idx, Hq, Hkv, n, key0, k, sr, out,
+                                            parts, st);
         return cudaGetLastError();
     };
     switch (d) {

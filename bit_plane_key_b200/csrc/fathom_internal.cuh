@@ -115,9 +115,13 @@ cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hk
                           const uint16_t* K_rows, const uint16_t* V_rows, int64_t row_stride, int64_t rows_n,
                           int rows_host, int groups, uint8_t* depths, int32_t* idx, float* top_scores, float* out,
                           void* workspace, cudaStream_t stream);
+// key0 / parts: the rows hold keys [key0, key0 + n) of a key range split
+// across GPUs; with parts non-null the kernel writes per-head partials
+// [Hq][d + 2] (o relative to m, then m, l) instead of out.
 cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
                           int64_t row_stride, const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k, int sort_rows, float* out,
-                          cudaStream_t stream);
+                          cudaStream_t stream, int64_t key0 = 0, float* parts = nullptr);
+cudaError_t launch_attend_merge(const float* parts, int world, int Hq, int d, float* out, cudaStream_t stream);
 
 cudaError_t launch_probe(const void* src, size_t bytes, unsigned long long* sink, int ctas,
                          cudaStream_t stream);

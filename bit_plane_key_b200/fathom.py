@@ -63,6 +63,8 @@ _sig("fathom_topk", _I, [_P, _P, _L, _L, _I, _I, _P, _P, _P, _Z, _P])
 _sig("fathom_scan_workspace_bytes", _Z, [_SP, _I, _I])
 _sig("fathom_scan_topk", _I, [_SP, _P, _I, _P, _I, _I, _P, _P, _P, _Z, _P])
 _sig("fathom_sparse_attend", _I, [_P, _I, _P, _P, _L, _I, _P, _I, _I, _L, _I, _I, _P, _P])
+_sig("fathom_sparse_attend_partial", _I, [_P, _I, _P, _P, _L, _I, _L, _P, _I, _I, _L, _I, _I, _P, _P])
+_sig("fathom_attend_merge", _I, [_P, _I, _I, _I, _P, _P])
 _sig("fathom_last_device_status", _I, [_P])
 _sig("fathom_status_string", ctypes.c_char_p, [_I])
 _sig("fathom_read_probe", _I, [_P, _Z, _I, _P, _I, _P])
@@ -319,6 +321,35 @@ def sparse_attend(q, K_rows, V_rows, idx, n_kv_heads=None, out=None, stream=None
     _check(_lib.fathom_sparse_attend(_ptr(q), _dtype_code(q), _ptr(K_rows), _ptr(V_rows), int(K_rows.stride(1)),
                                      int(host), _ptr(idx), Hq, Hkv, n, d, int(k), _ptr(out), _stream(stream)),
            "fathom_sparse_attend")
+    return out
+
+
+def sparse_attend_partial(q, K_rows, V_rows, idx, key0, n_kv_heads=None, parts=None, stream=None):
+    """Partials f32 [Hq][d + 2] (o relative to m, then m, l) of attention over
+    the rows this rank holds: K_rows/V_rows as sparse_attend, holding keys
+    [key0, key0 + n); idx are global key indices (others and -1 skipped)."""
+    Hq, d = q.shape
+    Hkv, n, _ = K_rows.shape
+    k = idx.shape[1]
+    host = not K_rows.is_cuda
+    if K_rows.stride() != V_rows.stride() or K_rows.stride(2) != 1 or K_rows.stride(0) != n * K_rows.stride(1):
+        raise ValueError("K_rows and V_rows need strides (n*s, s, 1), the same for both")
+    if parts is None:
+        parts = torch.empty((Hq, d + 2), dtype=torch.float32, device=q.device)
+    _check(_lib.fathom_sparse_attend_partial(_ptr(q), _dtype_code(q), _ptr(K_rows), _ptr(V_rows),
+                                             int(K_rows.stride(1)), int(host), int(key0), _ptr(idx), Hq, Hkv, n, d,
+                                             int(k), _ptr(parts), _stream(stream)),
+           "fathom_sparse_attend_partial")
+    return parts
+
+
+def attend_merge(parts, out=None, stream=None):
+    """o f32 [Hq][d] from the ranks' partials f32 [world][Hq][d + 2]."""
+    world, Hq, d2 = parts.shape
+    if out is None:
+        out = torch.empty((Hq, d2 - 2), dtype=torch.float32, device=parts.device)
+    _check(_lib.fathom_attend_merge(_ptr(parts.contiguous()), world, Hq, d2 - 2, _ptr(out), _stream(stream)),
+           "fathom_attend_merge")
     return out
 
 

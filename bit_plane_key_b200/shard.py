@@ -8,7 +8,10 @@ its local top-k; one all-gather of the (score, global index) pairs per query
 head follows, and fathom_topk_merge selects the top-k of all keys on every
 rank.  Because the ranges are ascending and each local list is in (score
 descending, index ascending) order, ties resolve to the lower global index,
-so the result equals the top-k of the unsplit scores.
+so the result equals the top-k of the unsplit scores.  Attention over the
+selected keys then runs on each rank over the rows it holds and writes
+per-head partials (o, m, l); one more all-gather and a GPU merge give every
+rank the full output.
 """
 
 
@@ -51,6 +54,38 @@ def local_topk(store_shard, key0, q, depths, k):
         idx = torch.cat([idx, torch.full((rows, k - kl), -1, dtype=idx.dtype, device=idx.device)], dim=1)
         top = torch.cat([top, torch.full((rows, k - kl), float("-inf"), dtype=top.dtype, device=top.device)], dim=1)
     return top.contiguous(), idx.contiguous()
+
+
+def gather_partials(parts, group=None):
+    """All-gather of every rank's attention partials [Hq][d + 2] into
+    [world][Hq][d + 2], rank by rank."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    out = [torch.empty_like(parts) for _ in range(world)]
+    dist.all_gather(out, parts.contiguous(), group=group)
+    return torch.stack(out).contiguous()
+
+
+def sharded_attend(q, K_rows, V_rows, key0, idx, n_kv_heads=None, group=None):
+    """Exact attention over the selected keys of a key-range-sharded layer:
+    each rank attends over the selected rows it holds (keys [key0, key0 +
+    n)), one all-gather of the per-head partials, the GPU merge.  Every rank
+    returns the same [Hq][d] output."""
+    from . import fathom as F
+    if K_rows.shape[1] == 0:   # an empty range: m = -inf, l = 0 for every head
+        parts = empty_partials(q.shape[0], q.shape[1], q.device)
+    else:
+        parts = F.sparse_attend_partial(q, K_rows, V_rows, idx, key0, n_kv_heads)
+    return F.attend_merge(gather_partials(parts, group))
+
+
+def empty_partials(n_q_heads, d, device):
+    """The partials of a rank that holds no selected row: o = 0, m = -inf, l = 0."""
+    import torch
+    parts = torch.zeros((n_q_heads, d + 2), dtype=torch.float32, device=device)
+    parts[:, d] = float("-inf")
+    return parts
 
 
 def sharded_scan_topk(store_shard, key0, q, depths, k, group=None):

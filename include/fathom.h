@@ -327,6 +327,33 @@ int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, con
                          int n_kv_heads, int64_t n, int d, int k, float* out, fathom_stream_t stream);
 
 /*
+ * Attention over a key range split across GPUs (not on the pages, whose
+ * system runs on one GPU).  Each rank holds the rows of keys [key0, key0 + n)
+ * and runs fathom_sparse_attend_partial with the merged global indices (see
+ * fathom_topk_merge): indices outside its range, and -1 padding, are skipped.
+ * It writes per-head partials instead of the output:
+ *   parts   device, f32 [Hq][d + 2]: o[0..d) = sum_j 2^(s_j - m) V_j over this
+ *           range's selected rows, then m = max_j s_j and l = sum_j 2^(s_j - m),
+ *           with s_j = q . K_j log2(e) / sqrt(d); a head with no row here has
+ *           m = -inf, l = 0.
+ * Other arguments as fathom_sparse_attend (K_rows / V_rows hold this range's
+ * n rows per KV head; key0 >= 0).  The ranks' partials are gathered (one
+ * all-gather of Hq (d + 2) floats per rank) and combined by
+ * fathom_attend_merge:
+ *   parts   device, f32 [world][Hq][d + 2], the ranks' partials.
+ *   out     device, f32 [Hq][d] = sum_r o_r 2^(m_r - M) / sum_r l_r 2^(m_r - M),
+ *           M = max_r m_r, ranks summed in order; 0 for a head with no rows.
+ * The result equals fathom_sparse_attend over all rows up to fp32 rounding
+ * (the partials are merged in a different order).
+ * Errors: as fathom_sparse_attend; EINVAL for key0 < 0, world < 1.
+ */
+int fathom_sparse_attend_partial(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
+                                 int64_t row_stride, int rows_host_resident, int64_t key0, const int32_t* idx,
+                                 int n_q_heads, int n_kv_heads, int64_t n, int d, int k, float* parts,
+                                 fathom_stream_t stream);
+int fathom_attend_merge(const float* parts, int world, int n_q_heads, int d, float* out, fathom_stream_t stream);
+
+/*
  * One decode step of one layer in one call: per-query depths, the scan, top-k
  * and exact attention over the selected rows.  [ai-feeds summary 方法: 输入,
  * 关键模块 2-5, 输出]  The results equal fathom_alloc_depths, then

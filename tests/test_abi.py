@@ -67,6 +67,14 @@ def test_null_arguments_rejected_before_any_cuda_call(libpath):
     assert L.fathom_sparse_attend(None, 0, None, None, 128, 0, None, 1, 1, 10, 128, 1, None, None) == F.EINVAL
     assert L.fathom_decode_step(None, None, 0, None, 4, 92, 0, 16, None, None, 10, 128, 0, 1, None, None, None,
                                 None, None, 0, None) == F.EINVAL
+    assert L.fathom_sparse_attend_partial(None, 0, None, None, 128, 0, 0, None, 1, 1, 10, 128, 1, None,
+                                          None) == F.EINVAL
+    assert L.fathom_attend_merge(None, 1, 1, 128, None, None) == F.EINVAL
+    # non-null but impossible sizes are rejected before the pointers are looked at
+    fake = ctypes.c_void_p(16)
+    assert L.fathom_sparse_attend_partial(fake, 0, fake, fake, 128, 0, -1, fake, 1, 1, 10, 128, 1, fake,
+                                          None) == F.EINVAL
+    assert L.fathom_attend_merge(fake, 0, 1, 128, fake, None) == F.EINVAL
 
 
 def test_decode_workspace_sizes(libpath):

@@ -140,3 +140,60 @@ def test_shard_ranges_cover_the_keys_on_aligned_cuts():
                 assert a1 == b0
             for a0, a1 in cuts:   # every non-empty range starts on a 1024-key cut; empty ones sit at n
                 assert (a0 % 1024 == 0) if a0 < a1 else (a0 == n)
+
+
+def _attn_rank_main(rank, world, port, outdir):
+    """Attention over a key range split across two gloo ranks: each rank forms
+    the (o, m, l) partials of the selected rows it holds (plain numpy here, the
+    layout fathom_sparse_attend_partial writes), the partials are all-gathered
+    rank by rank, and the log-sum-exp merge gives the full attention."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    from bit_plane_key_b200.ranks import Ranks
+    from bit_plane_key_b200.shard import gather_partials, shard_range
+    ranks = Ranks("gloo", device=torch.device("cpu"), timeout_s=60)
+    rng = np.random.default_rng(11)
+    Hq, d, n, k = 3, 16, 3000, 50
+    q = rng.standard_normal((Hq, d))
+    K = rng.standard_normal((n, d))
+    V = rng.standard_normal((n, d))
+    idx = np.stack([rng.choice(n, k, replace=False) for _ in range(Hq)])
+    idx[2] = np.arange(k)                       # head 2: every row in rank 0's range
+    k0, k1 = shard_range(n, world, rank)
+    parts = np.zeros((Hq, d + 2), np.float32)
+    for h in range(Hq):
+        sel = [i for i in idx[h] if k0 <= i < k1]
+        if not sel:
+            parts[h, d] = -np.inf
+            continue
+        s = K[sel] @ q[h] * np.log2(np.e) / np.sqrt(d)
+        m = s.max()
+        p = np.exp2(s - m)
+        parts[h, :d] = p @ V[sel]
+        parts[h, d], parts[h, d + 1] = m, p.sum()
+    allp = gather_partials(torch.from_numpy(parts)).numpy().astype(np.float64)
+    ranks.close()
+    M = allp[:, :, d].max(axis=0)
+    f = np.where(np.isinf(allp[:, :, d]), 0.0, np.exp2(allp[:, :, d] - M))
+    out = (allp[:, :, :d] * f[:, :, None]).sum(0) / (allp[:, :, d + 1] * f).sum(0)[:, None]
+    want = np.zeros((Hq, d))
+    for h in range(Hq):
+        s = K[idx[h]] @ q[h] / np.sqrt(d)
+        p = np.exp(s - s.max())
+        want[h] = p @ V[idx[h]] / p.sum()
+    with open(os.path.join(outdir, "attn%d.json" % rank), "w") as fh:
+        json.dump({"shape": list(allp.shape), "err": float(np.abs(out - want).max()),
+                   "m_rank1_head2": float(allp[1, 2, d]) if world > 1 else None}, fh)
+
+
+@pytest.mark.timeout(180)
+def test_sharded_attention_partials_on_two_gloo_ranks(tmp_path):
+    world = 2
+    mp.start_processes(_attn_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    for r in range(world):
+        x = json.load(open(tmp_path / ("attn%d.json" % r)))
+        assert x["shape"] == [world, 3, 18]
+        assert x["err"] < 1e-5                  # fp32 partials, fp64 merge
+        assert x["m_rank1_head2"] == float("-inf")   # rank 1 holds none of head 2's rows
