@@ -85,7 +85,7 @@ def _rel_err(got, want):
 @pytest.mark.parametrize("n,world,k,where,interleaved", [(20000, 4, 2048, "device", False),
                                                           (9000, 3, 512, "host", True),
                                                           (3000, 4, 1500, "device", True)])
-def test_sharded_attention_equals_unsplit(n, world, k, where, interleaved):
+def test_sharded_attention_equals_unsplit(ref, n, world, k, where, interleaved):
     inp = synth.layer_inputs(2, layer=5, n=n, n_kv_heads=2, n_q_heads=8, needles=0, with_values=True)
     q = torch.from_numpy(inp["q_bf16"].view(np.int16)).to(DEV).view(torch.bfloat16)
     dep = F.alloc_depths(q, torch.from_numpy(inp["sigma2"]).to(DEV), 92)
@@ -102,6 +102,9 @@ def test_sharded_attention_equals_unsplit(n, world, k, where, interleaved):
         parts.append(F.sparse_attend_partial(q, Kl, Vl, idx, k0))
     got = F.attend_merge(torch.stack(parts))
     assert _rel_err(got, want) <= 1e-5
+    # and against the oracle's fp64 attention over the same rows
+    oref = ref.attend(synth.bf16_bits_to_f32(inp["q_bf16"]), inp["K_rows"], inp["V_rows"], idx.cpu().numpy())
+    assert _rel_err(got.cpu().double(), torch.from_numpy(oref)) <= 1e-3
     assert F.last_device_status() == 0
 
 
@@ -117,7 +120,7 @@ def test_attend_merge_empty_ranges_and_padding():
     idx[3, -10:] = -1
     idx_d = torch.from_numpy(idx).to(DEV)
     Kf, Vf = _rows(inp, "device", True)
-    want = F.sparse_attend(q[:3], Kf, Vf, idx_d[:3].contiguous())
+    want = torch.cat([F.sparse_attend(q[h:h + 1], Kf, Vf, idx_d[h:h + 1].contiguous()) for h in range(3)])
     want3 = F.sparse_attend(q[3:], Kf, Vf, idx_d[3:, :k - 10].contiguous())
     parts = []
     for k0, k1 in ((0, 3072), (3072, n)):
