@@ -604,10 +604,18 @@ def config_bench(args):
             U = dep.view(S, 8, 4, 128)[sidx].amax(dim=1)
             nbytes += st.plane_bytes_read(U)
         ms = float(np.median(t))
+        # the oracle on session 0's first KV group (single thread), scaled to the
+        # step's keys x KV heads
+        st0 = stores[0]
+        t0 = time.perf_counter()
+        oracle.decode(st0.planes[0:1].cpu().numpy().view(np.uint32), st0.scales[0:1].cpu().numpy().view(np.uint16),
+                      lengths[0], qs[0][:4].float().cpu().numpy(), s2s[0][0:1].cpu().numpy(), B, k)
+        t_or = time.perf_counter() - t0
         out.append({"config": 4, "case": "16 sessions batched", "workload": cfg["name"], "sessions": S,
                     "total_keys": sum(lengths), "step_ms": ms, "gkeys_per_s": keys / (ms * 1e-3) / 1e9,
                     "scan_bytes_per_key_per_kv_head": nbytes / keys, "link_gbs": nbytes / (ms * 1e-3) / 1e9,
-                    "launches_per_step": 1 + 1 + 9})
+                    "launches_per_step": 1 + 1 + 9, "oracle_s_session0_kv_group0": t_or, "oracle_cores": 1,
+                    "oracle_s_step_extrapolated": t_or * keys / lengths[0]})
     elif args.config == 5:
         cfg = synth.CONFIGS[5]
         n, L = cfg["n"], cfg["layers"]
@@ -636,9 +644,20 @@ def config_bench(args):
                 F.decode_step(st, qd, s2d, b, k, Kr, Vr, **bufs)
         t = _events_ms(torch, token, max(3, args.steps // 3), 1, flush)
         ms = float(np.median(t))
+        # the oracle on layer 0's first KV group (single thread), extrapolated to
+        # the token (8 KV groups x 36 layers) and labelled as such
+        st0, q0, s20, b0 = layers[0]
+        t0 = time.perf_counter()
+        oracle.decode(st0.planes[0:1].cpu().numpy().view(np.uint32), st0.scales[0:1].cpu().numpy().view(np.uint16), n,
+                      q0[:4].float().cpu().numpy(), s20[0:1].cpu().numpy(), b0, k,
+                      K_rows=Kr[0:1].contiguous().view(torch.int16).numpy().view(np.uint16),
+                      V_rows=Vr[0:1].contiguous().view(torch.int16).numpy().view(np.uint16))
+        t_or = time.perf_counter() - t0
         out.append({"config": 5, "case": "36-layer decode token", "workload": cfg["name"], "layers": L, "n": n,
                     "budgets_mean": float(np.mean(budgets)), "token_ms": ms, "per_layer_ms": ms / L,
-                    "gkeys_per_s": n * 8 * L / (ms * 1e-3) / 1e9, "kv_rows": "one buffer shared by all layers"})
+                    "gkeys_per_s": n * 8 * L / (ms * 1e-3) / 1e9, "kv_rows": "one buffer shared by all layers",
+                    "oracle_s_layer0_kv_group0": t_or, "oracle_cores": 1,
+                    "oracle_s_token_extrapolated": t_or * 8 * L})
     for line in out:
         print(json.dumps(line), flush=True)
 
