@@ -289,29 +289,66 @@ class Layer:
         return self.store.plane_bytes_read(U), U
 
     @staticmethod
-    def launches_per_step(groups):
-        # depths, then per group: scan, top-k (init, 3x hist+select, compact, finish), attention
-        return 1 + groups * (1 + 9 + 1)
+    def launches_per_step(groups, n, k):
+        """Kernels one decode step launches: depths, then per group of KV heads
+        the scan, the top-k and the attention."""
+        return 1 + groups * (1 + topk_launches(n, k) + 1)
+
+
+def topk_launches(n, k, n_max=None):
+    """Launches of one top-k call after the scan (the path fathom_scan_topk
+    takes) on rows of n keys (the shortest row, for ragged batches; n_max the
+    longest): rows with at least 8k blocks of 64 keys take the block-maxima
+    path (threshold, compaction, final sort); rows of at most 131072 keys one
+    cluster kernel; other rows the histogram path (init, level-0 histogram and
+    select, two refine levels of histogram and select, compaction, final
+    sort)."""
+    n_max = n if n_max is None else n_max
+    if n // 64 >= 8 * k:
+        return 3
+    if n_max <= 131072:
+        return 1
+    return 9
+
+
+# Link / DRAM bytes per unit (key x KV head) of the scan kernel, from one ncu
+# capture each (the summaries and commands are in profiles/); the sha256 is
+# that of scan.cu when the counters were taken.
+SCAN_TRAFFIC = {}
 
 
 def profiled_traffic(resident, units):
-    """Bytes per scan launch from the committed ncu capture of this scan
-    kernel (profiles/scan_*), scaled to `units` keys x KV heads; None when
-    scan.cu has changed since that capture."""
+    """Bytes per scan launch from the recorded ncu capture of this scan
+    kernel, scaled to `units` keys x KV heads; (None, reason) when scan.cu has
+    changed since that capture or none was recorded."""
     import hashlib
-    name = "scan_host_n262144_traffic.md" if resident == "host" else "scan_hbm_n1M_B92.md"
-    path = os.path.join(ROOT, "profiles", name)
-    if not os.path.exists(path):
-        return None, None
-    rec = None
-    for line in open(path):
-        if line.startswith("traffic_json:"):
-            rec = json.loads(line.split(":", 1)[1])
+    rec = SCAN_TRAFFIC.get(resident)
     src = os.path.join(ROOT, "bit_plane_key_b200", "csrc", "scan.cu")
-    if rec is None or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["kernel_src_sha256"]:
-        return None, None
-    return rec["bytes_per_unit"] * units, "%s from profiles/%s, scaled from %d to %d units" % (
-        rec["counter"], name, rec["captured_units"], units)
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if rec is None or rec["kernel_src_sha256"] != sha:
+        return None, "no ncu capture of the current scan.cu"
+    return rec["bytes_per_unit"] * units, "scaled ncu capture: %s per unit from %s (%d units), times %d units" % (
+        rec["counter"], rec["capture"], rec["captured_units"], units)
+
+
+def gqa_overlap(idx, G):
+    """How much the query heads of one KV head agree in their selections:
+    distinct rows per KV head / (G * k), averaged over KV heads (1.0 = no key
+    selected twice), and the share of selected keys that another head of the
+    group also selected."""
+    Hq, k = idx.shape
+    ratios, shared = [], []
+    for g in range(Hq // G):
+        sets = [set(idx[g * G + h].tolist()) for h in range(G)]
+        union = set().union(*sets)
+        ratios.append(len(union) / (G * k))
+        counts = {}
+        for st in sets:
+            for i in st:
+                counts[i] = counts.get(i, 0) + 1
+        shared.append(sum(1 for st in sets for i in st if counts[i] > 1) / (G * k))
+    return {"distinct_rows_per_kv_head_over_Gk": float(np.mean(ratios)),
+            "selected_by_another_head_of_group": float(np.mean(shared))}
 
 
 def link_peak(F, torch, dev, nbytes=1 << 30, reps=10):
@@ -614,7 +651,8 @@ def config_bench(args):
         out.append({"config": 4, "case": "16 sessions batched", "workload": cfg["name"], "sessions": S,
                     "total_keys": sum(lengths), "step_ms": ms, "gkeys_per_s": keys / (ms * 1e-3) / 1e9,
                     "scan_bytes_per_key_per_kv_head": nbytes / keys, "link_gbs": nbytes / (ms * 1e-3) / 1e9,
-                    "launches_per_step": 1 + 1 + 9, "oracle_s_session0_kv_group0": t_or, "oracle_cores": 1,
+                    "launches_per_step": 1 + 1 + topk_launches(min(lengths), k, max(lengths)),
+                    "oracle_s_session0_kv_group0": t_or, "oracle_cores": 1,
                     "oracle_s_step_extrapolated": t_or * keys / lengths[0]})
     elif args.config == 5:
         cfg = synth.CONFIGS[5]
@@ -802,6 +840,7 @@ def main():
     needles = set(layer.inp.get("needles", np.array([], np.int64)).tolist())
     idx0 = set(layer.idx[0].cpu().numpy().tolist())
     recall = len(needles & idx0) / len(needles) if needles else None
+    overlap = gqa_overlap(layer.idx.cpu().numpy(), layer.Hq // layer.Hkv)
 
     extras = {}
     if not args.no_extras:
@@ -889,8 +928,8 @@ def main():
                         "note": "q and sigma2 copied in and idx + attention output read back every step; the "
                                 "bit planes and K/V rows stay in page-locked host memory and cross the link "
                                 "inside the scan and attention kernels"},
-                "gpu_launches": Layer.launches_per_step(groups) * args.steps,
-                "needle_recall_head0": recall, "cpu_baseline": cpu, "compare": extras}
+                "gpu_launches": Layer.launches_per_step(groups, args.n, args.k) * args.steps,
+                "needle_recall_head0": recall, "gqa_selection": overlap, "cpu_baseline": cpu, "compare": extras}
         print(json.dumps(line), flush=True)
     ranks.close()
 

@@ -1,5 +1,7 @@
 // C-ABI entry points of libfathom: argument checks, pointer classification,
 // kernel launches.  Declarations and contracts: include/fathom.h.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "fathom_internal.cuh"
@@ -11,10 +13,52 @@ namespace {
 __device__ unsigned int g_status;
 
 constexpr int kMaxDevices = 64;
-unsigned int* g_status_ptr[kMaxDevices] = {};
+CtxCache g_status_ptr[kMaxDevices];
 std::mutex g_status_mu;
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+std::once_flag g_ctx_fn_once;
+
 }  // namespace
+
+unsigned long long current_context_id() {
+    // the driver's functions through the runtime, so that the library needs
+    // no link to libcuda (it loads on machines without a GPU driver)
+    std::call_once(g_ctx_fn_once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult r;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &r) == cudaSuccess &&
+            r == cudaDriverEntryPointSuccess)
+            g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &r) == cudaSuccess &&
+            r == cudaDriverEntryPointSuccess)
+            g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f);
+        cudaGetLastError();
+    });
+    if (!g_ctx_get_current || !g_ctx_get_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    if (g_ctx_get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+void* CtxCache::get(const void* symbol) {
+    const unsigned long long id = current_context_id();
+    if (ptr && id != 0 && id == ctx) return ptr;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    ptr = p;
+    ctx = current_context_id();   // the look-up creates the context if there was none
+    return ptr;
+}
 
 // Where a pointer lives.  Returns the device-usable address through `dev`.
 Where classify(const void* p, const void** dev) {
@@ -54,7 +98,7 @@ int resolve_store(const fathom_store* s, const uint32_t** planes, const uint16_t
     if (!s || !s->planes || !s->scales) return FATHOM_EINVAL;
     if (!dims_ok(s->n_kv_heads, s->d) || s->n < 1 || s->n_pad < n_pad_of(s->n) || s->n_pad % kPad)
         return FATHOM_EINVAL;
-    if ((reinterpret_cast<uintptr_t>(s->planes) & 15) || (reinterpret_cast<uintptr_t>(s->scales) & 1))
+    if ((reinterpret_cast<uintptr_t>(s->planes) & 15) || (reinterpret_cast<uintptr_t>(s->scales) & 15))
         return FATHOM_EINVAL;
     const void* dp = nullptr;
     const void* ds = nullptr;
@@ -70,12 +114,7 @@ unsigned int* device_status_ptr() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(g_status_mu);
-    if (!g_status_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
-        g_status_ptr[dev] = static_cast<unsigned int*>(p);
-    }
-    return g_status_ptr[dev];
+    return static_cast<unsigned int*>(g_status_ptr[dev].get(&g_status));
 }
 
 }  // namespace fathom
@@ -164,7 +203,8 @@ int fathom_scan_scores(const fathom_store* store, const void* q, int q_dtype, co
     if (!scan_fits(store->d, n_q_heads, store->n_kv_heads)) return FATHOM_EUNSUPPORTED;
     if (!device_status_ptr()) return FATHOM_ECUDA;
     return to_status(launch_scan(planes, scales, store->n_kv_heads, store->d, store->n, store->n_pad, q, q_dtype,
-                                 depths, n_q_heads, scores, (cudaStream_t)stream, block_max));
+                                 depths, n_q_heads, scores, (cudaStream_t)stream, block_max,
+                                 store->host_resident != 0));
 }
 
 size_t fathom_topk_workspace_bytes(int64_t n, int n_rows, int k) {
@@ -233,7 +273,7 @@ int fathom_scan_topk(const fathom_store* store, const void* q, int q_dtype, cons
     uint32_t* bmax = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + lay.bmax_off);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = launch_scan(planes, scales, store->n_kv_heads, store->d, store->n, store->n_pad, q, q_dtype,
-                                depths, n_q_heads, scores, s, bmax);
+                                depths, n_q_heads, scores, s, bmax, store->host_resident != 0);
     if (e != cudaSuccess) return FATHOM_ECUDA;
     e = launch_topk_blocks(scores, bmax, store->n, ld, n_q_heads, k, idx, top_scores,
                            static_cast<char*>(workspace) + lay.topk_off, s);
@@ -285,8 +325,10 @@ int fathom_scan_topk_batched(const fathom_store* stores, int n_sessions, const v
     rm.max_n = 0;
     int tiles = 0;
     size_t off = 0;
+    bool any_host = false;
     for (int s = 0; s < n_sessions; ++s) {
         const fathom_store& st = stores[s];
+        any_host = any_host || st.host_resident != 0;
         if (k > st.n || st.n > INT32_MAX) return FATHOM_EINVAL;
         int rc = resolve_store(&st, &sm.planes[s], &sm.scales[s]);
         if (rc) return rc;
@@ -294,7 +336,7 @@ int fathom_scan_topk_batched(const fathom_store* stores, int n_sessions, const v
         sm.n_pad[s] = st.n_pad;
         sm.score_base[s] = (int64_t)(off / sizeof(float));
         sm.tile0[s] = tiles;
-        const int64_t t = n_pad_of(st.n) / 1024;
+        const int64_t t = scan_tiles(st.n);
         if (t > INT32_MAX - tiles) return FATHOM_EINVAL;
         tiles += (int)t;
         rm.base[s] = sm.score_base[s];
@@ -314,7 +356,7 @@ int fathom_scan_topk_batched(const fathom_store* stores, int n_sessions, const v
     uint32_t* bmax = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + off);
     cudaStream_t cs = (cudaStream_t)stream;
     cudaError_t e = launch_scan_batched(sm, stores[0].n_kv_heads, stores[0].d, q, q_dtype, depths, n_q_heads, scores,
-                                        cs, bmax);
+                                        cs, bmax, any_host);
     if (e != cudaSuccess) return FATHOM_ECUDA;
     return to_status(launch_topk_blocks_map(scores, bmax, rm, n_sessions * n_q_heads, k, idx, top_scores,
                                             static_cast<char*>(workspace) + off + a256(off / kBlock), cs));
@@ -409,7 +451,8 @@ int fathom_decode_step(const fathom_store* store, const void* q, int q_dtype, co
         !is_device(workspace) || (top_scores && !is_device(top_scores)))
         return FATHOM_EINVAL;
     if (!device_status_ptr()) return FATHOM_ECUDA;
-    return to_status(launch_decode(planes, scales, Hkv, d, n, store->n_pad, q, q_dtype, sigma2, n_q_heads,
+    return to_status(launch_decode(planes, scales, store->host_resident, Hkv, d, n, store->n_pad, q, q_dtype, sigma2,
+                                   n_q_heads,
                                    budget_bits, fixed_r, k, static_cast<const uint16_t*>(kd),
                                    static_cast<const uint16_t*>(vd), row_stride, rows_n, rows_host_resident, kv_groups,
                                    depths, idx, top_scores, out, workspace, (cudaStream_t)stream));

@@ -25,6 +25,7 @@ constexpr int kMaxDevices = 64;
 constexpr int kMaxGroups = 64;
 
 struct Aux {
+    unsigned long long ctx = 0;             // id of the context the handles belong to
     cudaStream_t stream = nullptr;
     cudaEvent_t scanned[kMaxGroups] = {};   // group i's scores are written
     cudaEvent_t done = nullptr;             // the auxiliary stream's work is finished
@@ -32,21 +33,29 @@ struct Aux {
 Aux g_aux[kMaxDevices];
 std::mutex g_aux_mu;
 
-// The current device's auxiliary stream and events, created on first use.
-// Calls on one device share them: steps issued concurrently from several host
-// threads serialise their top-k and attention on the one auxiliary stream.
+// The current device's auxiliary stream and events, created on first use in
+// each context (after cudaDeviceReset the old handles are gone with their
+// context, and new ones are made).  Calls on one device share them: steps
+// issued concurrently from several host threads serialise their top-k and
+// attention on the one auxiliary stream.
 Aux* aux_for_device() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(g_aux_mu);
     Aux& a = g_aux[dev];
-    if (!a.stream) {
+    const unsigned long long id = current_context_id();
+    // a new set on first use, and when the context is known to have changed
+    // (when the driver cannot name the context, the first set is kept)
+    if (!a.stream || (id != 0 && id != a.ctx)) {
+        Aux fresh;
         cudaStream_t s = nullptr;
         if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
         for (int i = 0; i < kMaxGroups; ++i)
-            if (cudaEventCreateWithFlags(&a.scanned[i], cudaEventDisableTiming) != cudaSuccess) return nullptr;
-        if (cudaEventCreateWithFlags(&a.done, cudaEventDisableTiming) != cudaSuccess) return nullptr;
-        a.stream = s;
+            if (cudaEventCreateWithFlags(&fresh.scanned[i], cudaEventDisableTiming) != cudaSuccess) return nullptr;
+        if (cudaEventCreateWithFlags(&fresh.done, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+        fresh.stream = s;
+        fresh.ctx = current_context_id();   // creating the stream made the context if there was none
+        a = fresh;
     }
     return &a;
 }
@@ -57,8 +66,8 @@ size_t decode_workspace_bytes(int64_t n, int Hq, int groups, int k) {
     return scan_topk_layout(n, Hq, Hq / groups, k).total;
 }
 
-cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n, int64_t n_pad,
-                          const void* q, int q_dtype, const float* sigma2, int Hq, int budget, int fixed_r, int k,
+cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int store_host, int Hkv, int d, int64_t n,
+                          int64_t n_pad, const void* q, int q_dtype, const float* sigma2, int Hq, int budget, int fixed_r, int k,
                           const uint16_t* K_rows, const uint16_t* V_rows, int64_t row_stride, int64_t rows_n,
                           int rows_host, int groups, uint8_t* depths, int32_t* idx, float* top_scores, float* out,
                           void* workspace, cudaStream_t stream) {
@@ -81,7 +90,8 @@ cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hk
         float* si = scores + (size_t)h0 * ld;
         uint32_t* bi = bmax + (size_t)h0 * (ld / kBlock);
         e = launch_scan(planes + (size_t)g0 * d * 4 * (n_pad / 32), scales + (size_t)g0 * d * (n_pad / kBlock),
-                        hkv_g, d, n, n_pad, qi, q_dtype, depths + (size_t)h0 * d, hq_g, si, stream, bi);
+                        hkv_g, d, n, n_pad, qi, q_dtype, depths + (size_t)h0 * d, hq_g, si, stream, bi,
+                        store_host != 0);
         if (e == cudaSuccess) e = cudaEventRecord(aux->scanned[i], stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(aux->stream, aux->scanned[i], 0);
         int32_t* ii = idx + (size_t)h0 * k;

@@ -18,9 +18,29 @@ constexpr size_t kMaxSmem = 227 * 1024;  // opt-in shared memory per CTA on sm_1
 
 __host__ __device__ inline int64_t n_pad_of(int64_t n) { return ((n + kPad - 1) / kPad) * kPad; }
 
+// Keys per CTA of the scan; the last tile of a store may hold kScanTile / 2
+// keys (n_pad_of(n) is a multiple of 1024).
+constexpr int kScanTile = 2048;
+__host__ __device__ inline int64_t scan_tiles(int64_t n) { return (n_pad_of(n) + kScanTile - 1) / kScanTile; }
+
 // Per-device status word (FATHOM_DEV_* bits); its device address is passed
 // to every kernel that can set a bit.
 unsigned int* device_status_ptr();
+
+// Unique id of the calling thread's current CUDA context (the driver's
+// cuCtxGetId), 0 when there is none or the driver cannot say.  A device reset
+// ends the context, and the next one has a new id.
+unsigned long long current_context_id();
+
+// The device address of a __device__ variable, looked up once per context:
+// cached with the id of the context it was looked up in, and looked up again
+// when the current context differs (after cudaDeviceReset the module is
+// loaded anew and the variable may move).  Callers hold their own lock.
+struct CtxCache {
+    unsigned long long ctx = 0;
+    void* ptr = nullptr;
+    void* get(const void* symbol);
+};
 
 // Host-side argument checks shared by the entry points (api.cu).
 enum class Where { kDevice, kHostPinned, kOther };
@@ -44,10 +64,11 @@ cudaError_t launch_depths(const void* q, int q_dtype, const float* sigma2, int H
                           int budget, int fixed_r, uint8_t* depths, cudaStream_t stream, int pooled = 0);
 size_t scan_smem_bytes(int d, int G);
 // bmax (optional): the max score of every 64-key block as an ordered key,
-// [Hq][n_pad_of(n)/64], for launch_topk_blocks
+// [Hq][n_pad_of(n)/64], for launch_topk_blocks; host: the store is in
+// page-locked host memory (planes and scales are its device-mapped addresses)
 cudaError_t launch_scan(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n,
                         int64_t n_pad, const void* q, int q_dtype, const uint8_t* depths, int Hq,
-                        float* scores, cudaStream_t stream, uint32_t* bmax = nullptr);
+                        float* scores, cudaStream_t stream, uint32_t* bmax, bool host);
 size_t topk_workspace_bytes(int64_t n, int rows, int k);
 
 // Where the score rows are: rows are grouped in sets of `rows_per_set`
@@ -106,12 +127,13 @@ struct SessionMap {
     int64_t score_base[kMaxSets];
     int tile0[kMaxSets + 1];
 };
+// host: some session's store is in page-locked host memory
 cudaError_t launch_scan_batched(const SessionMap& map, int Hkv, int d, const void* q, int q_dtype,
                                 const uint8_t* depths, int Hq, float* scores, cudaStream_t stream,
-                                uint32_t* bmax = nullptr);
+                                uint32_t* bmax, bool host);
 size_t decode_workspace_bytes(int64_t n, int Hq, int groups, int k);
-cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n, int64_t n_pad,
-                          const void* q, int q_dtype, const float* sigma2, int Hq, int budget, int fixed_r, int k,
+cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int store_host, int Hkv, int d, int64_t n,
+                          int64_t n_pad, const void* q, int q_dtype, const float* sigma2, int Hq, int budget, int fixed_r, int k,
                           const uint16_t* K_rows, const uint16_t* V_rows, int64_t row_stride, int64_t rows_n,
                           int rows_host, int groups, uint8_t* depths, int32_t* idx, float* top_scores, float* out,
                           void* workspace, cudaStream_t stream);

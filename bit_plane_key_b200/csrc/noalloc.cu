@@ -15,7 +15,10 @@
 // Host code must not pass the array's name to a kernel: on the host that
 // name is only a stand-in, not a device address.  The first call on a device
 // looks the device address up with cudaGetSymbolAddress (with that device
-// current) and caches it; make that first call before any stream capture.
+// current) and caches it together with the id of the current context; a later
+// call in another context (after cudaDeviceReset) looks it up again.  Make the
+// first call on a device, and the first after a reset, before any stream
+// capture.
 // All calls share the one array and it keeps the previous call's contents:
 // the top-k clears its own counters and histograms at the start of every
 // call, and the scan overwrites every score it later reads.  Calls whose
@@ -33,20 +36,17 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
-void* g_scratch_dev[kMaxDevices] = {};
+CtxCache g_scratch_dev[kMaxDevices];
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device (set up once).
+// Device address of the scratch array on the current device: looked up with
+// cudaGetSymbolAddress, with that device current, on the first call in each
+// context, and cached with the context's id.
 void* scratch_address() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_dev[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-        g_scratch_dev[dev] = p;
-    }
-    return g_scratch_dev[dev];
+    return g_scratch_dev[dev].get(g_noalloc_scratch);
 }
 
 }  // namespace
@@ -83,7 +83,7 @@ int fathom_scan_topk_noalloc(const fathom_store* store, const void* q, int q_dty
     uint32_t* bmax = reinterpret_cast<uint32_t*>(scratch + lay.bmax_off);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = launch_scan(planes, scales, store->n_kv_heads, store->d, store->n, store->n_pad, q, q_dtype,
-                                depths, n_q_heads, scores, s, bmax);
+                                depths, n_q_heads, scores, s, bmax, store->host_resident != 0);
     if (e != cudaSuccess) return FATHOM_ECUDA;
     return to_status(launch_topk_blocks(scores, bmax, store->n, ld, n_q_heads, k, idx, top_scores,
                                         scratch + lay.topk_off, s));

@@ -10,73 +10,76 @@
 // 关键模块 5: only the budgeted planes are pulled); channels nobody reads are
 // never touched, nor are their scales.
 //
-// Arithmetic.  Let code be the channel's 4-bit code with the unread planes
-// as zero bits and P_t = code with its low 4-t bits cleared (the t-bit prefix
-// in place).  With F_t = 1/2 (1 + P_t/16), an fp32 number whose mantissa bits
-// 22..19 are exactly P_t,
+// Arithmetic.  Let P_t be the channel's 4-bit code with its low 4-t bits
+// cleared (the t-bit prefix in place).  With F_t = 1/2 (1 + P_t/16), an fp32
+// number whose mantissa bits 22..19 are exactly P_t,
 //   v_t = 2^(3-t)(2m + 1) - 8 = 32 F_t - 24 + 2^(3-t),
-// so a (channel, head) pair adds (32 q Delta) F_t per key, and
-// Delta q (2^(3-t) - 24) per (block, head) once.
+// so a (channel, head) pair adds W F_t per key with W = 32 q Delta, and
+// Delta q (2^(3-t) - 24) per (block, head) once.  One byte permute builds F_t
+// from a code byte; W F_t products are exact in fp32 for bf16 q.
 //
-// Work.  One CTA per (tile of 1024 keys, KV head).  A channel's codes in a
-// tile are 8 x 32 words: word (s, w) holds the codes of keys 32w + s + 8k,
-// k = 0..3, one per byte at bits 6..3.  The tile's active channels
-// (U_c > 0) are streamed in chunks of 16:
-//   stage: thread (channel group, plane word w) loads the U_c plane words of
-//     its channels (row pointers prepared once per tile) and transposes them
-//     to the 8 code words (s, w) (planes paired, then merged to nibbles, one
-//     rotate + mask per word), stored with conflict-free 32-bit stores.  Thread (channel, block) pairs form
-//     the coefficients 32 q Delta of every head and add Delta q (2^(3-t) - 24)
-//     into a per-(block, head) constant kept in registers.
-//   compute: warp (head h, key split) walks head h's item list of the chunk:
-//     the channels h reads, first those read to the union depth, then those
-//     read to fewer planes (their code bytes masked to t planes).  Lane
-//     (block b, variant half) owns 32 / S keys of block b: per item one
-//     coefficient load, 64-bit loads of its code words, and per key one byte
-//     permute building F and one FMA.  No per-head branch, no unread channel.
-//   The next chunk's plane words and scales are loaded into registers before
-//   the current chunk is computed, so the loads overlap the arithmetic.
-// The same kernel serves a host-resident store: its loads then cross the host
-// link as 128-byte runs per (channel, plane) and tile.
+// Work.  One CTA per (tile of 2048 keys, KV head); the G query heads of the
+// KV head form groups of up to 4 heads, and each group has 128 threads.  A
+// thread owns 16 keys of one 64-key block (4 threads per block) and the
+// accumulators of every head of its group, so a code value F_t is built once
+// per key and shared by all heads of the group that read the channel to depth
+// t.  The tile's active channels (U_c > 0) are streamed in chunks of 8:
+//   load:  the chunk's U_c plane rows (256 bytes each in the tile) and scale
+//          rows go to shared memory one chunk ahead of use: by cp.async from a
+//          device-resident store; by 16-byte loads held in registers until
+//          the current chunk is computed from a host-resident one (over the
+//          host link each warp's loads are then runs of whole lines);
+//   stage: thread (channel, block) transposes its 2 x U_c plane words into 16
+//          code words (4 keys each, code at bits 6..3 of a byte) with a few
+//          shifts and masks; thread (block, head) forms the head's
+//          coefficients W (stored twice, for paired FMAs) of every channel of
+//          the chunk and adds Delta q (2^(3-t) - 24) to the block's constant;
+//   compute: the group's items, one per (channel, distinct depth), in channel
+//          order: per item one 128-bit load of the thread's 16 code bytes,
+//          masked to the item's depth, 16 byte permutes, and for each head
+//          that reads the channel to that depth (a uniform branch) 8 paired
+//          FMAs (fma.rn.f32x2) over 2 keys each.
 #include "fathom_internal.cuh"
 
 namespace fathom {
 namespace {
 
-constexpr int kTileKeys = 1024;
-constexpr int kTileWords = kTileKeys / 32;   // 32 plane words per tile row
-constexpr int kTileBlocks = kTileKeys / kBlock;
-constexpr int kChanWords = 8 * kTileWords;   // code words of one channel in a tile
-constexpr int kChunk = 16;                   // active channels per stage
+constexpr int kTile = kScanTile;             // keys per CTA
+constexpr int kNB = kTile / kBlock;          // 64-key blocks per tile
+constexpr int kTW = kTile / 32;              // plane words per row in a tile
+constexpr int kCH = 8;                       // active channels per chunk
+constexpr int kMaxItems = 4 * kCH;           // items per (head group, chunk)
 constexpr uint32_t kHalfExp = 0x3F000000u;   // bits of 0.5f: exponent byte of F
 
 // Launch geometry for G query heads per KV head.
 template <int G>
 struct Geo {
-    static constexpr int S = G >= 4 ? 1 : 4 / G;    // warps per query head (key splits)
-    static constexpr int NW = G * S;                // warps per CTA
-    static constexpr int T = 32 * NW;               // threads per CTA
-    static constexpr int NSV = 4 / S;               // code variants per compute thread
-    static constexpr int CPT = kChunk / NW;         // staged channels per thread
-    static constexpr int DPT = kChunk * kTileBlocks / T;   // staged (channel, block) scales per thread
-    static constexpr int MinBlocks = T <= 128 ? 4 : 2;
-    static_assert(CPT >= 1 && DPT >= 1 && NSV >= 1, "geometry");
+    static constexpr int HG = G < 4 ? G : 4;   // heads per head group
+    static constexpr int NHG = G / HG;         // head groups
+    static constexpr int TPG = kNB * 4;        // threads per head group (4 per block)
+    static constexpr int T = TPG * NHG;        // threads per CTA
+    // host-resident stores hold the next chunk's rows in registers (see scan_tile)
+    template <bool HOST>
+    static constexpr int min_blocks() { return HOST ? (T <= 128 ? 3 : 1) : (T <= 128 ? 4 : 2); }
 };
 
-// Shared memory of one CTA (byte offsets; every region 16-byte aligned for d % 32 == 0).
+// Shared memory of one CTA (byte offsets; every region 16-byte aligned).
 struct ScanSmem {
     int d, G;
-    __host__ __device__ size_t codes() const { return 0; }   // [2][kChunk][8][32] u32
-    __host__ __device__ size_t coef() const { return codes() + 2u * kChunk * kChanWords * 4; }   // [2][G][kChunk][16] f32
-    __host__ __device__ size_t prow() const { return coef() + 2u * G * kChunk * kTileBlocks * 4; }   // [d] plane-0 row ptr
-    __host__ __device__ size_t srow() const { return prow() + (size_t)d * 8; }      // [d] scale row ptr
-    __host__ __device__ size_t items() const { return srow() + (size_t)d * 8; }     // [G][d] u32
-    __host__ __device__ size_t q32() const { return items() + (size_t)G * d * 4; }   // [d][G] f32
-    __host__ __device__ size_t qk() const { return q32() + (size_t)G * d * 4; }      // [d][G] f32
-    __host__ __device__ size_t off() const { return qk() + (size_t)G * d * 4; }      // [G][d/8 + 4] i32
-    __host__ __device__ size_t act() const { return off() + (size_t)G * (d / 8 + 4) * 4; }   // [d] i32
-    __host__ __device__ size_t uni() const { return act() + (size_t)d * 4; }         // [d] u8
-    __host__ __device__ size_t tdep() const { return uni() + (size_t)d; }            // [G][d] u8
+    __host__ __device__ int hg() const { return G < 4 ? G : 4; }
+    __host__ __device__ int nhg() const { return G / hg(); }
+    __host__ __device__ int maxchunks() const { return (d + kCH - 1) / kCH; }
+    __host__ __device__ size_t raw() const { return 0; }                                   // [2][kCH][4][kTW] u32
+    __host__ __device__ size_t rawsc() const { return raw() + 2u * kCH * 4 * kTW * 4; }    // [2][kCH][kNB] u16
+    __host__ __device__ size_t codes() const { return rawsc() + 2u * kCH * kNB * 2; }      // [kCH][kNB][8][2] u32
+    __host__ __device__ size_t w2() const { return codes() + (size_t)kCH * kNB * 16 * 4; } // [nhg][kCH][kNB][hg][2] f32
+    __host__ __device__ size_t q32() const { return w2() + (size_t)nhg() * kCH * kNB * hg() * 8; }   // [d][G] f32
+    __host__ __device__ size_t qk() const { return q32() + (size_t)d * G * 4; }            // [d][G] f32
+    __host__ __device__ size_t items() const { return qk() + (size_t)d * G * 4; }          // [nhg*maxchunks][kMaxItems] u32
+    __host__ __device__ size_t act() const { return items() + (size_t)nhg() * maxchunks() * kMaxItems * 4; }   // [d] i32
+    __host__ __device__ size_t nitems() const { return act() + (size_t)d * 4; }            // [nhg*maxchunks] u8
+    __host__ __device__ size_t uni() const { return nitems() + (size_t)nhg() * maxchunks(); }   // [d] u8
+    __host__ __device__ size_t tdep() const { return uni() + (size_t)d; }                  // [G][d] u8
     __host__ __device__ size_t bytes() const { return (tdep() + (size_t)G * d + 15) & ~size_t(15); }
 };
 
@@ -115,65 +118,118 @@ __device__ __forceinline__ void codes_of(const uint32_t (&p)[4], int U, uint32_t
     }
 }
 
-// F of byte k of a code word (he = kHalfExp)
-__device__ __forceinline__ float f_of(uint32_t x, uint32_t he, uint32_t k) {
-    return __uint_as_float(__byte_perm(x, he, 0x7044u | (k << 8)));
+// F of byte k of a code word
+__device__ __forceinline__ float f_of(uint32_t x, uint32_t k) {
+    return __uint_as_float(__byte_perm(x, kHalfExp, 0x7044u | (k << 8)));
 }
 
-// G consecutive floats of shared memory (16-byte aligned when G >= 4)
-template <int G>
-__device__ __forceinline__ void load_g(const float* p, float (&v)[G]) {
-    if constexpr (G % 4 == 0) {
-#pragma unroll
-        for (int i = 0; i < G; i += 4) {
-            const float4 t = *reinterpret_cast<const float4*>(p + i);
-            v[i] = t.x; v[i + 1] = t.y; v[i + 2] = t.z; v[i + 3] = t.w;
+// acc += w * f on both halves (one paired instruction: two correctly rounded FMAs)
+__device__ __forceinline__ void ffma2(float2& acc, const float2& w, const float2& f) { acc = __ffma2_rn(w, f, acc); }
+
+// Code words of (slot, block): 64 bytes, four 16-byte pieces; piece v sits at
+// position v ^ swz(block), so that the 32 stores of a warp staging 32 blocks
+// and the loads of a warp computing 8 blocks both hit every bank once.
+__device__ __forceinline__ int swz(int block) { return (block >> 1) & 3; }
+
+__device__ __forceinline__ uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// The items of one (head group, chunk): an item is a channel slot of the
+// chunk, a depth t and the set M of the group's heads that read the slot's
+// channel to exactly depth t (item bits 0..2: slot, 4..7: M, 8..15: the byte
+// mask of t planes).  Per item: the thread's 16 code bytes masked to depth t,
+// 16 byte permutes into F_t, and for each head of M one coefficient pair and
+// 8 paired FMAs.  Every lane reads the same item word; a warp reduction of it
+// gives the compiler a value it knows to be warp-uniform, so the per-head
+// tests are plain uniform branches.  The next item's code words are loaded
+// before the current item is computed.  acc[h][2w + r] holds keys (byte 2r,
+// byte 2r + 1) of code word w of the thread.
+template <int HG>
+__device__ __forceinline__ void chunk_items(const uint32_t* __restrict__ items, int nit,
+                                            const unsigned char* __restrict__ cth, const float* __restrict__ wth,
+                                            float2 (&acc)[HG][8]) {
+    constexpr int kSlotCode = kNB * 16 * 4;   // bytes of one slot's code words
+    constexpr int kSlotW = kNB * HG * 2;      // floats of one slot's coefficients
+    if (nit <= 0) return;
+    uint32_t dn = __reduce_or_sync(0xffffffffu, items[0]);
+    uint4 Xn = *reinterpret_cast<const uint4*>(cth + (dn & 7) * kSlotCode);
+#pragma unroll 1
+    for (int it = 0; it < nit; ++it) {
+        const uint32_t desc = dn;
+        uint4 X = Xn;
+        if (it + 1 < nit) {
+            dn = __reduce_or_sync(0xffffffffu, items[it + 1]);
+            Xn = *reinterpret_cast<const uint4*>(cth + (dn & 7) * kSlotCode);
         }
-    } else {
+        const uint32_t bm = __byte_perm(desc, 0u, 0x1111u);   // byte 1 in all four bytes
+        X.x &= bm;
+        X.y &= bm;
+        X.z &= bm;
+        X.w &= bm;
+        const uint32_t xs[4] = {X.x, X.y, X.z, X.w};
+        float2 F[8];
 #pragma unroll
-        for (int i = 0; i < G; ++i) v[i] = p[i];
+        for (int w = 0; w < 4; ++w) {
+            F[2 * w] = make_float2(f_of(xs[w], 0), f_of(xs[w], 1));
+            F[2 * w + 1] = make_float2(f_of(xs[w], 2), f_of(xs[w], 3));
+        }
+        const float* wa = wth + (desc & 7) * kSlotW;
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+            if (desc & (16u << h)) {
+                const float2 W = *reinterpret_cast<const float2*>(wa + 2 * h);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ffma2(acc[h][i], W, F[i]);
+            }
+        }
     }
 }
 
-// One (tile of 1024 keys, KV head g) of one store; q, depths and scores are
+// One (tile of kTile keys, KV head g) of one store; q, depths and scores are
 // the store's own [Hq][d], [Hq][d] and [Hq][n_pad_of(n)] arrays; n_pad is the
 // store's row stride (its capacity, >= n_pad_of(n)).
-template <int G>
+template <int G, bool HOST>
 __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ scales,
                                           int d, int64_t n, int64_t n_pad, int tile, int g,
                                           const void* __restrict__ q, int q_dtype,
                                           const uint8_t* __restrict__ depths, float* __restrict__ scores,
                                           uint32_t* __restrict__ bmax, unsigned int* status) {
     using Z = Geo<G>;
+    constexpr int HG = Z::HG, NHG = Z::NHG, T = Z::T;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const ScanSmem lay{d, G};
+    uint32_t* s_raw = reinterpret_cast<uint32_t*>(smem_raw + lay.raw());
+    uint16_t* s_rawsc = reinterpret_cast<uint16_t*>(smem_raw + lay.rawsc());
     uint32_t* s_codes = reinterpret_cast<uint32_t*>(smem_raw + lay.codes());
-    float* s_coef = reinterpret_cast<float*>(smem_raw + lay.coef());
-    const uint32_t** s_prow = reinterpret_cast<const uint32_t**>(smem_raw + lay.prow());
-    const uint16_t** s_srow = reinterpret_cast<const uint16_t**>(smem_raw + lay.srow());
-    uint32_t* s_items = reinterpret_cast<uint32_t*>(smem_raw + lay.items());
+    float* s_w2 = reinterpret_cast<float*>(smem_raw + lay.w2());
     float* s_q32 = reinterpret_cast<float*>(smem_raw + lay.q32());
     float* s_qk = reinterpret_cast<float*>(smem_raw + lay.qk());
-    int* s_off = reinterpret_cast<int*>(smem_raw + lay.off());
+    uint32_t* s_items = reinterpret_cast<uint32_t*>(smem_raw + lay.items());
     int* s_act = reinterpret_cast<int*>(smem_raw + lay.act());
+    uint8_t* s_nitems = smem_raw + lay.nitems();
     uint8_t* s_U = smem_raw + lay.uni();
     uint8_t* s_t = smem_raw + lay.tdep();
     __shared__ int s_L;
-    __shared__ uint32_t s_bmax[8 * kTileBlocks];   // per (head, block) max score as an ordered key; G <= 8
-    const int off_stride = d / 8 + 4;
 
-    const int64_t tile0 = (int64_t)tile * kTileKeys;
-    const int64_t words_total = n_pad / 32;
+    const int64_t tile0 = (int64_t)tile * kTile;
+    const int64_t words_total = n_pad / 32;   // plane row stride
     const int64_t nblk_total = n_pad / kBlock;
-    const int64_t wrem = words_total - tile0 / 32;
-    const int nwords = wrem < kTileWords ? (int)wrem : kTileWords;   // multiple of 4
-    const int nblocks = nwords / 2;
+    const int64_t len = n_pad_of(n);          // keys covered by tiles
+    const int keys_here = (int)(len - tile0 < kTile ? len - tile0 : kTile);   // a multiple of 1024
+    const int nw = keys_here / 32;
+    const int nblocks = keys_here / kBlock;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // ---- plan: depths, union list, row pointers, per-head item lists, per-(channel, head) factors ----
-    for (int e = tid; e < G * kTileBlocks; e += Z::T) s_bmax[e] = 0u;   // below every ordered key
-    for (int e = tid; e < G * d; e += Z::T) {
+    // ---- plan: depths, union list, per-(slot, head) factors, item runs ----
+    for (int e = tid; e < G * d; e += T) {
         int t = depths[(int64_t)g * G * d + e];
         if (t > 4) {
             atomicOr(status, (unsigned)FATHOM_DEV_BAD_DEPTH);
@@ -200,16 +256,9 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
         if (lane == 0) s_L = base;
     }
     __syncthreads();
-    const int L = s_L;
-    const int nchunks = (L + kChunk - 1) / kChunk;
-    for (int a = tid; a < nchunks * kChunk; a += Z::T) {   // slots past the list: nothing to read
-        const bool live = a < L;
-        const int64_t row = (int64_t)g * d + (live ? s_act[a] : 0);
-        s_prow[a] = planes + row * 4 * words_total + tile0 / 32;
-        s_srow[a] = scales + row * nblk_total + tile0 / kBlock;
-        if (!live) s_U[a] = 0;
-    }
-    for (int e = tid; e < L * G; e += Z::T) {
+    const int L = (int)__reduce_or_sync(0xffffffffu, (unsigned)s_L);   // warp-uniform to the compiler
+    const int nchunks = (L + kCH - 1) / kCH;
+    for (int e = tid; e < L * G; e += T) {
         const int a = e / G, hh = e - a * G;
         const int c = s_act[a];
         const int t = s_t[hh * d + c];
@@ -217,207 +266,216 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
         s_q32[e] = (t > 0) ? 32.0f * qv : 0.0f;
         s_qk[e] = (t > 0) ? qv * (__uint_as_float((uint32_t)(130 - t) << 23) - 24.0f) : 0.0f;
     }
-    for (int e = L * G + tid; e < nchunks * kChunk * G; e += Z::T) {   // the last chunk's unused slots
-        s_q32[e] = 0.0f;
-        s_qk[e] = 0.0f;
-    }
-    if (warp < G) {
-        // item list of head h = warp, chunk by chunk: channels read to the
-        // union depth, then channels read to fewer planes.  An item holds the
-        // word offset of the channel's codes in a chunk buffer (slot *
-        // kChanWords, bits 0..11) and, for a shallower read, the byte mask
-        // (bits 16..23)
-        const int h = warp;
-        uint32_t* items = s_items + h * d;
-        int* off = s_off + h * off_stride;
-        int base = 0;
-        for (int a0 = 0; a0 < L; a0 += 32) {
-            const int a = a0 + lane;
-            const int t = (a < L) ? (int)s_t[h * d + s_act[a]] : 0;
-            const int U = (a < L) ? (int)s_U[a] : 0;
-            const bool full = t > 0 && t == U, part = t > 0 && t < U;
-            const unsigned mf = __ballot_sync(0xffffffffu, full);
-            const unsigned mp = __ballot_sync(0xffffffffu, part);
-            const int nf0 = __popc(mf & 0xFFFFu), np0 = __popc(mp & 0xFFFFu);
-            const int nf1 = __popc(mf >> 16), np1 = __popc(mp >> 16);
-            const int start0 = base, start1 = base + nf0 + np0;
-            const bool upper = lane >= 16;
-            const unsigned below = ((1u << lane) - 1u) & (upper ? 0xFFFF0000u : 0x0000FFFFu);
-            const int cstart = upper ? start1 : start0, cnf = upper ? nf1 : nf0;
-            const uint32_t slot = (uint32_t)(a & 15) * kChanWords;
-            if (full) items[cstart + __popc(mf & below)] = slot;
-            if (part) items[cstart + cnf + __popc(mp & below)] = slot | (((0x780u >> t) & 0x78u) << 16);
-            if (lane == 0) {
-                const int ch = a0 / 16;
-                off[2 * ch] = start0;
-                off[2 * ch + 1] = start0 + nf0;
-                off[2 * ch + 2] = start1;
-                off[2 * ch + 3] = start1 + nf1;
-            }
-            base = start1 + nf1 + np1;
+    // items of (head group, chunk): lane (slot, depth) -> an item when some head
+    // of the group reads the slot's channel to exactly that depth; kept in
+    // lane order (slot, then depth)
+    for (int task = warp; task < NHG * nchunks; task += T / 32) {
+        const int hg = task % NHG, ch = task / NHG;
+        const int al = lane >> 2, tt = (lane & 3) + 1, a = ch * kCH + al;
+        uint32_t m = 0;
+        if (a < L) {
+            const int c = s_act[a];
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh) m |= (uint32_t)(s_t[(hg * HG + hh) * d + c] == tt) << hh;
         }
-        if (lane == 0) off[2 * nchunks] = base;
-    }
-    __syncthreads();
-
-    // ---- stage role: channels cg*CPT + i of a chunk at plane word w; scales (al, bb) ----
-    const int cg = warp, w = lane;
-    const bool wok = w < nwords;
-    const int bb = tid & 15;   // block of this thread's scales (the same for every u: T is a multiple of 16)
-    uint32_t pw[Z::CPT][4];
-    float pd[Z::DPT];
-    float cstp[G];
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh) cstp[hh] = 0.0f;
-
-    auto load_chunk = [&](int ch) {
-#pragma unroll
-        for (int i = 0; i < Z::CPT; ++i) {
-            const int a = ch * kChunk + cg * Z::CPT + i;   // warp-uniform
-            const int U = wok ? s_U[a] : 0;
-            const uint32_t* p = s_prow[a] + w;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) pw[i][j] = (j < U) ? __ldg(p + j * words_total) : 0u;
+        const unsigned v = __ballot_sync(0xffffffffu, m != 0);
+        if (m) {
+            const uint32_t bm = (0x780u >> tt) & 0x78u;   // the first tt of the code's bits 6..3
+            s_items[task * kMaxItems + __popc(v & ((1u << lane) - 1u))] = (uint32_t)al | (m << 4) | (bm << 8);
         }
+        if (lane == 0) s_nitems[task] = (uint8_t)__popc(v);
+    }
+
+    // ---- roles ----
+    const int hg = tid / Z::TPG, lt = tid % Z::TPG;
+    const int b = lt >> 2, p = lt & 3;   // compute / coefficient thread: block b, word pair p
+    float2 acc[HG][8];
 #pragma unroll
-        for (int u = 0; u < Z::DPT; ++u) {
-            const int a = ch * kChunk + ((tid + u * Z::T) >> 4);
-            pd[u] = (a < L && bb < nblocks) ? __half2float(__ushort_as_half(__ldg(s_srow[a] + bb))) : 0.0f;
+    for (int h = 0; h < HG; ++h)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[h][i] = make_float2(0.0f, 0.0f);
+    float cst_own = 0.0f;   // constant of (block b, head p of the group), summed over the slots in order
+    const unsigned char* cth = reinterpret_cast<const unsigned char*>(s_codes) + b * 64 + 16 * (p ^ swz(b));
+    const float* wth = s_w2 + ((size_t)hg * kCH * kNB + b) * HG * 2;
+
+    __syncthreads();   // plan complete
+
+    // The rows of chunk ch: 16-byte pieces e of its plane rows (slot al, plane
+    // j, piece) and scale rows; piece_src() gives a piece's source or null,
+    // piece_dst() its place in raw buffer buf.
+    constexpr int kRowPieces = kTW / 4;                  // 16-byte pieces of a tile's plane row
+    constexpr int kPlanePieces = kCH * 4 * kRowPieces;   // of a chunk's plane rows
+    constexpr int kScalePieces = kCH * (kNB / 8);        // of a chunk's scale rows
+    auto piece_src = [&](int ch, int e) -> const void* {
+        if (e < kPlanePieces) {
+            const int al = e / (4 * kRowPieces), j = (e / kRowPieces) & 3, piece = e % kRowPieces;
+            const int a = ch * kCH + al;
+            if (a < L && j < (int)s_U[a] && piece * 4 < nw)
+                return planes + ((int64_t)(g * d + s_act[a]) * 4 + j) * words_total + tile0 / 32 + piece * 4;
+            return nullptr;
+        }
+        const int es = e - kPlanePieces, al = es / (kNB / 8), piece = es % (kNB / 8);
+        const int a = ch * kCH + al;
+        if (a < L && piece * 8 < nblocks)
+            return scales + (int64_t)(g * d + s_act[a]) * nblk_total + tile0 / kBlock + piece * 8;
+        return nullptr;
+    };
+    auto piece_dst = [&](int buf, int e) -> void* {
+        if (e < kPlanePieces) return s_raw + (size_t)buf * kCH * 4 * kTW + (size_t)e * 4;   // [al][j][piece] in order
+        const int es = e - kPlanePieces;
+        return s_rawsc + (size_t)buf * kCH * kNB + (size_t)es * 8;
+    };
+    // device-resident store: cp.async, one chunk ahead
+    auto load_chunk = [&](int ch, int buf) {
+        for (int e = tid; e < kPlanePieces + kScalePieces; e += T) {
+            const void* src = piece_src(ch, e);
+            if (src) cp_async16(piece_dst(buf, e), src);
+        }
+        cp_async_commit();
+    };
+    // host-resident store: plain 16-byte loads into registers, one chunk ahead
+    // (over the host link each load of a warp is one run of whole lines;
+    // cp.async of page-locked memory carried 2.5x the bytes)
+    constexpr int kPF = (kPlanePieces + kScalePieces + T - 1) / T;
+    uint4 pf[HOST ? kPF : 1];
+    auto fetch_chunk = [&](int ch) {
+#pragma unroll
+        for (int i = 0; i < kPF; ++i) {
+            const int e = tid + i * T;
+            const void* src = (e < kPlanePieces + kScalePieces) ? piece_src(ch, e) : nullptr;
+            pf[i] = src ? ldg16(src) : make_uint4(0u, 0u, 0u, 0u);
         }
     };
-    auto store_chunk = [&](int ch, int buf) {
-        uint32_t* cbase = s_codes + (size_t)buf * kChunk * kChanWords + w;
+    auto put_chunk = [&](int ch, int buf) {
 #pragma unroll
-        for (int i = 0; i < Z::CPT; ++i) {
-            const int al = cg * Z::CPT + i, a = ch * kChunk + al;
-            const int U = s_U[a];   // warp-uniform; 0 past the list
-            uint32_t x[8];
-            codes_of(pw[i], U, x);
-#pragma unroll
-            for (int sv = 0; sv < 8; ++sv) cbase[al * kChanWords + sv * kTileWords] = x[sv];
-        }
-        float* cf = s_coef + (size_t)buf * G * kChunk * kTileBlocks;
-#pragma unroll
-        for (int u = 0; u < Z::DPT; ++u) {
-            const int al = (tid + u * Z::T) >> 4, a = ch * kChunk + al;   // a < d: nchunks * 16 <= d
-            float qv[G], kv[G];
-            load_g<G>(s_q32 + a * G, qv);   // zero past the union list
-            load_g<G>(s_qk + a * G, kv);
-#pragma unroll
-            for (int hh = 0; hh < G; ++hh) {
-                cf[(hh * kChunk + al) * kTileBlocks + bb] = qv[hh] * pd[u];
-                cstp[hh] = fmaf(kv[hh], pd[u], cstp[hh]);
-            }
-        }
-    };
-
-    // ---- compute role: head h; lane (block b, variant half) ----
-    const int h = warp / Z::S, sp = warp % Z::S;
-    const int b = lane & 15, sv0 = Z::NSV * (2 * sp + (lane >> 4));
-    // key of acc[i][wd][k]: 64 b + 32 wd + sv0 + i + 8 k
-    float acc[Z::NSV][2][4];
-#pragma unroll
-    for (int i = 0; i < Z::NSV; ++i)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[i][0][k] = acc[i][1][k] = 0.0f;
-    const uint32_t he = kHalfExp;
-    const uint32_t* cth = s_codes + sv0 * kTileWords + 2 * b;                  // + buffer + slot + i * 32
-    const float* cfth = s_coef + (size_t)h * kChunk * kTileBlocks + b;         // + buffer + slot * 16
-
-    auto item = [&](const uint32_t* cb, const float* cfb, uint32_t it, bool masked) {
-        const uint32_t slot = it & 0xFFFu;
-        const uint32_t* rp = cb + slot;
-        const float c = cfb[slot >> 4];                       // slot / kChanWords * kTileBlocks
-        const uint32_t mk = __byte_perm(it, 0u, 0x2222u);     // byte 2 in all four bytes
-#pragma unroll
-        for (int i = 0; i < Z::NSV; ++i) {
-            const uint2 X = *reinterpret_cast<const uint2*>(rp + i * kTileWords);
-            const uint32_t x0 = masked ? (X.x & mk) : X.x, x1 = masked ? (X.y & mk) : X.y;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                acc[i][0][k] = fmaf(c, f_of(x0, he, (uint32_t)k), acc[i][0][k]);
-                acc[i][1][k] = fmaf(c, f_of(x1, he, (uint32_t)k), acc[i][1][k]);
-            }
+        for (int i = 0; i < kPF; ++i) {
+            const int e = tid + i * T;
+            if (e < kPlanePieces + kScalePieces && piece_src(ch, e))
+                *reinterpret_cast<uint4*>(piece_dst(buf, e)) = pf[i];
         }
     };
 
     if (nchunks > 0) {
-        load_chunk(0);
-        store_chunk(0, 0);
+        if constexpr (HOST) {
+            fetch_chunk(0);
+            put_chunk(0, 0);
+        } else {
+            load_chunk(0, 0);
+        }
     }
-    __syncthreads();
-    const uint32_t* items = s_items + h * d;
-    const int* off = s_off + h * off_stride;
     for (int ch = 0; ch < nchunks; ++ch) {
         const int buf = ch & 1;
-        if (ch + 1 < nchunks) load_chunk(ch + 1);
-        const uint32_t* cb = cth + (size_t)buf * kChunk * kChanWords;
-        const float* cfb = cfth + (size_t)buf * G * kChunk * kTileBlocks;
-        const int f0 = off[2 * ch], p0 = off[2 * ch + 1], e0 = off[2 * ch + 2];
-        for (int k = f0; k < p0; ++k) item(cb, cfb, items[k], false);
-        for (int k = p0; k < e0; ++k) item(cb, cfb, items[k], true);
-        if (ch + 1 < nchunks) store_chunk(ch + 1, buf ^ 1);
-        __syncthreads();
+        if constexpr (HOST) {
+            if (ch + 1 < nchunks) fetch_chunk(ch + 1);   // in flight during this chunk's stage and compute
+        } else {
+            if (ch + 1 < nchunks) {
+                load_chunk(ch + 1, buf ^ 1);
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+        }
+        __syncthreads();   // chunk ch's rows are in; the previous chunk's compute is done
+
+        // stage: (slot, block) -> 16 code words
+        for (int u = tid; u < kCH * kNB; u += T) {
+            const int al = u / kNB, bb = u % kNB, a = ch * kCH + al;
+            const int U = (a < L) ? (int)s_U[a] : 0;   // warp-uniform: a warp stages one slot
+            if (U == 0 || bb >= nblocks) continue;
+            const uint32_t* r = s_raw + (size_t)(buf * kCH + al) * 4 * kTW + 2 * bb;
+            uint32_t p0[4], p1[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (j < U) {
+                    const uint2 v = *reinterpret_cast<const uint2*>(r + j * kTW);
+                    p0[j] = v.x;
+                    p1[j] = v.y;
+                } else {
+                    p0[j] = p1[j] = 0u;
+                }
+            }
+            uint32_t x0[8], x1[8];
+            codes_of(p0, U, x0);
+            codes_of(p1, U, x1);
+            uint4* dst = reinterpret_cast<uint4*>(s_codes + (size_t)(al * kNB + bb) * 16);
+            const int sw = swz(bb);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v ^ sw] = make_uint4(x0[2 * v], x1[2 * v], x0[2 * v + 1], x1[2 * v + 1]);
+        }
+        // coefficients: thread (b, p) those of head p of its group, block b, every slot
+        if (p < HG) {
+            const int hq = hg * HG + p;
+#pragma unroll 2
+            for (int al = 0; al < kCH; ++al) {
+                const int a = ch * kCH + al;
+                if (a >= L) break;
+                const float D = __half2float(__ushort_as_half(s_rawsc[(size_t)(buf * kCH + al) * kNB + b]));
+                const float w = s_q32[a * G + hq] * D;
+                *reinterpret_cast<float2*>(s_w2 + ((((size_t)hg * kCH + al) * kNB + b) * HG + p) * 2) =
+                    make_float2(w, w);
+                cst_own = fmaf(s_qk[a * G + hq], D, cst_own);
+            }
+        }
+        __syncthreads();   // codes and coefficients of chunk ch are ready
+
+        const int task = ch * NHG + hg;
+        chunk_items<HG>(s_items + task * kMaxItems, (int)__reduce_or_sync(0xffffffffu, s_nitems[task]), cth, wth,
+                        acc);
+        if constexpr (HOST) {
+            // raw buffer buf ^ 1 was last read by chunk ch - 1's stage, before this chunk's first barrier
+            if (ch + 1 < nchunks) put_chunk(ch + 1, buf ^ 1);
+        }
     }
 
-    // ---- constants: the per-thread partials of each (block, head), summed in a fixed order ----
-    float* s_cred = reinterpret_cast<float*>(smem_raw + lay.codes());   // [NW][16][G]; the codes are dead now
-    float* s_cst = s_cred + Z::NW * 16 * G;                              // [G][16]
+    // ---- epilogue: the block's constants (head h's is held by thread p = h of
+    // the block), scores, and the maximum of every 64-key block for the top-k ----
+    float cst[HG];
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-        const float v = cstp[hh] + __shfl_xor_sync(0xffffffffu, cstp[hh], 16);
-        if (lane < 16) s_cred[(warp * 16 + lane) * G + hh] = v;
-    }
-    __syncthreads();
-    if (tid < 16 * G) {
-        const int hh = tid >> 4, b16 = tid & 15;
-        float v = 0.0f;
-        for (int wv = 0; wv < Z::NW; ++wv) v += s_cred[(wv * 16 + b16) * G + hh];
-        s_cst[hh * 16 + b16] = v;
-    }
-    __syncthreads();
-
-    // ---- epilogue ----
-    if (b < nblocks) {
-        const int64_t k0 = tile0 + 64 * b + sv0;   // key of acc[0][0][0]
-        float* out = scores + ((int64_t)g * G + h) * n_pad_of(n) + k0;
-        const float cst = s_cst[h * 16 + b];
-        const bool whole = tile0 + kTileKeys <= n;
-        uint32_t kmax = 0u;
+    for (int h = 0; h < HG; ++h) cst[h] = __shfl_sync(0xffffffffu, cst_own, (lane & ~3) | h);
+    if (b < nblocks) {   // uniform per warp: a warp covers 8 blocks and nblocks is a multiple of 16
+        const int64_t ld = len;
+        const int64_t kb = tile0 + 64 * b + 2 * p;   // key of (word 2p, half 0, byte 0)
+        const bool whole = tile0 + keys_here <= n;
 #pragma unroll
-        for (int i = 0; i < Z::NSV; ++i)
+        for (int h = 0; h < HG; ++h) {
+            const int hq = g * G + hg * HG + h;
+            float* out = scores + (int64_t)hq * ld + kb;
+            uint32_t kmax = 0u;
 #pragma unroll
             for (int wd = 0; wd < 2; ++wd)
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const int o = 32 * wd + i + 8 * k;
-                    const float v = (whole || k0 + o < n) ? acc[i][wd][k] + cst : -INFINITY;
-                    out[o] = v;
-                    kmax = max(kmax, float_to_ordered(v));
+                    const float2 a0 = acc[h][2 * wd + (k >> 1)];       // word 2p: keys kb + 32 wd + 8k
+                    const float2 a1 = acc[h][2 * (2 + wd) + (k >> 1)]; // word 2p + 1: one key later
+                    const int o = 32 * wd + 8 * k;
+                    float v0 = ((k & 1) ? a0.y : a0.x) + cst[h];
+                    float v1 = ((k & 1) ? a1.y : a1.x) + cst[h];
+                    if (!whole) {
+                        if (kb + o >= n) v0 = -INFINITY;
+                        if (kb + o + 1 >= n) v1 = -INFINITY;
+                    }
+                    *reinterpret_cast<float2*>(out + o) = make_float2(v0, v1);
+                    kmax = max(kmax, max(float_to_ordered(v0), float_to_ordered(v1)));
                 }
-        atomicMax(&s_bmax[h * kTileBlocks + b], kmax);
-    }
-    // the maximum of every 64-key block, for the top-k that reads only the
-    // blocks that can hold a selected key
-    __syncthreads();
-    if (bmax && tid < G * kTileBlocks) {
-        const int hh = tid / kTileBlocks, bb = tid % kTileBlocks;
-        bmax[((int64_t)g * G + hh) * (n_pad_of(n) / kBlock) + tile0 / kBlock + bb] = s_bmax[tid];
+            kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, 1));
+            kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, 2));
+            if (bmax && p == 0) bmax[(int64_t)hq * (ld / kBlock) + tile0 / kBlock + b] = kmax;
+        }
     }
 }
 
-template <int G>
-__global__ void __launch_bounds__(Geo<G>::T, Geo<G>::MinBlocks)
+template <int G, bool HOST>
+__global__ void __launch_bounds__(Geo<G>::T, Geo<G>::template min_blocks<HOST>())
 scan_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ scales, int d, int64_t n,
             int64_t n_pad, const void* __restrict__ q, int q_dtype, const uint8_t* __restrict__ depths,
             float* __restrict__ scores, uint32_t* __restrict__ bmax, unsigned int* status) {
-    scan_tile<G>(planes, scales, d, n, n_pad, (int)blockIdx.x, (int)blockIdx.y, q, q_dtype, depths, scores, bmax,
-                 status);
+    scan_tile<G, HOST>(planes, scales, d, n, n_pad, (int)blockIdx.x, (int)blockIdx.y, q, q_dtype, depths, scores,
+                       bmax, status);
 }
 
 // Batched sessions: blockIdx.x runs over the tiles of all sessions.
-template <int G>
-__global__ void __launch_bounds__(Geo<G>::T, Geo<G>::MinBlocks)
+template <int G, bool HOST>
+__global__ void __launch_bounds__(Geo<G>::T, Geo<G>::template min_blocks<HOST>())
 scan_batched_kernel(const __grid_constant__ SessionMap map, int d, int Hq, const void* __restrict__ q, int q_dtype,
                     const uint8_t* __restrict__ depths, float* __restrict__ scores, uint32_t* __restrict__ bmax,
                     unsigned int* status) {
@@ -433,35 +491,50 @@ scan_batched_kernel(const __grid_constant__ SessionMap map, int d, int Hq, const
     const void* qs = (q_dtype == FATHOM_BF16)
                          ? static_cast<const void*>(static_cast<const uint16_t*>(q) + sidx * qstride)
                          : static_cast<const void*>(static_cast<const float*>(q) + sidx * qstride);
-    scan_tile<G>(map.planes[sidx], map.scales[sidx], d, map.n[sidx], map.n_pad[sidx], t - map.tile0[sidx],
-                 (int)blockIdx.y, qs, q_dtype, depths + sidx * qstride, scores + map.score_base[sidx],
-                 bmax ? bmax + map.score_base[sidx] / kBlock : nullptr, status);
+    scan_tile<G, HOST>(map.planes[sidx], map.scales[sidx], d, map.n[sidx], map.n_pad[sidx], t - map.tile0[sidx],
+                       (int)blockIdx.y, qs, q_dtype, depths + sidx * qstride, scores + map.score_base[sidx],
+                       bmax ? bmax + map.score_base[sidx] / kBlock : nullptr, status);
 }
 
-template <int G>
+template <int G, bool HOST>
 cudaError_t launch_scan_g(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n,
                           int64_t n_pad, const void* q, int q_dtype, const uint8_t* depths, float* scores,
                           uint32_t* bmax, cudaStream_t stream) {
     const size_t smem = ScanSmem{d, G}.bytes();
-    auto kern = scan_kernel<G>;
+    auto kern = scan_kernel<G, HOST>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)(n_pad_of(n) / kTileKeys), (unsigned)Hkv);   // the tiles holding keys; n_pad is the stride
+    dim3 grid((unsigned)scan_tiles(n), (unsigned)Hkv);   // the tiles holding keys; n_pad is the stride
     kern<<<grid, Geo<G>::T, smem, stream>>>(planes, scales, d, n, n_pad, q, q_dtype, depths, scores, bmax,
                                             device_status_ptr());
     return cudaGetLastError();
 }
 
-template <int G>
+template <int G, bool HOST>
 cudaError_t launch_scan_batched_g(const SessionMap& map, int Hkv, int d, const void* q, int q_dtype,
                                   const uint8_t* depths, int Hq, float* scores, uint32_t* bmax, cudaStream_t stream) {
     const size_t smem = ScanSmem{d, G}.bytes();
-    auto kern = scan_batched_kernel<G>;
+    auto kern = scan_batched_kernel<G, HOST>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)map.tile0[map.nsess], (unsigned)Hkv);
     kern<<<grid, Geo<G>::T, smem, stream>>>(map, d, Hq, q, q_dtype, depths, scores, bmax, device_status_ptr());
     return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t launch_scan_r(bool host, const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n,
+                          int64_t n_pad, const void* q, int q_dtype, const uint8_t* depths, float* scores,
+                          uint32_t* bmax, cudaStream_t stream) {
+    return host ? launch_scan_g<G, true>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream)
+                : launch_scan_g<G, false>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
+}
+
+template <int G>
+cudaError_t launch_scan_batched_r(bool host, const SessionMap& map, int Hkv, int d, const void* q, int q_dtype,
+                                  const uint8_t* depths, int Hq, float* scores, uint32_t* bmax, cudaStream_t stream) {
+    return host ? launch_scan_batched_g<G, true>(map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream)
+                : launch_scan_batched_g<G, false>(map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream);
 }
 
 }  // namespace
@@ -470,23 +543,24 @@ size_t scan_smem_bytes(int d, int G) { return ScanSmem{d, G}.bytes(); }
 
 cudaError_t launch_scan(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n, int64_t n_pad,
                         const void* q, int q_dtype, const uint8_t* depths, int Hq, float* scores,
-                        cudaStream_t stream, uint32_t* bmax) {
+                        cudaStream_t stream, uint32_t* bmax, bool host) {
     switch (Hq / Hkv) {
-        case 1: return launch_scan_g<1>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
-        case 2: return launch_scan_g<2>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
-        case 4: return launch_scan_g<4>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
-        case 8: return launch_scan_g<8>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
+        case 1: return launch_scan_r<1>(host, planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
+        case 2: return launch_scan_r<2>(host, planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
+        case 4: return launch_scan_r<4>(host, planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
+        case 8: return launch_scan_r<8>(host, planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_scan_batched(const SessionMap& map, int Hkv, int d, const void* q, int q_dtype,
-                                const uint8_t* depths, int Hq, float* scores, cudaStream_t stream, uint32_t* bmax) {
+                                const uint8_t* depths, int Hq, float* scores, cudaStream_t stream, uint32_t* bmax,
+                                bool host) {
     switch (Hq / Hkv) {
-        case 1: return launch_scan_batched_g<1>(map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream);
-        case 2: return launch_scan_batched_g<2>(map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream);
-        case 4: return launch_scan_batched_g<4>(map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream);
-        case 8: return launch_scan_batched_g<8>(map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream);
+        case 1: return launch_scan_batched_r<1>(host, map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream);
+        case 2: return launch_scan_batched_r<2>(host, map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream);
+        case 4: return launch_scan_batched_r<4>(host, map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream);
+        case 8: return launch_scan_batched_r<8>(host, map, Hkv, d, q, q_dtype, depths, Hq, scores, bmax, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -19,8 +19,18 @@
  *   host-link runs (Sec 3.6).
  *
  * Conventions for every entry point:
- *   - The caller owns all memory; no call allocates.  The library's only
- *     state is one status word per device (see below).
+ *   - The caller owns all memory it passes; no call allocates device
+ *     memory for it.  The library keeps this state of its own, per device:
+ *       . one status word (see below), a __device__ variable;
+ *       . for fathom_decode_step, one auxiliary stream and 65 events, made on
+ *         the first call in a context;
+ *       . for fathom_scan_topk_noalloc, a fixed scratch array of
+ *         fathom_noalloc_scratch_bytes(), a __device__ variable that every GPU
+ *         which loads the library holds until the process exits.
+ *     The host-side handles and the device addresses of these variables are
+ *     cached with the id of the CUDA context they belong to, and made or
+ *     looked up again when a call runs in another context (e.g. after
+ *     cudaDeviceReset).
  *   - Device pointers must be cudaMalloc'd (or equivalent) on the current
  *     device.  "Host-resident" pointers must be page-locked host memory
  *     (cudaHostAlloc / cudaHostRegister), mapped into the device address space
@@ -82,6 +92,9 @@ enum {
  *           bytes.
  *   scales  u16 [Hkv][d][n_pad/64]: fp16 bit pattern of the block scale Delta
  *           of (KV head, channel, 64-token block); 0 for all-padding blocks.
+ *   Both arrays start on a 16-byte boundary (the scan copies their rows to
+ *           shared memory in 16-byte pieces); a store that violates this is
+ *           rejected with FATHOM_EINVAL.
  *   host_resident: 0 = both arrays in device memory, 1 = both in page-locked
  *           host memory (the scan then streams only the budgeted planes over
  *           the host link).

@@ -24,7 +24,7 @@
  * channel importance w = fl32(fl32(q*q) * sigma2).  Build with
  * -ffp-contract=off so that no fused multiply-add changes those roundings.
  *
- * Readings taken where the pages are silent (each listed in the design doc):
+ * Readings taken where the pages are silent (the same readings as the CUDA path):
  *   - mid-rise code: Delta = fp16_rn(amax/8), u = floor(x/Delta),
  *     code = clamp(u,-8,7)+8, offset binary, plane 0 = most significant bit;
  *   - basis rule: a t-plane prefix is rebuilt with the signed plane basis

@@ -164,3 +164,52 @@ def test_config5_decode_step_sampled_layers(ref):
         del inp, st, Kr, Vr
         torch.cuda.empty_cache()
     assert F.last_device_status() == 0
+
+
+def test_config3_decode_step_as_benchmarked(ref):
+    """The call bench.py times, at its size: one fathom_decode_step on the n = 2^20 layer with the planes, the
+    scales and the interleaved K|V rows in page-locked host memory, B = 92, k = 2048, one KV-head group (the
+    top-k takes its block-maxima path: 16384 blocks >= 8k).  Depths bit-exact; sampled scores of every KV head
+    against fp64; the complete top-k property of all 32 heads on the scan's own scores; every needle found;
+    exact attention of heads in four KV groups against fp64; the one-call step equal to the separate calls."""
+    n, k, B = 1 << 20, 2048, 92
+    inp = synth.layer_inputs_cuda(3, n=n, device=DEV, with_values=True)
+    q = inp["q_dev"]
+    st = F.pack_bitplanes(inp["K"]).to_host()
+    Kr, Vr = F.kv_rows(8, n, 128, pin_memory=True)
+    Kr.copy_(inp["K_rows"])
+    Vr.copy_(inp["V_rows"])
+    dep, idx, top, out = F.decode_step(st, q, inp["sigma2_dev"], B, k, Kr, Vr, kv_groups=1)
+    torch.cuda.synchronize()
+    dep_h = dep.cpu().numpy()
+    assert np.array_equal(dep_h, ref.alloc_depths(inp["q"], inp["sigma2"], B))
+
+    # the same step as separate calls: bit for bit
+    bmax = F.block_max_buffer(32, n, DEV)
+    scores = F.scan_scores(st, q, dep, block_max=bmax)
+    idx2, top2 = F.scan_topk(st, q, dep, k)
+    out2 = F.sparse_attend(q, Kr, Vr, idx2)
+    assert torch.equal(idx, idx2)
+    assert torch.equal(top.view(torch.int32), top2.view(torch.int32))
+    assert torch.equal(out.view(torch.int32), out2.view(torch.int32))
+
+    scores_h = scores.cpu().numpy()[:, :n]
+    check_windows(ref, inp["K"], inp["q"], dep_h, scores_h, n, np.random.default_rng(33), count=1,
+                  kv_heads=list(range(8)))
+    idx_h = idx.cpu().numpy()
+    for h in range(32):
+        check_topk_property(scores_h[h], idx_h[h], k)
+    assert set(inp["needles"].tolist()) <= set(idx_h[0].tolist())
+
+    o = out.cpu().numpy()
+    for h in (0, 9, 18, 27):
+        g = h // 4
+        rows = np.sort(idx_h[h])
+        sel = torch.from_numpy(rows).to(DEV)
+        Kh = inp["K_rows"][g, sel].cpu().view(torch.int16).numpy().view(np.uint16)
+        Vh = inp["V_rows"][g, sel].cpu().view(torch.int16).numpy().view(np.uint16)
+        pos = {int(r): j for j, r in enumerate(rows)}
+        local = np.array([[pos[int(r)] for r in idx_h[h]]], np.int32)
+        o_ref = ref.attend(inp["q"][h:h + 1], Kh[None], Vh[None], local)[0]
+        assert np.linalg.norm(o[h] - o_ref) <= 1e-3 * np.linalg.norm(o_ref), h
+    assert F.last_device_status() == 0

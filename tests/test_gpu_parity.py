@@ -172,7 +172,8 @@ def test_pooled_depths_bit_exact(ref, G):
 # --------------------------------------------------------------------------
 # a4: scan scores within tolerance (+ the basis rule at every depth)
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("case", ["config1", "gqa_ragged", "d256_g2", "g8", "depth_mix"])
+@pytest.mark.parametrize("case", ["config1", "gqa_ragged", "d256_g2", "g8", "depth_mix", "depth_mix_g8",
+                                  "depth_mix_g2_tail", "depth_mix_g1"])
 def test_scan_scores(ref, case):
     if case == "config1":
         inp = make(1)                                       # Hkv=1, n=4096, d=128, f32 q
@@ -186,8 +187,17 @@ def test_scan_scores(ref, case):
     elif case == "g8":
         inp = make(2, n=1100, Hkv=1, Hq=8, d=64)
         B = 46
-    else:
+    elif case == "depth_mix":
         inp = make(1, n=2100, Hkv=1, Hq=4, d=128)
+        B = None
+    elif case == "depth_mix_g8":                            # two head groups of 4 per KV head
+        inp = make(2, n=7000, Hkv=2, Hq=16, d=96)
+        B = None
+    elif case == "depth_mix_g2_tail":                       # several full tiles and a half tile
+        inp = make(2, n=9217, Hkv=3, Hq=6, d=64)
+        B = None
+    else:
+        inp = make(1, n=4100, Hkv=2, Hq=2, d=256)
         B = None
     K, q = inp["K"], inp["q"]
     n = K.shape[1]
