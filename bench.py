@@ -56,6 +56,11 @@ def parse():
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     p.add_argument("--config", type=int, default=None, choices=[1, 2, 4, 5],
                    help="measure another workload of the method (one JSON line per case; not the headline)")
+    p.add_argument("--shard-keys", action="store_true",
+                   help="key-range sharding (under torchrun): every rank holds --n keys of one context of N x --n "
+                        "keys; local scan + top-k, all-gather, merge, attention partials, all-gather, merge")
+    p.add_argument("--matched", action="store_true",
+                   help="matched-GPU-time comparison against the fixed 68-bit read on the n=2^20 host-resident layer")
     p.add_argument("--fidelity", type=int, default=None, choices=[2, 3],
                    help="fidelity of the sparse step against exact dense attention on config 2 or 3 (a measurement "
                         "harness: attention error, recall of the exact top-k, needle recall, bytes per key)")
@@ -544,6 +549,114 @@ def _graph_of(torch, fn, warmup=3):
     return g
 
 
+def config12_cases(F, torch, dev, config, steps, warmup, flush, with_oracle=True):
+    """Configs 1 and 2 (HBM-resident): one record per budget case (config 2
+    adds fixed68 / fixed136), each timed through the one-call decode step: L2
+    flushed, warm, and replayed from a CUDA graph; the scan alone; and (with
+    with_oracle) the oracle on one KV group over all keys, single thread."""
+    import synth
+    import oracle
+    cfg = synth.CONFIGS[config]
+    inp = synth.layer_inputs_cuda(config, device=dev)
+    Hkv, Hq, n, k = cfg["n_kv_heads"], cfg["n_q_heads"], cfg["n"], cfg["k"]
+    st = F.pack_bitplanes(inp["K"])
+    Kr, Vr = inp["K_rows"], inp["V_rows"]
+    ws = torch.empty(F.decode_workspace_bytes(st, Hq, k, 1), dtype=torch.uint8, device=dev)
+    bufs = dict(depths=torch.empty((Hq, 128), dtype=torch.uint8, device=dev),
+                idx=torch.empty((Hq, k), dtype=torch.int32, device=dev),
+                top_scores=torch.empty((Hq, k), dtype=torch.float32, device=dev),
+                out=torch.empty((Hq, 128), dtype=torch.float32, device=dev), workspace=ws)
+    cases = [("B=%d" % b, b, 0) for b in cfg["budgets"]]
+    if config == 2:
+        cases += [("fixed68_r16", 0, 16), ("fixed136_r32", 0, 32)]
+    out = []
+    for name, b, fr in cases:
+        step = lambda: F.decode_step(st, inp["q_dev"], inp["sigma2_dev"], b, k, Kr, Vr, fixed_r=fr, **bufs)
+        t_flush = _events_ms(torch, step, steps, warmup, flush)
+        t_warm = _events_ms(torch, step, steps, warmup)
+        graph = _graph_of(torch, step)   # the same call replayed from a CUDA graph: no host launch cost
+        t_graph = _events_ms(torch, graph.replay, steps, warmup, flush)
+        del graph
+        dep = F.alloc_depths(inp["q_dev"], inp["sigma2_dev"], b, fixed_r=fr)
+        scan = _events_ms(torch, lambda: F.scan_scores(st, inp["q_dev"], dep), steps, warmup, flush)
+        U = dep.view(Hkv, Hq // Hkv, 128).amax(dim=1)
+        nbytes = st.plane_bytes_read(U)
+        rec = {"config": config, "case": name, "workload": cfg["name"], "n": n, "n_kv_heads": Hkv,
+               "n_q_heads": Hq, "k": k, "step_us_l2_flushed": float(np.median(t_flush)) * 1e3,
+               "step_us_warm": float(np.median(t_warm)) * 1e3,
+               "step_us_cuda_graph_l2_flushed": float(np.median(t_graph)) * 1e3,
+               "scan_us": float(np.median(scan)) * 1e3,
+               "gkeys_per_s_step": n * Hkv / (float(np.median(t_flush)) * 1e-3) / 1e9,
+               "scan_bytes_per_key_per_kv_head": nbytes / (n * Hkv),
+               "scan_hbm_gbs": nbytes / (float(np.median(scan)) * 1e-3) / 1e9}
+        if with_oracle:   # the oracle on one KV group over all n keys (single thread)
+            G = Hq // Hkv
+            planes = st.planes[0:1].cpu().numpy().view(np.uint32)
+            scales = st.scales[0:1].cpu().numpy().view(np.uint16)
+            Krg = Kr[0:1].cpu().view(torch.int16).numpy().view(np.uint16)
+            Vrg = Vr[0:1].cpu().view(torch.int16).numpy().view(np.uint16)
+            t0 = time.perf_counter()
+            oracle.decode(planes, scales, n, inp["q"][:G], inp["sigma2"][0:1], b, k, K_rows=Krg, V_rows=Vrg,
+                          fixed_r=fr)
+            t_or = time.perf_counter() - t0
+            rec.update({"oracle_s_one_kv_group": t_or, "oracle_cores": 1,
+                        "gpu_vs_oracle_per_kv_group": t_or / (float(np.median(t_flush)) * 1e-3 / Hkv)})
+        out.append(rec)
+    return out
+
+
+def config4_step(F, torch, dev, steps, warmup, flush, with_oracle=True):
+    """Config 4: 16 decode sessions of seeded lengths in [64k, 512k] keys,
+    host-resident stores, B = 68, k = 1024: depths, then one batched scan +
+    top-k call per step (CUDA events, L2 flushed)."""
+    import synth
+    import oracle
+    cfg = synth.CONFIGS[4]
+    rng = synth.rng_for(4, 0, 9)
+    lengths = (rng.integers(cfg["n_lo"] // 64, cfg["n_hi"] // 64 + 1, cfg["sessions"]) * 64).tolist()
+    stores, qs, s2s = [], [], []
+    for sidx, n in enumerate(lengths):
+        inp = synth.layer_inputs_cuda(4, layer=sidx, n=n, device=dev, with_values=False)
+        stores.append(F.pack_bitplanes(inp["K"]).to_host())
+        qs.append(inp["q_dev"])
+        s2s.append(inp["sigma2_dev"])
+        del inp
+        torch.cuda.empty_cache()
+    q = torch.stack(qs)
+    s2 = torch.cat(s2s)
+    S, Hq, k, B = len(lengths), 32, cfg["k"], cfg["budgets"][0]
+    dep = torch.empty((S * Hq, 128), dtype=torch.uint8, device=dev)
+    ws = torch.empty(F.scan_batched_workspace_bytes(stores, Hq, k), dtype=torch.uint8, device=dev)
+    idx = torch.empty((S, Hq, k), dtype=torch.int32, device=dev)
+    top = torch.empty((S, Hq, k), dtype=torch.float32, device=dev)
+
+    def step():
+        F.alloc_depths(q.view(-1, 128), s2, B, out=dep)
+        F.scan_topk_batched(stores, q, dep.view(S, Hq, 128), k, idx=idx, top_scores=top, workspace=ws)
+    t = _events_ms(torch, step, steps, warmup, flush)
+    keys = sum(lengths) * 8
+    nbytes = 0
+    for sidx, st in enumerate(stores):
+        U = dep.view(S, 8, 4, 128)[sidx].amax(dim=1)
+        nbytes += st.plane_bytes_read(U)
+    ms = float(np.median(t))
+    rec = {"config": 4, "case": "16 sessions batched", "workload": cfg["name"], "sessions": S,
+           "total_keys": sum(lengths), "step_ms": ms, "gkeys_per_s": keys / (ms * 1e-3) / 1e9,
+           "scan_bytes_per_key_per_kv_head": nbytes / keys, "link_gbs": nbytes / (ms * 1e-3) / 1e9,
+           "launches_per_step": 1 + 1 + topk_launches(min(lengths), k, max(lengths))}
+    if with_oracle:   # the oracle on session 0's first KV group (single thread), scaled to the step
+        st0 = stores[0]
+        t0 = time.perf_counter()
+        oracle.decode(st0.planes[0:1].cpu().numpy().view(np.uint32), st0.scales[0:1].cpu().numpy().view(np.uint16),
+                      lengths[0], qs[0][:4].float().cpu().numpy(), s2s[0][0:1].cpu().numpy(), B, k)
+        t_or = time.perf_counter() - t0
+        rec.update({"oracle_s_session0_kv_group0": t_or, "oracle_cores": 1,
+                    "oracle_s_step_extrapolated": t_or * keys / lengths[0]})
+    del stores, ws
+    torch.cuda.empty_cache()
+    return rec
+
+
 def config_bench(args):
     """The pages' other workloads, each timed through the one-call decode step
     or the batched entry point (one JSON line per case):
@@ -562,98 +675,9 @@ def config_bench(args):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     out = []
     if args.config in (1, 2):
-        cfg = synth.CONFIGS[args.config]
-        inp = synth.layer_inputs_cuda(args.config, device=dev)
-        Hkv, Hq, n, k = cfg["n_kv_heads"], cfg["n_q_heads"], cfg["n"], cfg["k"]
-        st = F.pack_bitplanes(inp["K"])
-        Kr, Vr = inp["K_rows"], inp["V_rows"]
-        ws = torch.empty(F.decode_workspace_bytes(st, Hq, k, 1), dtype=torch.uint8, device=dev)
-        bufs = dict(depths=torch.empty((Hq, 128), dtype=torch.uint8, device=dev),
-                    idx=torch.empty((Hq, k), dtype=torch.int32, device=dev),
-                    top_scores=torch.empty((Hq, k), dtype=torch.float32, device=dev),
-                    out=torch.empty((Hq, 128), dtype=torch.float32, device=dev), workspace=ws)
-        cases = [("B=%d" % b, b, 0) for b in cfg["budgets"]]
-        if args.config == 2:
-            cases += [("fixed68_r16", 0, 16), ("fixed136_r32", 0, 32)]
-        for name, b, fr in cases:
-            step = lambda: F.decode_step(st, inp["q_dev"], inp["sigma2_dev"], b, k, Kr, Vr, fixed_r=fr, **bufs)
-            t_flush = _events_ms(torch, step, args.steps, args.warmup, flush)
-            t_warm = _events_ms(torch, step, args.steps, args.warmup)
-            graph = _graph_of(torch, step)   # the same call replayed from a CUDA graph: no host launch cost
-            t_graph = _events_ms(torch, graph.replay, args.steps, args.warmup, flush)
-            del graph
-            dep = F.alloc_depths(inp["q_dev"], inp["sigma2_dev"], b, fixed_r=fr)
-            scan = _events_ms(torch, lambda: F.scan_scores(st, inp["q_dev"], dep), args.steps, args.warmup, flush)
-            U = dep.view(Hkv, Hq // Hkv, 128).amax(dim=1)
-            nbytes = st.plane_bytes_read(U)
-            # the oracle on one KV group over all n keys (single thread)
-            g0 = 0
-            planes = st.planes[g0:g0 + 1].cpu().numpy().view(np.uint32)
-            scales = st.scales[g0:g0 + 1].cpu().numpy().view(np.uint16)
-            G = Hq // Hkv
-            qg = inp["q"][:G]
-            s2g = inp["sigma2"][g0:g0 + 1]
-            Krg = Kr[g0:g0 + 1].cpu().view(torch.int16).numpy().view(np.uint16)
-            Vrg = Vr[g0:g0 + 1].cpu().view(torch.int16).numpy().view(np.uint16)
-            t0 = time.perf_counter()
-            if fr:
-                oracle.decode(planes, scales, n, qg, s2g, 0, k, K_rows=Krg, V_rows=Vrg, fixed_r=fr)
-            else:
-                oracle.decode(planes, scales, n, qg, s2g, b, k, K_rows=Krg, V_rows=Vrg)
-            t_or = time.perf_counter() - t0
-            out.append({"config": args.config, "case": name, "workload": cfg["name"], "n": n, "n_kv_heads": Hkv,
-                        "n_q_heads": Hq, "k": k, "step_us_l2_flushed": float(np.median(t_flush)) * 1e3,
-                        "step_us_warm": float(np.median(t_warm)) * 1e3,
-                        "step_us_cuda_graph_l2_flushed": float(np.median(t_graph)) * 1e3,
-                        "scan_us": float(np.median(scan)) * 1e3,
-                        "gkeys_per_s_step": n * Hkv / (float(np.median(t_flush)) * 1e-3) / 1e9,
-                        "scan_bytes_per_key_per_kv_head": nbytes / (n * Hkv),
-                        "scan_hbm_gbs": nbytes / (float(np.median(scan)) * 1e-3) / 1e9,
-                        "oracle_s_one_kv_group": t_or, "oracle_cores": 1,
-                        "gpu_vs_oracle_per_kv_group": t_or / (float(np.median(t_flush)) * 1e-3 / Hkv)})
+        out = config12_cases(F, torch, dev, args.config, args.steps, args.warmup, flush)
     elif args.config == 4:
-        cfg = synth.CONFIGS[4]
-        rng = synth.rng_for(4, 0, 9)
-        lengths = (rng.integers(cfg["n_lo"] // 64, cfg["n_hi"] // 64 + 1, cfg["sessions"]) * 64).tolist()
-        stores, qs, s2s = [], [], []
-        for sidx, n in enumerate(lengths):
-            inp = synth.layer_inputs_cuda(4, layer=sidx, n=n, device=dev, with_values=False)
-            stores.append(F.pack_bitplanes(inp["K"]).to_host())
-            qs.append(inp["q_dev"])
-            s2s.append(inp["sigma2_dev"])
-            del inp
-            torch.cuda.empty_cache()
-        q = torch.stack(qs)
-        s2 = torch.cat(s2s)
-        S, Hq, k, B = len(lengths), 32, cfg["k"], cfg["budgets"][0]
-        dep = torch.empty((S * Hq, 128), dtype=torch.uint8, device=dev)
-        ws = torch.empty(F.scan_batched_workspace_bytes(stores, Hq, k), dtype=torch.uint8, device=dev)
-        idx = torch.empty((S, Hq, k), dtype=torch.int32, device=dev)
-        top = torch.empty((S, Hq, k), dtype=torch.float32, device=dev)
-
-        def step():
-            F.alloc_depths(q.view(-1, 128), s2, B, out=dep)
-            F.scan_topk_batched(stores, q, dep.view(S, Hq, 128), k, idx=idx, top_scores=top, workspace=ws)
-        t = _events_ms(torch, step, args.steps, args.warmup, flush)
-        keys = sum(lengths) * 8
-        nbytes = 0
-        for sidx, st in enumerate(stores):
-            U = dep.view(S, 8, 4, 128)[sidx].amax(dim=1)
-            nbytes += st.plane_bytes_read(U)
-        ms = float(np.median(t))
-        # the oracle on session 0's first KV group (single thread), scaled to the
-        # step's keys x KV heads
-        st0 = stores[0]
-        t0 = time.perf_counter()
-        oracle.decode(st0.planes[0:1].cpu().numpy().view(np.uint32), st0.scales[0:1].cpu().numpy().view(np.uint16),
-                      lengths[0], qs[0][:4].float().cpu().numpy(), s2s[0][0:1].cpu().numpy(), B, k)
-        t_or = time.perf_counter() - t0
-        out.append({"config": 4, "case": "16 sessions batched", "workload": cfg["name"], "sessions": S,
-                    "total_keys": sum(lengths), "step_ms": ms, "gkeys_per_s": keys / (ms * 1e-3) / 1e9,
-                    "scan_bytes_per_key_per_kv_head": nbytes / keys, "link_gbs": nbytes / (ms * 1e-3) / 1e9,
-                    "launches_per_step": 1 + 1 + topk_launches(min(lengths), k, max(lengths)),
-                    "oracle_s_session0_kv_group0": t_or, "oracle_cores": 1,
-                    "oracle_s_step_extrapolated": t_or * keys / lengths[0]})
+        out = [config4_step(F, torch, dev, args.steps, args.warmup, flush)]
     elif args.config == 5:
         cfg = synth.CONFIGS[5]
         n, L = cfg["n"], cfg["layers"]
@@ -700,12 +724,50 @@ def config_bench(args):
         print(json.dumps(line), flush=True)
 
 
+def fidelity_refs(torch, q, Kr, Vr, k, G):
+    """References of the fidelity harness, per query head (plain fp32 torch on
+    the GPU; measurement only): exact dense attention over all n keys, the
+    exact top-k (the k largest q.k over the bf16 keys, torch.topk), the dense
+    softmax, and attention restricted to the exact top-k."""
+    Hq, d = q.shape
+    Hkv, n = Kr.shape[0], Kr.shape[1]
+    qf = q.float()
+    dense = torch.empty((Hq, d), dtype=torch.float32, device=q.device)
+    exact_idx = torch.empty((Hq, k), dtype=torch.int64, device=q.device)
+    probs = torch.empty((Hq, n), dtype=torch.float32, device=q.device)
+    for g in range(Hkv):
+        Kg = Kr[g].float()
+        s = qf[g * G:(g + 1) * G] @ Kg.T                       # [G][n]
+        exact_idx[g * G:(g + 1) * G] = torch.topk(s, k, dim=1).indices
+        p = torch.softmax(s / d ** 0.5, dim=1)
+        probs[g * G:(g + 1) * G] = p
+        dense[g * G:(g + 1) * G] = p @ Vr[g].float()
+        del Kg, s, p
+    return {"dense": dense, "exact_idx": exact_idx, "probs": probs,
+            "mass_exact": torch.gather(probs, 1, exact_idx).sum(1)}
+
+
+def fidelity_of(torch, refs, idx, out, exact_sparse=None):
+    """Per query head, numpy arrays: softmax mass of the selected keys, recall
+    of the exact top-k, relative L2 error of the attention output against dense
+    attention and (if given) against attention over the exact top-k."""
+    k = idx.shape[1]
+    mass = torch.gather(refs["probs"], 1, idx.long()).sum(1).cpu().numpy()
+    dense = refs["dense"]
+    err = ((out - dense).norm(dim=1) / dense.norm(dim=1)).cpu().numpy()
+    ih, eh = idx.cpu().numpy(), refs["exact_idx"].cpu().numpy()
+    rec = np.array([len(set(ih[h].tolist()) & set(eh[h].tolist())) / k for h in range(ih.shape[0])])
+    res = {"mass": mass, "recall": rec, "err_dense": err}
+    if exact_sparse is not None:
+        res["err_exact_topk"] = ((out - exact_sparse).norm(dim=1) / exact_sparse.norm(dim=1)).cpu().numpy()
+    return res
+
+
 def fidelity_bench(args):
     """Per read policy (B in {46, 68, 92, 136}, fixed68, fixed136, pooled B=92):
     the one-call decode step's attention output against exact dense attention
-    over all n keys (a plain fp32 torch reference, measurement only), the
-    recall of the exact top-k (top-k of q.k over the bf16 keys), the needles
-    found (config 3) and the plane + scale bytes the scan reads."""
+    over all n keys, the recall of the exact top-k, the needles found (config
+    3) and the plane + scale bytes the scan reads (fidelity_refs, fidelity_of)."""
     import torch
     import synth
     from bit_plane_key_b200 import fathom as F
@@ -719,22 +781,8 @@ def fidelity_bench(args):
     del inp["K"]
     Kr, Vr = inp["K_rows"], inp["V_rows"]
     q = inp["q_dev"]
-    qf = q.float()
-    # exact dense attention, the exact top-k and the dense softmax, per KV head
-    dense = torch.empty((Hq, d), dtype=torch.float32, device=dev)
-    exact_idx = torch.empty((Hq, k), dtype=torch.int64, device=dev)
-    probs = torch.empty((Hq, n), dtype=torch.float32, device=dev)
-    for g in range(Hkv):
-        Kg = Kr[g].float()
-        s = qf[g * G:(g + 1) * G] @ Kg.T                       # [G][n]
-        exact_idx[g * G:(g + 1) * G] = torch.topk(s, k, dim=1).indices
-        p = torch.softmax(s / d ** 0.5, dim=1)
-        probs[g * G:(g + 1) * G] = p
-        dense[g * G:(g + 1) * G] = p @ Vr[g].float()
-        del Kg, s, p
-    # attention restricted to the exact top-k: the best any k-row selection can do
-    exact_sparse = F.sparse_attend(q, Kr, Vr, exact_idx.to(torch.int32).contiguous())
-    mass_exact = torch.gather(probs, 1, exact_idx).sum(1)
+    refs = fidelity_refs(torch, q, Kr, Vr, k, G)
+    exact_sparse = F.sparse_attend(q, Kr, Vr, refs["exact_idx"].to(torch.int32).contiguous())
     needles = set(inp.get("needles", np.array([], np.int64)).tolist())
     policies = [("B=%d" % b, b, 0, False) for b in (46, 68, 92, 136)]
     policies += [("fixed68_r16", 0, 16, False), ("fixed136_r32", 0, 32, False), ("pooled_B92", 92, 0, True)]
@@ -747,30 +795,158 @@ def fidelity_bench(args):
             dep, idx, _, out = F.decode_step(st, q, inp["sigma2_dev"], b, k, Kr, Vr, fixed_r=fr)
         U = dep.view(Hkv, G, d).amax(dim=1)
         nbytes = st.plane_bytes_read(U)
-        err = ((out - dense).norm(dim=1) / dense.norm(dim=1)).cpu().numpy()
-        err_x = ((out - exact_sparse).norm(dim=1) / exact_sparse.norm(dim=1)).cpu().numpy()
-        mass = torch.gather(probs, 1, idx.long()).sum(1)
-        rec = []
-        for h in range(Hq):
-            a = set(idx[h].cpu().numpy().tolist())
-            e = set(exact_idx[h].cpu().numpy().tolist())
-            rec.append(len(a & e) / k)
+        m = fidelity_of(torch, refs, idx, out, exact_sparse)
         found = len(needles & set(idx[0].cpu().numpy().tolist())) / len(needles) if needles else None
         print(json.dumps({"fidelity": args.fidelity, "policy": name, "n": n, "k": k,
                           "scan_bytes_per_key_per_kv_head": nbytes / (n * Hkv),
-                          "softmax_mass_captured_mean": float(mass.mean()),
-                          "softmax_mass_exact_topk_mean": float(mass_exact.mean()),
-                          "attn_rel_err_vs_exact_topk_mean": float(err_x.mean()),
-                          "attn_rel_err_vs_exact_topk_max": float(err_x.max()),
-                          "attn_rel_err_vs_dense_mean": float(err.mean()),
-                          "exact_topk_recall_mean": float(np.mean(rec)), "exact_topk_recall_min": float(np.min(rec)),
+                          "softmax_mass_captured_mean": float(m["mass"].mean()),
+                          "softmax_mass_exact_topk_mean": float(refs["mass_exact"].mean()),
+                          "attn_rel_err_vs_exact_topk_mean": float(m["err_exact_topk"].mean()),
+                          "attn_rel_err_vs_exact_topk_max": float(m["err_exact_topk"].max()),
+                          "attn_rel_err_vs_dense_mean": float(m["err_dense"].mean()),
+                          "exact_topk_recall_mean": float(m["recall"].mean()),
+                          "exact_topk_recall_min": float(m["recall"].min()),
                           "needle_recall_head0": found}), flush=True)
+
+
+def shard_bench(args):
+    """One decode step of a context split by key range across the ranks (one
+    process per GPU): rank r holds keys [r n, (r + 1) n) of one layer (its own
+    keys, the layer's channel scales and queries; sigma2 averaged over the
+    ranks once, outside the timed steps, as the layer's statistic).  A step:
+    depths, the local scan + top-k, one all-gather of (score, global index) per
+    query head and the GPU merge (shard.sharded_scan_topk), then attention over
+    the selected rows each rank holds, one all-gather of the per-head partials
+    and their merge (shard.sharded_attend).  CUDA events on the launching
+    stream (NCCL's work is ordered before the stream's next use of its
+    output), max over ranks.  Whole-job Gkeys/s = world x n x Hkv / step."""
+    import torch
+    import synth
+    from bit_plane_key_b200 import fathom as F, shard
+    from bit_plane_key_b200.ranks import Ranks
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    ranks = Ranks("nccl", device=dev, sync=torch.cuda.synchronize, timeout_s=300)
+    world, rank = ranks.world, ranks.rank
+    n, k, B = args.n, args.k, args.budget
+    inp = synth.layer_inputs_cuda(3, n=n, device=dev, with_values=True, needles=0, part=rank)
+    st = F.pack_bitplanes(inp["K"])
+    torch.cuda.synchronize()
+    del inp["K"]
+    s2 = inp["sigma2_dev"].clone()
+    if ranks.dist:
+        ranks.dist.all_reduce(s2)
+        s2 /= world
+    if args.resident == "host":
+        st = st.to_host()
+        Kr, Vr = F.kv_rows(8, n, 128, pin_memory=True)
+        Kr.copy_(inp["K_rows"])
+        Vr.copy_(inp["V_rows"])
+    else:
+        Kr, Vr = inp["K_rows"], inp["V_rows"]
+    q = inp["q_dev"]
+    key0 = rank * n
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        dep = F.alloc_depths(q, s2, B)
+        idx, top = shard.sharded_scan_topk(st, key0, q, dep, k)
+        return shard.sharded_attend(q, Kr, Vr, key0, idx)
+
+    for _ in range(args.warmup):
+        step()
+    ranks.barrier()
+    ts = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ranks.barrier()
+    total = ranks.max(float(np.sum(ts)))
+    ms = total / args.steps
+    if rank == 0:
+        print(json.dumps({"metric": METRIC, "value": world * n * 8 / (ms * 1e-3) / 1e9, "unit": UNIT,
+                          "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                          "data": "synthetic (seeded generator, one key range per rank)",
+                          "config": {"workload": "one context of %d keys split by key range over %d ranks (%d keys "
+                                                 "each), 8 KV heads / 32 q heads, d=128, B=%d, k=%d, %s-resident"
+                                                 % (world * n, world, n, B, k, args.resident),
+                                     "mode": "key-range sharded: local scan + top-k, NCCL all-gather, merge; "
+                                             "attention partials, NCCL all-gather, merge",
+                                     "l2": "flushed between steps (256 MB write)"}}), flush=True)
+    ranks.close()
+
+
+def matched_bench(args):
+    """Matched-GPU-time comparison (the pages compare read policies at equal
+    GPU time against a fixed 68-bit read): on the n = 2^20 layer with the store
+    and the K/V rows in page-locked host memory, the one-call decode step is
+    timed for a sweep of budgets B and for fixed68 / fixed136 (CUDA events, L2
+    flushed); each policy's bytes per key and fidelity come from the same
+    call's outputs.  The B whose step time equals fixed68's is found by linear
+    interpolation between the two bracketing budgets, and its bytes per key,
+    attention error and recall are interpolated the same way."""
+    import torch
+    import synth
+    from bit_plane_key_b200 import fathom as F
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    args.n = synth.CONFIGS[3]["n"]
+    layer = Layer(F, torch, args, layer=0, resident="host", dev=dev)
+    Hkv, Hq, d, n, k = layer.Hkv, layer.Hq, layer.d, layer.n, args.k
+    G = Hq // Hkv
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    refs = fidelity_refs(torch, layer.q, layer.inp["K_rows"], layer.inp["V_rows"], k, G)
+    rows = []
+    budgets = (36, 40, 46, 52, 56, 60, 68, 80, 92)
+    for name, b, fr in [("B=%d" % b, b, 0) for b in budgets] + [("fixed68_r16", 0, 16), ("fixed136_r32", 0, 32)]:
+        t = timed_pipelined(torch, layer, b, args.steps, args.warmup, fr, flush, 1)["step_ms"]
+        nbytes, _ = layer.union_bytes()
+        m = fidelity_of(torch, refs, layer.idx, layer.out)
+        rows.append({"policy": name, "budget_bits": b, "fixed_r": fr, "step_ms": float(np.median(t)),
+                     "scan_bytes_per_key_per_kv_head": nbytes / (n * Hkv),
+                     "attn_rel_err_vs_dense_mean": float(m["err_dense"].mean()),
+                     "exact_topk_recall_mean": float(m["recall"].mean()),
+                     "softmax_mass_captured_mean": float(m["mass"].mean())})
+        print(json.dumps(dict(rows[-1], matched=False)), flush=True)
+    ref = next(r for r in rows if r["policy"] == "fixed68_r16")
+    sweep = [r for r in rows if r["fixed_r"] == 0]
+    out = {"matched": True, "against": "fixed68_r16", "fixed68_step_ms": ref["step_ms"],
+           "fixed68_bytes_per_key": ref["scan_bytes_per_key_per_kv_head"]}
+    for lo, hi in zip(sweep, sweep[1:]):
+        if lo["step_ms"] <= ref["step_ms"] <= hi["step_ms"] and hi["step_ms"] > lo["step_ms"]:
+            w = (ref["step_ms"] - lo["step_ms"]) / (hi["step_ms"] - lo["step_ms"])
+            lerp = lambda key: lo[key] + w * (hi[key] - lo[key])
+            out.update({"matched_budget_bits": lerp("budget_bits"),
+                        "bytes_per_key_at_matched_time": lerp("scan_bytes_per_key_per_kv_head"),
+                        "bytes_vs_fixed68": lerp("scan_bytes_per_key_per_kv_head")
+                                            / ref["scan_bytes_per_key_per_kv_head"],
+                        "attn_rel_err_vs_dense_at_matched_time": lerp("attn_rel_err_vs_dense_mean"),
+                        "fixed68_attn_rel_err_vs_dense": ref["attn_rel_err_vs_dense_mean"],
+                        "exact_topk_recall_at_matched_time": lerp("exact_topk_recall_mean"),
+                        "fixed68_exact_topk_recall": ref["exact_topk_recall_mean"]})
+            break
+    else:
+        out["note"] = "fixed68's step time lies outside the budget sweep"
+    print(json.dumps(out), flush=True)
 
 
 def main():
     args = parse()
     if args.fidelity:
         fidelity_bench(args)
+        return
+    if args.matched:
+        matched_bench(args)
+        return
+    if args.shard_keys:
+        shard_bench(args)
         return
     if args.config:
         config_bench(args)
@@ -892,6 +1068,10 @@ def main():
                 "ops_per_key_per_kv_head": ops / (args.n * layer.Hkv),
                 "peak_source": "%d SMs x 128 lanes x %.0f MHz (sampled)" % (sms, mhz)}
             layer.store, layer.K_rows, layer.V_rows = keep
+        # the pages' other workloads on the same kernels: config 2 (n = 131072,
+        # HBM, B sweep and fixed68/136) and one config-4 batched step
+        extras["config2"] = config12_cases(F, torch, dev, 2, args.steps, args.warmup, flush, with_oracle=False)
+        extras["config4"] = config4_step(F, torch, dev, args.steps, args.warmup, flush, with_oracle=False)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:

@@ -73,9 +73,10 @@ struct ScanSmem {
     __host__ __device__ size_t rawsc() const { return raw() + 2u * kCH * 4 * kTW * 4; }    // [2][kCH][kNB] u16
     __host__ __device__ size_t codes() const { return rawsc() + 2u * kCH * kNB * 2; }      // [kCH][kNB][8][2] u32
     __host__ __device__ size_t w2() const { return codes() + (size_t)kCH * kNB * 16 * 4; } // [nhg][kCH][kNB][hg][2] f32
-    __host__ __device__ size_t q32() const { return w2() + (size_t)nhg() * kCH * kNB * hg() * 8; }   // [d][G] f32
-    __host__ __device__ size_t qk() const { return q32() + (size_t)d * G * 4; }            // [d][G] f32
-    __host__ __device__ size_t items() const { return qk() + (size_t)d * G * 4; }          // [nhg*maxchunks][kMaxItems] u32
+    __host__ __device__ size_t qq() const { return w2() + (size_t)nhg() * kCH * kNB * hg() * 8; }   // [d][G] (32q, qk) f32x2
+    __host__ __device__ size_t prow() const { return qq() + (size_t)d * G * 8; }          // [d] plane-0 row of the tile
+    __host__ __device__ size_t srow() const { return prow() + (size_t)d * 8; }           // [d] scale row of the tile
+    __host__ __device__ size_t items() const { return srow() + (size_t)d * 8; }          // [nhg*maxchunks][kMaxItems] u32
     __host__ __device__ size_t act() const { return items() + (size_t)nhg() * maxchunks() * kMaxItems * 4; }   // [d] i32
     __host__ __device__ size_t nitems() const { return act() + (size_t)d * 4; }            // [nhg*maxchunks] u8
     __host__ __device__ size_t uni() const { return nitems() + (size_t)nhg() * maxchunks(); }   // [d] u8
@@ -141,16 +142,24 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+// The FMAs of one head h for an item: its coefficient pair, 8 paired FMAs.
+template <int HG>
+__device__ __forceinline__ void head_fma(int h, const float* wa, const float2 (&F)[8], float2 (&acc)[HG][8]) {
+    const float2 W = *reinterpret_cast<const float2*>(wa + 2 * h);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ffma2(acc[h][i], W, F[i]);
+}
+
 // The items of one (head group, chunk): an item is a channel slot of the
 // chunk, a depth t and the set M of the group's heads that read the slot's
 // channel to exactly depth t (item bits 0..2: slot, 4..7: M, 8..15: the byte
 // mask of t planes).  Per item: the thread's 16 code bytes masked to depth t,
 // 16 byte permutes into F_t, and for each head of M one coefficient pair and
-// 8 paired FMAs.  Every lane reads the same item word; a warp reduction of it
-// gives the compiler a value it knows to be warp-uniform, so the per-head
-// tests are plain uniform branches.  The next item's code words are loaded
-// before the current item is computed.  acc[h][2w + r] holds keys (byte 2r,
-// byte 2r + 1) of code word w of the thread.
+// 8 paired FMAs, reached by one jump on M.  Every lane reads the same item
+// word; a warp reduction of it gives the compiler a value it knows to be
+// warp-uniform, so the jump needs no divergence handling.  The next item's
+// code words are loaded before the current item is computed.  acc[h][2w + r]
+// holds keys (byte 2r, byte 2r + 1) of code word w of the thread.
 template <int HG>
 __device__ __forceinline__ void chunk_items(const uint32_t* __restrict__ items, int nit,
                                             const unsigned char* __restrict__ cth, const float* __restrict__ wth,
@@ -181,14 +190,37 @@ __device__ __forceinline__ void chunk_items(const uint32_t* __restrict__ items, 
             F[2 * w + 1] = make_float2(f_of(xs[w], 2), f_of(xs[w], 3));
         }
         const float* wa = wth + (desc & 7) * kSlotW;
-#pragma unroll
-        for (int h = 0; h < HG; ++h) {
-            if (desc & (16u << h)) {
-                const float2 W = *reinterpret_cast<const float2*>(wa + 2 * h);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) ffma2(acc[h][i], W, F[i]);
+#define FATHOM_HEAD_FMA(h) head_fma<HG>(h, wa, F, acc)
+        if constexpr (HG == 1) {
+            FATHOM_HEAD_FMA(0);
+        } else if constexpr (HG == 2) {
+            switch ((desc >> 4) & 3) {
+                case 1: FATHOM_HEAD_FMA(0); break;
+                case 2: FATHOM_HEAD_FMA(1); break;
+                case 3: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(1); break;
+                default: break;
+            }
+        } else {
+            switch ((desc >> 4) & 15) {
+                case 1: FATHOM_HEAD_FMA(0); break;
+                case 2: FATHOM_HEAD_FMA(1); break;
+                case 3: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(1); break;
+                case 4: FATHOM_HEAD_FMA(2); break;
+                case 5: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(2); break;
+                case 6: FATHOM_HEAD_FMA(1); FATHOM_HEAD_FMA(2); break;
+                case 7: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(1); FATHOM_HEAD_FMA(2); break;
+                case 8: FATHOM_HEAD_FMA(3); break;
+                case 9: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(3); break;
+                case 10: FATHOM_HEAD_FMA(1); FATHOM_HEAD_FMA(3); break;
+                case 11: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(1); FATHOM_HEAD_FMA(3); break;
+                case 12: FATHOM_HEAD_FMA(2); FATHOM_HEAD_FMA(3); break;
+                case 13: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(2); FATHOM_HEAD_FMA(3); break;
+                case 14: FATHOM_HEAD_FMA(1); FATHOM_HEAD_FMA(2); FATHOM_HEAD_FMA(3); break;
+                case 15: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(1); FATHOM_HEAD_FMA(2); FATHOM_HEAD_FMA(3); break;
+                default: break;
             }
         }
+#undef FATHOM_HEAD_FMA
     }
 }
 
@@ -209,8 +241,9 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
     uint16_t* s_rawsc = reinterpret_cast<uint16_t*>(smem_raw + lay.rawsc());
     uint32_t* s_codes = reinterpret_cast<uint32_t*>(smem_raw + lay.codes());
     float* s_w2 = reinterpret_cast<float*>(smem_raw + lay.w2());
-    float* s_q32 = reinterpret_cast<float*>(smem_raw + lay.q32());
-    float* s_qk = reinterpret_cast<float*>(smem_raw + lay.qk());
+    float2* s_qq = reinterpret_cast<float2*>(smem_raw + lay.qq());
+    const uint32_t** s_prow = reinterpret_cast<const uint32_t**>(smem_raw + lay.prow());
+    const uint16_t** s_srow = reinterpret_cast<const uint16_t**>(smem_raw + lay.srow());
     uint32_t* s_items = reinterpret_cast<uint32_t*>(smem_raw + lay.items());
     int* s_act = reinterpret_cast<int*>(smem_raw + lay.act());
     uint8_t* s_nitems = smem_raw + lay.nitems();
@@ -263,8 +296,13 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
         const int c = s_act[a];
         const int t = s_t[hh * d + c];
         const float qv = load_q(q, q_dtype, ((int64_t)g * G + hh) * d + c);
-        s_q32[e] = (t > 0) ? 32.0f * qv : 0.0f;
-        s_qk[e] = (t > 0) ? qv * (__uint_as_float((uint32_t)(130 - t) << 23) - 24.0f) : 0.0f;
+        s_qq[e] = (t > 0) ? make_float2(32.0f * qv, qv * (__uint_as_float((uint32_t)(130 - t) << 23) - 24.0f))
+                          : make_float2(0.0f, 0.0f);
+    }
+    for (int a = tid; a < L; a += T) {   // the tile's rows of every active channel
+        const int64_t row = (int64_t)g * d + s_act[a];
+        s_prow[a] = planes + row * 4 * words_total + tile0 / 32;
+        s_srow[a] = scales + row * nblk_total + tile0 / kBlock;
     }
     // items of (head group, chunk): lane (slot, depth) -> an item when some head
     // of the group reads the slot's channel to exactly that depth; kept in
@@ -300,59 +338,55 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
 
     __syncthreads();   // plan complete
 
-    // The rows of chunk ch: 16-byte pieces e of its plane rows (slot al, plane
-    // j, piece) and scale rows; piece_src() gives a piece's source or null,
-    // piece_dst() its place in raw buffer buf.
-    constexpr int kRowPieces = kTW / 4;                  // 16-byte pieces of a tile's plane row
-    constexpr int kPlanePieces = kCH * 4 * kRowPieces;   // of a chunk's plane rows
-    constexpr int kScalePieces = kCH * (kNB / 8);        // of a chunk's scale rows
-    auto piece_src = [&](int ch, int e) -> const void* {
-        if (e < kPlanePieces) {
-            const int al = e / (4 * kRowPieces), j = (e / kRowPieces) & 3, piece = e % kRowPieces;
-            const int a = ch * kCH + al;
-            if (a < L && j < (int)s_U[a] && piece * 4 < nw)
-                return planes + ((int64_t)(g * d + s_act[a]) * 4 + j) * words_total + tile0 / 32 + piece * 4;
-            return nullptr;
-        }
-        const int es = e - kPlanePieces, al = es / (kNB / 8), piece = es % (kNB / 8);
-        const int a = ch * kCH + al;
-        if (a < L && piece * 8 < nblocks)
-            return scales + (int64_t)(g * d + s_act[a]) * nblk_total + tile0 / kBlock + piece * 8;
-        return nullptr;
+    // The rows of chunk ch in 16-byte pieces: thread tid copies piece lp of
+    // plane lj of slots la0 + kSlotStep * i (i < kPlaneIters), and threads
+    // tid < kScalePieces piece tid & 3 of the scale row of slot tid >> 2.
+    constexpr int kRowPieces = kTW / 4;                          // 16-byte pieces of a tile's plane row
+    constexpr int kPlaneIters = kCH * 4 * kRowPieces / T;        // plane pieces per thread
+    constexpr int kSlotStep = T / (4 * kRowPieces);              // slots apart for one thread
+    constexpr int kScalePieces = kCH * (kNB / 8);
+    static_assert(kCH * 4 * kRowPieces % T == 0 && kScalePieces <= T, "loader geometry");
+    const int lp = tid % kRowPieces, lj = (tid / kRowPieces) & 3, la0 = tid / (4 * kRowPieces);
+    const int64_t ljw = (int64_t)lj * words_total;
+    const bool lp_ok = lp * 4 < nw;
+    auto plane_src = [&](int ch, int i) -> const uint32_t* {
+        const int a = ch * kCH + la0 + kSlotStep * i;
+        return (lp_ok && a < L && lj < (int)s_U[a]) ? s_prow[a] + ljw + lp * 4 : nullptr;
     };
-    auto piece_dst = [&](int buf, int e) -> void* {
-        if (e < kPlanePieces) return s_raw + (size_t)buf * kCH * 4 * kTW + (size_t)e * 4;   // [al][j][piece] in order
-        const int es = e - kPlanePieces;
-        return s_rawsc + (size_t)buf * kCH * kNB + (size_t)es * 8;
+    auto plane_dst = [&](int buf, int i) {
+        return s_raw + ((size_t)(buf * kCH + la0 + kSlotStep * i) * 4 + lj) * kTW + lp * 4;
     };
+    auto scale_src = [&](int ch) -> const uint16_t* {
+        const int a = ch * kCH + (tid >> 2);
+        return (tid < kScalePieces && a < L && (tid & 3) * 8 < nblocks) ? s_srow[a] + (tid & 3) * 8 : nullptr;
+    };
+    auto scale_dst = [&](int buf) { return s_rawsc + (size_t)(buf * kCH + (tid >> 2)) * kNB + (tid & 3) * 8; };
     // device-resident store: cp.async, one chunk ahead
     auto load_chunk = [&](int ch, int buf) {
-        for (int e = tid; e < kPlanePieces + kScalePieces; e += T) {
-            const void* src = piece_src(ch, e);
-            if (src) cp_async16(piece_dst(buf, e), src);
-        }
+#pragma unroll
+        for (int i = 0; i < kPlaneIters; ++i)
+            if (const uint32_t* src = plane_src(ch, i)) cp_async16(plane_dst(buf, i), src);
+        if (const uint16_t* src = scale_src(ch)) cp_async16(scale_dst(buf), src);
         cp_async_commit();
     };
     // host-resident store: plain 16-byte loads into registers, one chunk ahead
     // (over the host link each load of a warp is one run of whole lines;
     // cp.async of page-locked memory carried 2.5x the bytes)
-    constexpr int kPF = (kPlanePieces + kScalePieces + T - 1) / T;
-    uint4 pf[HOST ? kPF : 1];
+    uint4 pf[HOST ? kPlaneIters + 1 : 1];
     auto fetch_chunk = [&](int ch) {
 #pragma unroll
-        for (int i = 0; i < kPF; ++i) {
-            const int e = tid + i * T;
-            const void* src = (e < kPlanePieces + kScalePieces) ? piece_src(ch, e) : nullptr;
+        for (int i = 0; i < kPlaneIters; ++i) {
+            const uint32_t* src = plane_src(ch, i);
             pf[i] = src ? ldg16(src) : make_uint4(0u, 0u, 0u, 0u);
         }
+        const uint16_t* ss = scale_src(ch);
+        pf[kPlaneIters] = ss ? ldg16(ss) : make_uint4(0u, 0u, 0u, 0u);
     };
     auto put_chunk = [&](int ch, int buf) {
 #pragma unroll
-        for (int i = 0; i < kPF; ++i) {
-            const int e = tid + i * T;
-            if (e < kPlanePieces + kScalePieces && piece_src(ch, e))
-                *reinterpret_cast<uint4*>(piece_dst(buf, e)) = pf[i];
-        }
+        for (int i = 0; i < kPlaneIters; ++i)
+            if (plane_src(ch, i)) *reinterpret_cast<uint4*>(plane_dst(buf, i)) = pf[i];
+        if (scale_src(ch)) *reinterpret_cast<uint4*>(scale_dst(buf)) = pf[kPlaneIters];
     };
 
     if (nchunks > 0) {
@@ -380,7 +414,8 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
         // stage: (slot, block) -> 16 code words
         for (int u = tid; u < kCH * kNB; u += T) {
             const int al = u / kNB, bb = u % kNB, a = ch * kCH + al;
-            const int U = (a < L) ? (int)s_U[a] : 0;   // warp-uniform: a warp stages one slot
+            // a warp stages one slot: its depth made warp-uniform to the compiler
+            const int U = (int)__reduce_or_sync(0xffffffffu, (a < L) ? (unsigned)s_U[a] : 0u);
             if (U == 0 || bb >= nblocks) continue;
             const uint32_t* r = s_raw + (size_t)(buf * kCH + al) * 4 * kTW + 2 * bb;
             uint32_t p0[4], p1[4];
@@ -404,16 +439,18 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
         }
         // coefficients: thread (b, p) those of head p of its group, block b, every slot
         if (p < HG) {
-            const int hq = hg * HG + p;
-#pragma unroll 2
+            const int hq = hg * HG + p, nal = L - ch * kCH;   // slots of this chunk: min(nal, kCH)
+            const uint16_t* dsc = s_rawsc + (size_t)buf * kCH * kNB + b;
+            float* wd = s_w2 + (((size_t)hg * kCH) * kNB + b) * HG * 2 + 2 * p;
+#pragma unroll
             for (int al = 0; al < kCH; ++al) {
-                const int a = ch * kCH + al;
-                if (a >= L) break;
-                const float D = __half2float(__ushort_as_half(s_rawsc[(size_t)(buf * kCH + al) * kNB + b]));
-                const float w = s_q32[a * G + hq] * D;
-                *reinterpret_cast<float2*>(s_w2 + ((((size_t)hg * kCH + al) * kNB + b) * HG + p) * 2) =
-                    make_float2(w, w);
-                cst_own = fmaf(s_qk[a * G + hq], D, cst_own);
+                if (al < nal) {
+                    const float D = __half2float(__ushort_as_half(dsc[al * kNB]));
+                    const float2 qq = s_qq[(ch * kCH + al) * G + hq];
+                    const float w = qq.x * D;
+                    *reinterpret_cast<float2*>(wd + (size_t)al * kNB * HG * 2) = make_float2(w, w);
+                    cst_own = fmaf(qq.y, D, cst_own);
+                }
             }
         }
         __syncthreads();   // codes and coefficients of chunk ch are ready

@@ -161,12 +161,14 @@ def layer_inputs(config, layer=0, n=None, n_kv_heads=None, n_q_heads=None, d=Non
 
 
 def layer_inputs_cuda(config, layer=0, n=None, n_kv_heads=None, n_q_heads=None, d=None, device="cuda",
-                      with_values=True, needles=None):
+                      with_values=True, needles=None, part=0):
     """One layer of a workload generated on the GPU (torch's Philox generator,
     seeded like the numpy path): same recipe, different draws.  Returns torch
     tensors on `device`: K f32, K_rows/V_rows bf16 [Hkv][n][d], q (f32 or bf16)
     [Hq][d], sigma2 f32 [Hkv][d]; plus numpy copies of q and sigma2 and the
-    needle positions."""
+    needle positions.  part > 0 draws the keys and values of another key range
+    of the same layer (same channel scales and queries; sigma2 is then that
+    range's own statistic)."""
     import torch
     cfg = CONFIGS[config]
     n = cfg.get("n", 4096) if n is None else n
@@ -175,7 +177,7 @@ def layer_inputs_cuda(config, layer=0, n=None, n_kv_heads=None, n_q_heads=None, 
     d = cfg["d"] if d is None else d
     sigma = channel_sigma(rng_for(config, layer, 0), Hkv, d)
     gen = torch.Generator(device=device)
-    gen.manual_seed(1000 * int(config) + int(layer))
+    gen.manual_seed(1000 * int(config) + int(layer) + 1000003 * int(part))
     K = torch.empty((Hkv, n, d), dtype=torch.float32, device=device)
     sig_t = torch.from_numpy(sigma.astype(np.float32)).to(device)
     for g in range(Hkv):
