@@ -142,94 +142,66 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// The FMAs of one head h for an item: its coefficient pair, 8 paired FMAs.
+// One item for the thread's 16 keys: an item is a channel slot of the chunk,
+// a depth t and the set M of the group's heads that read the slot's channel to
+// exactly depth t (desc bits 0..2: slot, 4..7: M, 8..15: the byte mask of t
+// planes).  The 16 code bytes X are masked to depth t, 16 byte permutes build
+// F_t, and each head of M adds its coefficient pair times F with 8 paired
+// FMAs.  acc[h][2w + r] holds keys (byte 2r, byte 2r + 1) of code word w.
 template <int HG>
-__device__ __forceinline__ void head_fma(int h, const float* wa, const float2 (&F)[8], float2 (&acc)[HG][8]) {
-    const float2 W = *reinterpret_cast<const float2*>(wa + 2 * h);
+__device__ __forceinline__ void item_fma(uint32_t desc, uint4 X, const float* __restrict__ wth,
+                                         float2 (&acc)[HG][8]) {
+    constexpr int kSlotW = kNB * HG * 2;   // floats of one slot's coefficients
+    const uint32_t bm = __byte_perm(desc, 0u, 0x1111u);   // byte 1 in all four bytes
+    X.x &= bm;
+    X.y &= bm;
+    X.z &= bm;
+    X.w &= bm;
+    const uint32_t xs[4] = {X.x, X.y, X.z, X.w};
+    float2 F[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) ffma2(acc[h][i], W, F[i]);
+    for (int w = 0; w < 4; ++w) {
+        F[2 * w] = make_float2(f_of(xs[w], 0), f_of(xs[w], 1));
+        F[2 * w + 1] = make_float2(f_of(xs[w], 2), f_of(xs[w], 3));
+    }
+    const float* wa = wth + (desc & 7) * kSlotW;
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+        if (desc & (16u << h)) {
+            const float2 W = *reinterpret_cast<const float2*>(wa + 2 * h);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ffma2(acc[h][i], W, F[i]);
+        }
+    }
 }
 
-// The items of one (head group, chunk): an item is a channel slot of the
-// chunk, a depth t and the set M of the group's heads that read the slot's
-// channel to exactly depth t (item bits 0..2: slot, 4..7: M, 8..15: the byte
-// mask of t planes).  Per item: the thread's 16 code bytes masked to depth t,
-// 16 byte permutes into F_t, and for each head of M one coefficient pair and
-// 8 paired FMAs, reached by one jump on M.  Every lane reads the same item
-// word; a warp reduction of it gives the compiler a value it knows to be
-// warp-uniform, so the jump needs no divergence handling.  The next item's
-// code words are loaded before the current item is computed.  acc[h][2w + r]
-// holds keys (byte 2r, byte 2r + 1) of code word w of the thread.
+// The items of one (head group, chunk), two per turn: both items' words and
+// code bytes are loaded before either is computed.  Every lane reads the same
+// item words; a warp reduction of each gives the compiler values it knows to
+// be warp-uniform, so the per-head tests are uniform branches.
 template <int HG>
 __device__ __forceinline__ void chunk_items(const uint32_t* __restrict__ items, int nit,
                                             const unsigned char* __restrict__ cth, const float* __restrict__ wth,
                                             float2 (&acc)[HG][8]) {
     constexpr int kSlotCode = kNB * 16 * 4;   // bytes of one slot's code words
-    constexpr int kSlotW = kNB * HG * 2;      // floats of one slot's coefficients
-    if (nit <= 0) return;
-    uint32_t dn = __reduce_or_sync(0xffffffffu, items[0]);
-    uint4 Xn = *reinterpret_cast<const uint4*>(cth + (dn & 7) * kSlotCode);
 #pragma unroll 1
-    for (int it = 0; it < nit; ++it) {
-        const uint32_t desc = dn;
-        uint4 X = Xn;
-        if (it + 1 < nit) {
-            dn = __reduce_or_sync(0xffffffffu, items[it + 1]);
-            Xn = *reinterpret_cast<const uint4*>(cth + (dn & 7) * kSlotCode);
-        }
-        const uint32_t bm = __byte_perm(desc, 0u, 0x1111u);   // byte 1 in all four bytes
-        X.x &= bm;
-        X.y &= bm;
-        X.z &= bm;
-        X.w &= bm;
-        const uint32_t xs[4] = {X.x, X.y, X.z, X.w};
-        float2 F[8];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            F[2 * w] = make_float2(f_of(xs[w], 0), f_of(xs[w], 1));
-            F[2 * w + 1] = make_float2(f_of(xs[w], 2), f_of(xs[w], 3));
-        }
-        const float* wa = wth + (desc & 7) * kSlotW;
-#define FATHOM_HEAD_FMA(h) head_fma<HG>(h, wa, F, acc)
-        if constexpr (HG == 1) {
-            FATHOM_HEAD_FMA(0);
-        } else if constexpr (HG == 2) {
-            switch ((desc >> 4) & 3) {
-                case 1: FATHOM_HEAD_FMA(0); break;
-                case 2: FATHOM_HEAD_FMA(1); break;
-                case 3: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(1); break;
-                default: break;
-            }
-        } else {
-            switch ((desc >> 4) & 15) {
-                case 1: FATHOM_HEAD_FMA(0); break;
-                case 2: FATHOM_HEAD_FMA(1); break;
-                case 3: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(1); break;
-                case 4: FATHOM_HEAD_FMA(2); break;
-                case 5: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(2); break;
-                case 6: FATHOM_HEAD_FMA(1); FATHOM_HEAD_FMA(2); break;
-                case 7: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(1); FATHOM_HEAD_FMA(2); break;
-                case 8: FATHOM_HEAD_FMA(3); break;
-                case 9: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(3); break;
-                case 10: FATHOM_HEAD_FMA(1); FATHOM_HEAD_FMA(3); break;
-                case 11: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(1); FATHOM_HEAD_FMA(3); break;
-                case 12: FATHOM_HEAD_FMA(2); FATHOM_HEAD_FMA(3); break;
-                case 13: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(2); FATHOM_HEAD_FMA(3); break;
-                case 14: FATHOM_HEAD_FMA(1); FATHOM_HEAD_FMA(2); FATHOM_HEAD_FMA(3); break;
-                case 15: FATHOM_HEAD_FMA(0); FATHOM_HEAD_FMA(1); FATHOM_HEAD_FMA(2); FATHOM_HEAD_FMA(3); break;
-                default: break;
-            }
-        }
-#undef FATHOM_HEAD_FMA
+    for (int it = 0; it < nit; it += 2) {
+        const bool two = it + 1 < nit;
+        const uint32_t d0 = __reduce_or_sync(0xffffffffu, items[it]);
+        const uint32_t d1 = two ? __reduce_or_sync(0xffffffffu, items[it + 1]) : 0u;
+        const uint4 X0 = *reinterpret_cast<const uint4*>(cth + (d0 & 7) * kSlotCode);
+        const uint4 X1 = *reinterpret_cast<const uint4*>(cth + (d1 & 7) * kSlotCode);
+        item_fma<HG>(d0, X0, wth, acc);
+        if (two) item_fma<HG>(d1, X1, wth, acc);
     }
 }
 
-// One (tile of kTile keys, KV head g) of one store; q, depths and scores are
-// the store's own [Hq][d], [Hq][d] and [Hq][n_pad_of(n)] arrays; n_pad is the
-// store's row stride (its capacity, >= n_pad_of(n)).
+// The tiles tile_begin, tile_begin + tile_step, ... of KV head g of one store:
+// the plan (depths, union list, per-(slot, head) factors, items) is made once
+// for the head, then every tile is loaded, staged and computed in turn.
 template <int G, bool HOST>
-__device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ scales,
-                                          int d, int64_t n, int64_t n_pad, int tile, int g,
+__device__ __forceinline__ void scan_head_tiles(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ scales,
+                                           int d, int64_t n, int64_t n_pad, int tile_begin, int tile_step, int g,
                                           const void* __restrict__ q, int q_dtype,
                                           const uint8_t* __restrict__ depths, float* __restrict__ scores,
                                           uint32_t* __restrict__ bmax, unsigned int* status) {
@@ -251,13 +223,13 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
     uint8_t* s_t = smem_raw + lay.tdep();
     __shared__ int s_L;
 
-    const int64_t tile0 = (int64_t)tile * kTile;
     const int64_t words_total = n_pad / 32;   // plane row stride
     const int64_t nblk_total = n_pad / kBlock;
     const int64_t len = n_pad_of(n);          // keys covered by tiles
-    const int keys_here = (int)(len - tile0 < kTile ? len - tile0 : kTile);   // a multiple of 1024
-    const int nw = keys_here / 32;
-    const int nblocks = keys_here / kBlock;
+    const int ntiles = (int)scan_tiles(n);
+    // the current tile (set at the top of each tile's turn; the loaders read them)
+    int64_t tile0 = 0;
+    int keys_here = 0, nw = 0, nblocks = 0;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -299,11 +271,6 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
         s_qq[e] = (t > 0) ? make_float2(32.0f * qv, qv * (__uint_as_float((uint32_t)(130 - t) << 23) - 24.0f))
                           : make_float2(0.0f, 0.0f);
     }
-    for (int a = tid; a < L; a += T) {   // the tile's rows of every active channel
-        const int64_t row = (int64_t)g * d + s_act[a];
-        s_prow[a] = planes + row * 4 * words_total + tile0 / 32;
-        s_srow[a] = scales + row * nblk_total + tile0 / kBlock;
-    }
     // items of (head group, chunk): lane (slot, depth) -> an item when some head
     // of the group reads the slot's channel to exactly that depth; kept in
     // lane order (slot, then depth)
@@ -327,12 +294,6 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
     // ---- roles ----
     const int hg = tid / Z::TPG, lt = tid % Z::TPG;
     const int b = lt >> 2, p = lt & 3;   // compute / coefficient thread: block b, word pair p
-    float2 acc[HG][8];
-#pragma unroll
-    for (int h = 0; h < HG; ++h)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[h][i] = make_float2(0.0f, 0.0f);
-    float cst_own = 0.0f;   // constant of (block b, head p of the group), summed over the slots in order
     const unsigned char* cth = reinterpret_cast<const unsigned char*>(s_codes) + b * 64 + 16 * (p ^ swz(b));
     const float* wth = s_w2 + ((size_t)hg * kCH * kNB + b) * HG * 2;
 
@@ -348,10 +309,9 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
     static_assert(kCH * 4 * kRowPieces % T == 0 && kScalePieces <= T, "loader geometry");
     const int lp = tid % kRowPieces, lj = (tid / kRowPieces) & 3, la0 = tid / (4 * kRowPieces);
     const int64_t ljw = (int64_t)lj * words_total;
-    const bool lp_ok = lp * 4 < nw;
     auto plane_src = [&](int ch, int i) -> const uint32_t* {
         const int a = ch * kCH + la0 + kSlotStep * i;
-        return (lp_ok && a < L && lj < (int)s_U[a]) ? s_prow[a] + ljw + lp * 4 : nullptr;
+        return (lp * 4 < nw && a < L && lj < (int)s_U[a]) ? s_prow[a] + ljw + lp * 4 : nullptr;
     };
     auto plane_dst = [&](int buf, int i) {
         return s_raw + ((size_t)(buf * kCH + la0 + kSlotStep * i) * 4 + lj) * kTW + lp * 4;
@@ -389,6 +349,23 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
         if (scale_src(ch)) *reinterpret_cast<uint4*>(scale_dst(buf)) = pf[kPlaneIters];
     };
 
+  for (int tile = tile_begin; tile < ntiles; tile += tile_step) {
+    tile0 = (int64_t)tile * kTile;
+    keys_here = (int)(len - tile0 < kTile ? len - tile0 : kTile);   // a multiple of 1024
+    nw = keys_here / 32;
+    nblocks = keys_here / kBlock;
+    float2 acc[HG][8];
+#pragma unroll
+    for (int h = 0; h < HG; ++h)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[h][i] = make_float2(0.0f, 0.0f);
+    float cst_own = 0.0f;   // constant of (block b, head p of the group), summed over the slots in order
+    for (int a = tid; a < L; a += T) {   // the tile's rows of every active channel
+        const int64_t row = (int64_t)g * d + s_act[a];
+        s_prow[a] = planes + row * 4 * words_total + tile0 / 32;
+        s_srow[a] = scales + row * nblk_total + tile0 / kBlock;
+    }
+    __syncthreads();   // the rows are set; the previous tile's loads and stages are done
     if (nchunks > 0) {
         if constexpr (HOST) {
             fetch_chunk(0);
@@ -499,15 +476,28 @@ __device__ __forceinline__ void scan_tile(const uint32_t* __restrict__ planes, c
             if (bmax && p == 0) bmax[(int64_t)hq * (ld / kBlock) + tile0 / kBlock + b] = kmax;
         }
     }
+  }
 }
 
+// persistent = 0: one tile per CTA, blockIdx.x = KV head * tiles + tile (head
+// major, so that the resident CTAs read consecutive tiles of one or two heads).
+// persistent = 1: blockIdx.x = first tile * Hkv + KV head, and a CTA takes
+// every (gridDim.x / Hkv)-th tile of its head from there.
 template <int G, bool HOST>
 __global__ void __launch_bounds__(Geo<G>::T, Geo<G>::template min_blocks<HOST>())
 scan_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ scales, int d, int64_t n,
-            int64_t n_pad, const void* __restrict__ q, int q_dtype, const uint8_t* __restrict__ depths,
-            float* __restrict__ scores, uint32_t* __restrict__ bmax, unsigned int* status) {
-    scan_tile<G, HOST>(planes, scales, d, n, n_pad, (int)blockIdx.x, (int)blockIdx.y, q, q_dtype, depths, scores,
-                       bmax, status);
+            int64_t n_pad, int Hkv, int persistent, const void* __restrict__ q, int q_dtype,
+            const uint8_t* __restrict__ depths, float* __restrict__ scores, uint32_t* __restrict__ bmax,
+            unsigned int* status) {
+    const int b = (int)blockIdx.x;
+    if (persistent) {
+        scan_head_tiles<G, HOST>(planes, scales, d, n, n_pad, b / Hkv, (int)gridDim.x / Hkv, b % Hkv, q, q_dtype,
+                                 depths, scores, bmax, status);
+    } else {
+        const int tiles = (int)scan_tiles(n);
+        scan_head_tiles<G, HOST>(planes, scales, d, n, n_pad, b % tiles, tiles, b / tiles, q, q_dtype, depths,
+                                 scores, bmax, status);
+    }
 }
 
 // Batched sessions: blockIdx.x runs over the tiles of all sessions.
@@ -528,9 +518,10 @@ scan_batched_kernel(const __grid_constant__ SessionMap map, int d, int Hq, const
     const void* qs = (q_dtype == FATHOM_BF16)
                          ? static_cast<const void*>(static_cast<const uint16_t*>(q) + sidx * qstride)
                          : static_cast<const void*>(static_cast<const float*>(q) + sidx * qstride);
-    scan_tile<G, HOST>(map.planes[sidx], map.scales[sidx], d, map.n[sidx], map.n_pad[sidx], t - map.tile0[sidx],
-                       (int)blockIdx.y, qs, q_dtype, depths + sidx * qstride, scores + map.score_base[sidx],
-                       bmax ? bmax + map.score_base[sidx] / kBlock : nullptr, status);
+    const int tile = t - map.tile0[sidx];
+    scan_head_tiles<G, HOST>(map.planes[sidx], map.scales[sidx], d, map.n[sidx], map.n_pad[sidx], tile, INT32_MAX - tile,
+                        (int)blockIdx.y, qs, q_dtype, depths + sidx * qstride, scores + map.score_base[sidx],
+                        bmax ? bmax + map.score_base[sidx] / kBlock : nullptr, status);
 }
 
 template <int G, bool HOST>
@@ -541,9 +532,29 @@ cudaError_t launch_scan_g(const uint32_t* planes, const uint16_t* scales, int Hk
     auto kern = scan_kernel<G, HOST>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)scan_tiles(n), (unsigned)Hkv);   // the tiles holding keys; n_pad is the stride
-    kern<<<grid, Geo<G>::T, smem, stream>>>(planes, scales, d, n, n_pad, q, q_dtype, depths, scores, bmax,
-                                            device_status_ptr());
+    // One CTA per (tile, KV head) for a host-resident store: the resident CTAs
+    // then read about 600 consecutive tiles of one or two heads at a time,
+    // which the host link serves best.  A device-resident store gets a
+    // persistent grid of as many CTAs as fit on the GPU (a multiple of Hkv):
+    // each CTA plans its head once and walks its tiles.
+    const int64_t tiles = scan_tiles(n);
+    int64_t ctas = tiles * Hkv;
+    int persistent = 0;
+    if (!HOST) {
+        int dev = 0, sms = 0, per_sm = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Geo<G>::T, smem)) != cudaSuccess)
+            return e;
+        const int64_t fit = (int64_t)sms * (per_sm > 0 ? per_sm : 1) / Hkv * Hkv;
+        if (fit >= Hkv && fit < ctas) {
+            ctas = fit;
+            persistent = 1;
+        }
+    }
+    if (ctas > INT32_MAX) return cudaErrorInvalidValue;
+    kern<<<(unsigned)ctas, Geo<G>::T, smem, stream>>>(planes, scales, d, n, n_pad, Hkv, persistent, q, q_dtype,
+                                                      depths, scores, bmax, device_status_ptr());
     return cudaGetLastError();
 }
 
