@@ -36,7 +36,10 @@ namespace {
 constexpr int kSplit = 8;      // CTAs per head (cluster size)
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kUnroll = 8;     // rows in flight per warp
+// rows in flight per warp: all of a lane's row words are loaded before any is
+// used; 16 rows (32 loads per lane) for d <= 128, 8 for d = 256
+template <int V>
+constexpr int unroll_of() { return V <= 4 ? 16 : 8; }
 constexpr int kSortCap = kMaxTopK;   // indices sorted in shared memory
 constexpr int kIdxRegs = (kMaxTopK + kSplit * kWarps * 32 - 1) / (kSplit * kWarps * 32);   // row indices per lane
 
@@ -135,6 +138,7 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
         const int mm = lane + 32 * e;
         my_idx[e] = (mm < rows_w) ? ih[r + kSplit * wp + stride * mm] : -1;
     }
+    constexpr int kUnroll = unroll_of<V>();
     for (int m0 = 0; m0 < rows_w; m0 += kUnroll) {
         RowWords<V> kw[kUnroll], vw[kUnroll];
         bool ok[kUnroll];

@@ -798,6 +798,58 @@ __device__ __forceinline__ void cluster_pick(uint32_t* hist, uint32_t* hsum, int
     }
 }
 
+// The top k of a row whose candidates (keys with (key >> 20) >= b12, at most
+// kMaxTopK of them over the cluster, at least k) are known: each CTA sorts its
+// own candidates (composites, descending) in its shared buffer; the rank of a
+// candidate in the row is its position in its CTA's list plus, for every
+// other CTA, the number of that CTA's candidates above it (a binary search in
+// that CTA's sorted list through distributed shared memory); ranks below k
+// are written out.  Composites are distinct (the index is part of them), so
+// the ranks are a permutation and ties order by index.
+template <int CL>
+__device__ void topk_rows_candidates(const uint32_t* keys, int cnt, int64_t start, uint32_t b12, int k, uint64_t* buf,
+                                     int* s_fill, int row, int32_t* __restrict__ idx,
+                                     float* __restrict__ top_scores) {
+    const int tid = threadIdx.x;
+    if (tid == 0) *s_fill = 0;
+    __syncthreads();
+    for (int e = tid; e < cnt; e += kRowThreads)
+        if ((keys[e] >> 20) >= b12) buf[atomicAdd(s_fill, 1)] = composite(keys[e], start + e);
+    __syncthreads();
+    const int c = *s_fill;
+    int S = 1;
+    while (S < c) S <<= 1;
+    for (int e = c + tid; e < S; e += kRowThreads) buf[e] = 0ull;   // below every composite of the row
+    __syncthreads();
+    if (S > 1) bitonic_desc(buf, S);
+    cluster_barrier<CL>();   // every CTA's list is sorted and its count published
+    for (int j = tid; j < c; j += kRowThreads) {
+        const uint64_t v = buf[j];
+        int r = j;
+        if constexpr (CL > 1) {
+            cg::cluster_group cluster = cg::this_cluster();
+            const int x = (int)cluster.block_rank();
+#pragma unroll
+            for (int y = 0; y < CL; ++y) {
+                if (y == x) continue;
+                const uint64_t* ly = cluster.map_shared_rank(buf, y);
+                int lo = 0, hi = *cluster.map_shared_rank(s_fill, y);   // first position below v
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (ly[mid] > v) lo = mid + 1;
+                    else hi = mid;
+                }
+                r += lo;
+            }
+        }
+        if (r < k) {
+            idx[(int64_t)row * k + r] = (int32_t)(0xFFFFFFFFu - (uint32_t)v);
+            if (top_scores) top_scores[(int64_t)row * k + r] = ordered_to_float((uint32_t)(v >> 32));
+        }
+    }
+    cluster_barrier<CL>();   // keep every CTA's list alive until all searches are done
+}
+
 template <int CL>
 __global__ void __launch_bounds__(kRowThreads)
 topk_rows(const float* __restrict__ scores, const __grid_constant__ RowMap m, int k, int32_t* __restrict__ idx,
@@ -862,8 +914,15 @@ topk_rows(const float* __restrict__ scores, const __grid_constant__ RowMap m, in
         need -= s_above;
         above += s_above;
         prefix = (shift == 32 ? 0u : (prefix << nbits)) | (uint32_t)s_bin;
+        const uint32_t in_bin = s_cnt;   // keys of the row in the picked bin (the same in every CTA)
         shift = sh;
         __syncthreads();   // s_bin / s_above are rewritten by the next step
+        if (shift == 20 && above + in_bin <= (uint32_t)kMaxTopK) {
+            // few keys at or above the k-th key's top-12-bit bin: they are the
+            // candidates, and an exact sort of them gives the top k
+            topk_rows_candidates<CL>(keys, cnt, start, prefix, k, buf, &s_fill, row, idx, top_scores);
+            return;
+        }
     }
     const uint32_t T = prefix;
     const int gt_row = (int)above, take_eq = k - gt_row;   // keys above T; ties to take (>= 1)
