@@ -586,6 +586,27 @@ def config12_cases(F, torch, dev, config, steps, warmup, flush, with_oracle=True
         del graph
         dep = F.alloc_depths(inp["q_dev"], inp["sigma2_dev"], b, fixed_r=fr)
         scan = _events_ms(torch, lambda: F.scan_scores(st, inp["q_dev"], dep), steps, warmup, flush)
+        # the same step as separate launches, each bracketed by CUDA events
+        sc = torch.empty((Hq, st.n_pad), dtype=torch.float32, device=dev)
+        bm = F.block_max_buffer(Hq, n, dev)
+        tws = torch.empty(F.topk_workspace_bytes(n, Hq, k), dtype=torch.uint8, device=dev)
+        parts = []
+        for it in range(warmup + steps):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            ev[0].record()
+            F.alloc_depths(inp["q_dev"], inp["sigma2_dev"], b, fixed_r=fr, out=bufs["depths"])
+            ev[1].record()
+            F.scan_scores(st, inp["q_dev"], bufs["depths"], out=sc, block_max=bm)
+            ev[2].record()
+            F.topk(sc, n, k, idx=bufs["idx"], top_scores=bufs["top_scores"], workspace=tws, block_max=bm)
+            ev[3].record()
+            F.sparse_attend(inp["q_dev"], Kr, Vr, bufs["idx"], out=bufs["out"])
+            ev[4].record()
+            ev[4].synchronize()
+            if it >= warmup:
+                parts.append([ev[j].elapsed_time(ev[j + 1]) * 1e3 for j in range(4)])
+        med = np.median(np.array(parts), axis=0)
         U = dep.view(Hkv, Hq // Hkv, 128).amax(dim=1)
         nbytes = st.plane_bytes_read(U)
         rec = {"config": config, "case": name, "workload": cfg["name"], "n": n, "n_kv_heads": Hkv,
@@ -593,6 +614,8 @@ def config12_cases(F, torch, dev, config, steps, warmup, flush, with_oracle=True
                "step_us_warm": float(np.median(t_warm)) * 1e3,
                "step_us_cuda_graph_l2_flushed": float(np.median(t_graph)) * 1e3,
                "scan_us": float(np.median(scan)) * 1e3,
+               "breakdown_us": {"depths": float(med[0]), "scan": float(med[1]), "topk": float(med[2]),
+                                "attend": float(med[3])},
                "gkeys_per_s_step": n * Hkv / (float(np.median(t_flush)) * 1e-3) / 1e9,
                "scan_bytes_per_key_per_kv_head": nbytes / (n * Hkv),
                "scan_hbm_gbs": nbytes / (float(np.median(scan)) * 1e-3) / 1e9}
@@ -834,7 +857,8 @@ def shard_bench(args):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    ranks = Ranks("nccl", device=dev, sync=torch.cuda.synchronize, timeout_s=300)
+    # the step's all-gathers run at every world size, one rank included
+    ranks = Ranks("nccl", device=dev, sync=torch.cuda.synchronize, timeout_s=300, always_group=True)
     world, rank = ranks.world, ranks.rank
     n, k, B = args.n, args.k, args.budget
     inp = synth.layer_inputs_cuda(3, n=n, device=dev, with_values=True, needles=0, part=rank)

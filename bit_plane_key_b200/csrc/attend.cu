@@ -6,11 +6,15 @@
 // g = h / (Hq/Hkv), K and V rows in bf16, fp32 accumulation, exp via exp2f.
 //
 // One thread-block cluster of kSplit CTAs per query head.  CTA r of the
-// cluster takes every kSplit-th of the head's k selected keys; inside it each
-// warp runs an online softmax over its rows (lane l holds channels
-// [l*d/32, (l+1)*d/32)).  The warps' partial (max, sum, o) merge in shared
-// memory, then CTA 0 merges the kSplit CTA partials through distributed
-// shared memory and writes o_h.  No workspace and no second kernel.
+// cluster takes every kSplit-th of the head's k selected keys.  Inside it a
+// row is held by d/16 lanes of a warp (16 channels each, read as 16-byte
+// pieces), so a warp works on 32/(d/16) rows at once, each group of lanes
+// running its own online softmax; the groups merge by shuffles, the warps'
+// partial (max, sum, o) in shared memory, then CTA 0 merges the kSplit CTA
+// partials through distributed shared memory and writes o_h.  No workspace
+// and no second kernel.  Products and sums use packed two-lane FMAs; the
+// running maximum moves only when a score passes it by more than 2^8, so the
+// per-row rescale of o is skipped on almost every row.
 // With a key range split across GPUs, each rank runs the same kernel over
 // the rows it holds (global indices shifted by its first key; the other
 // ranks' indices skipped) and writes the CTA 0 merge unnormalised: o relative
@@ -36,51 +40,44 @@ namespace {
 constexpr int kSplit = 8;      // CTAs per head (cluster size)
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-// rows in flight per warp: all of a lane's row words are loaded before any is
-// used; 16 rows (32 loads per lane) for d <= 128, 8 for d = 256
-template <int V>
-constexpr int unroll_of() { return V <= 4 ? 16 : 8; }
 constexpr int kSortCap = kMaxTopK;   // indices sorted in shared memory
 constexpr int kIdxRegs = (kMaxTopK + kSplit * kWarps * 32 - 1) / (kSplit * kWarps * 32);   // row indices per lane
+// A slot's running maximum is moved (and its sum and output rescaled) only
+// when a score passes it by more than kTau (log2 units): exp2(score - m) then
+// stays below 2^kTau, and the result is the same softmax up to rounding.
+constexpr float kTau = 8.0f;
 
-
-// A lane's V bf16 values of a row, kept as raw 32-bit words until used: the
-// loads of all rows in flight are issued before any value is converted.
-template <int V>
-struct RowWords {
-    static constexpr int W = (V + 1) / 2;
-    uint32_t w[W];
-    __device__ __forceinline__ void load(const uint16_t* __restrict__ p) {
-        if constexpr (V == 8) {
-            const uint4 u = *reinterpret_cast<const uint4*>(p);
-            w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
-        } else if constexpr (V == 4) {
-            const uint2 u = *reinterpret_cast<const uint2*>(p);
-            w[0] = u.x; w[1] = u.y;
-        } else if constexpr (V == 2) {
-            w[0] = *reinterpret_cast<const uint32_t*>(p);
-        } else {
-            w[0] = p[0];
-        }
-    }
-    __device__ __forceinline__ void clear() {
-#pragma unroll
-        for (int e = 0; e < W; ++e) w[e] = 0u;
-    }
-    __device__ __forceinline__ float at(int e) const {   // value e (bf16 -> f32 is a shift)
-        const uint32_t x = w[e >> 1];
-        return (V == 1) ? __uint_as_float(x << 16) : ((e & 1) ? __uint_as_float(x & 0xFFFF0000u)
-                                                              : __uint_as_float(x << 16));
-    }
+// Lane layout for head dimension D.  LPR = D / 16 lanes share a row ("a
+// slot"), each holding 16 channels: lane j of a slot reads the 16-byte pieces
+// t = 0, 1 of the K row and of the V row that start at channel t * D/2 + 8 j,
+// so one warp load instruction reads D contiguous bytes of each of the RPW =
+// 32 / LPR rows it covers.  A lane keeps R rows in flight: a warp loads RB =
+// R * RPW rows before it uses any of them.
+template <int D>
+struct Lanes {
+    static constexpr int LPR = D / 16;
+    static constexpr int RPW = 32 / LPR;
+    static constexpr int R = (D == 32) ? 2 : 4;
+    static constexpr int RB = R * RPW;
+    static_assert(32 % RB == 0, "a batch's row positions lie in one index register");
 };
 
-template <int V>
+// a word of two bf16 values as two floats (bf16 -> f32 is a shift)
+__device__ __forceinline__ float2 bf16x2_f2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int w) {
+    return w == 0 ? v.x : (w == 1 ? v.y : (w == 2 ? v.z : v.w));
+}
+
+template <int D>
 __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kThreads)
 attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restrict__ Kr,
               const uint16_t* __restrict__ Vr, int64_t row_stride, const int32_t* __restrict__ idx, int Hq, int Hkv,
               int64_t n, int64_t key0, int k, int sort_rows, float* __restrict__ out, float* __restrict__ parts,
               unsigned int* status) {
-    constexpr int d = V * 32;
+    using Ln = Lanes<D>;
+    constexpr int d = D;
     __shared__ int32_t s_idx[kSortCap];
     __shared__ float s_m[kWarps], s_l[kWarps];
     __shared__ float s_o[kWarps][d];
@@ -92,15 +89,28 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
     const int h = blockIdx.x / kSplit;
     const int g = h / (Hq / Hkv);
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    const int slot = lane / Ln::LPR, j = lane % Ln::LPR;
     const float scale = 1.4426950408889634f / sqrtf((float)d);  // log2(e)/sqrt(d)
 
-    float qv[V];
+    // the query's channels of this lane, in pairs: piece t, word w holds
+    // channels t * d/2 + 8 j + 2 w and the one after it
+    float2 q2[2][4];
 #pragma unroll
-    for (int e = 0; e < V; ++e) qv[e] = load_q(q, q_dtype, (int64_t)h * d + lane * V + e) * scale;
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int64_t c = (int64_t)h * d + t * (d / 2) + 8 * j + 2 * w;
+            q2[t][w] = make_float2(load_q(q, q_dtype, c) * scale, load_q(q, q_dtype, c + 1) * scale);
+        }
 
-    float m = -INFINITY, l = 0.0f, o[V];
+    // the slot's online softmax: maximum m and sum l (log2 units), output o
+    // for the lane's channels (same pairing as q2)
+    float m = -INFINITY, l = 0.0f;
+    float2 o2[2][4];
 #pragma unroll
-    for (int e = 0; e < V; ++e) o[e] = 0.0f;
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) o2[t][w] = make_float2(0.0f, 0.0f);
 
     const int32_t* ih = idx + (int64_t)h * k;
     const int64_t head_base = (int64_t)g * n * row_stride;
@@ -113,12 +123,12 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
         for (int size = 2; size <= P; size <<= 1) {
             for (int stride = size >> 1; stride > 0; stride >>= 1) {
                 for (int t = threadIdx.x; t < P / 2; t += kThreads) {
-                    const int i = 2 * t - (t & (stride - 1)), j = i + stride;
+                    const int i = 2 * t - (t & (stride - 1)), j2 = i + stride;
                     const bool up = (i & size) == 0;
-                    const int32_t a = s_idx[i], b2 = s_idx[j];
+                    const int32_t a = s_idx[i], b2 = s_idx[j2];
                     if ((a > b2) == up) {
                         s_idx[i] = b2;
-                        s_idx[j] = a;
+                        s_idx[j2] = a;
                     }
                 }
                 __syncthreads();
@@ -126,10 +136,10 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
         }
         ih = s_idx;
     }
-    // rows of this warp: positions p = r + kSplit * (wp + kWarps * m) of the (sorted) list,
+    // rows of this warp: positions p = r + kSplit * (wp + kWarps * mm) of the (sorted) list,
     // so the head's warps sweep the list together, in address order when sorted.
-    // The warp's row indices are read once, lane j holding those of m = j + 32 e,
-    // so every batch issues its row loads at once
+    // The warp's row indices are read once, lane x holding those of mm = x + 32 e;
+    // batch m0 takes mm = m0 + u * RPW + slot for u < R
     const int stride = kSplit * kWarps;
     const int rows_w = (k - (r + kSplit * wp) + stride - 1) / stride;   // rows of this warp (may be <= 0)
     int32_t my_idx[kIdxRegs];
@@ -138,48 +148,83 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
         const int mm = lane + 32 * e;
         my_idx[e] = (mm < rows_w) ? ih[r + kSplit * wp + stride * mm] : -1;
     }
-    constexpr int kUnroll = unroll_of<V>();
-    for (int m0 = 0; m0 < rows_w; m0 += kUnroll) {
-        RowWords<V> kw[kUnroll], vw[kUnroll];
-        bool ok[kUnroll];
+    for (int m0 = 0; m0 < rows_w; m0 += Ln::RB) {
+        int32_t reg = -1;   // the index register holding this batch (warp-uniform choice)
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int mm = m0 + u;
+        for (int e = 0; e < kIdxRegs; ++e)
+            if ((m0 >> 5) == e) reg = my_idx[e];
+        uint4 kp[Ln::R][2], vp[Ln::R][2];
+        bool ok[Ln::R];
+#pragma unroll
+        for (int u = 0; u < Ln::R; ++u) {
+            const int mm = m0 + u * Ln::RPW + slot;
+            const int32_t i = __shfl_sync(0xffffffffu, reg, (m0 & 31) + u * Ln::RPW + slot);
             ok[u] = false;
-            kw[u].clear();
-            vw[u].clear();
-            int32_t i = -1;
 #pragma unroll
-            for (int e = 0; e < kIdxRegs; ++e)
-                if ((mm >> 5) == e) i = __shfl_sync(0xffffffffu, my_idx[e], mm & 31);
+            for (int t = 0; t < 2; ++t) kp[u][t] = vp[u][t] = make_uint4(0u, 0u, 0u, 0u);
             if (mm < rows_w) {
                 const int64_t il = (int64_t)i - key0;   // row in this array
                 if (il >= 0 && il < n) {
                     ok[u] = true;
-                    const int64_t off = head_base + il * row_stride + lane * V;
-                    kw[u].load(Kr + off);
-                    vw[u].load(Vr + off);
-                } else if (!parts && lane == 0) {   // a partial skips the other ranges' rows
+                    const int64_t off = head_base + il * row_stride + 8 * j;
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        kp[u][t] = *reinterpret_cast<const uint4*>(Kr + off + t * (d / 2));
+                        vp[u][t] = *reinterpret_cast<const uint4*>(Vr + off + t * (d / 2));
+                    }
+                } else if (!parts && j == 0) {   // a partial skips the other ranges' rows
                     atomicOr(status, (unsigned)FATHOM_DEV_BAD_INDEX);
                 }
             }
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            float dot = 0.0f;
+        for (int u = 0; u < Ln::R; ++u) {
+            float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int e = 0; e < V; ++e) dot = fmaf(qv[e], kw[u].at(e), dot);
+            for (int t = 0; t < 2; ++t)
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-            if (!ok[u]) continue;   // warp-uniform
-            float mn = fmaxf(m, dot);
-            float a = exp2f(m - mn);     // 0 when m = -inf
-            float p = exp2f(dot - mn);
-            l = l * a + p;
+                for (int w = 0; w < 4; ++w) acc = __ffma2_rn(q2[t][w], bf16x2_f2(word_of(kp[u][t], w)), acc);
+            float x = acc.x + acc.y;
 #pragma unroll
-            for (int e = 0; e < V; ++e) o[e] = fmaf(p, vw[u].at(e), o[e] * a);
-            m = mn;
+            for (int off = Ln::LPR / 2; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+            if (!ok[u]) continue;   // uniform within the slot
+            if (x > m + kTau) {     // also the slot's first row (m = -inf)
+                const float a = exp2f(m - x);   // 0 when m = -inf
+                l *= a;
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) o2[t][w] = make_float2(o2[t][w].x * a, o2[t][w].y * a);
+                m = x;
+            }
+            const float p = exp2f(x - m);
+            l += p;
+            const float2 pp = make_float2(p, p);
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int w = 0; w < 4; ++w) o2[t][w] = __ffma2_rn(pp, bf16x2_f2(word_of(vp[u][t], w)), o2[t][w]);
         }
+    }
+
+    // merge the warp's slots: lane j of every slot holds the same channels
+#pragma unroll
+    for (int off = Ln::LPR; off < 32; off <<= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m, off);
+        const float lo = __shfl_xor_sync(0xffffffffu, l, off);
+        const float mn = fmaxf(m, mo);
+        const float fa = (m == -INFINITY) ? 0.0f : exp2f(m - mn);
+        const float fb = (mo == -INFINITY) ? 0.0f : exp2f(mo - mn);
+        l = l * fa + lo * fb;
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float ox = __shfl_xor_sync(0xffffffffu, o2[t][w].x, off);
+                const float oy = __shfl_xor_sync(0xffffffffu, o2[t][w].y, off);
+                o2[t][w] = make_float2(o2[t][w].x * fa + ox * fb, o2[t][w].y * fa + oy * fb);
+            }
+        m = mn;
     }
 
     // merge the warps of this CTA
@@ -187,8 +232,15 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
         s_m[wp] = m;
         s_l[wp] = l;
     }
+    if (slot == 0) {
 #pragma unroll
-    for (int e = 0; e < V; ++e) s_o[wp][lane * V + e] = o[e];
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                s_o[wp][t * (d / 2) + 8 * j + 2 * w] = o2[t][w].x;
+                s_o[wp][t * (d / 2) + 8 * j + 2 * w + 1] = o2[t][w].y;
+            }
+    }
     __syncthreads();
     {
         float M = -INFINITY;
@@ -281,10 +333,10 @@ cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, co
         return cudaGetLastError();
     };
     switch (d) {
-        case 32: return go(attend_kernel<1>);
-        case 64: return go(attend_kernel<2>);
-        case 128: return go(attend_kernel<4>);
-        case 256: return go(attend_kernel<8>);
+        case 32: return go(attend_kernel<32>);
+        case 64: return go(attend_kernel<64>);
+        case 128: return go(attend_kernel<128>);
+        case 256: return go(attend_kernel<256>);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -17,16 +17,20 @@ class Ranks:
     """The process group of a run launched by torch.distributed.run (or a
     single process when WORLD_SIZE is unset or 1)."""
 
-    def __init__(self, backend="nccl", device=None, sync=None, timeout_s=600):
+    def __init__(self, backend="nccl", device=None, sync=None, timeout_s=600, always_group=False):
+        """always_group: make a process group also for a single process (a
+        path that calls collectives itself then runs unchanged at world 1)."""
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.device = device
         self._sync = sync
         self.dist = None
-        if self.world > 1:
+        if self.world > 1 or always_group:
             import torch.distributed as dist
             os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            if self.world == 1 and "MASTER_PORT" not in os.environ:
+                os.environ.update(MASTER_PORT=str(_free_port()), RANK="0", WORLD_SIZE="1")
             kw = {"device_id": device} if backend == "nccl" and device is not None else {}
             dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
             self.dist = dist
@@ -52,6 +56,13 @@ class Ranks:
             self.dist.barrier()
             self.dist.destroy_process_group()
             self.dist = None
+
+
+def _free_port():
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
 
 
 def layer_of_rank(rank):

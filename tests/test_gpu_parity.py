@@ -459,6 +459,31 @@ def test_sparse_attend(ref, d, k, host_rows, interleaved):
     assert F.last_device_status() == 0
 
 
+@pytest.mark.parametrize("order", ["rising", "falling"])
+@pytest.mark.parametrize("d", [32, 128, 256])
+def test_sparse_attend_running_maximum_moves(ref, d, order):
+    """Rows given in order of rising exact score make the running maximum of
+    every lane group move again and again (the rescale branch on almost every
+    row); falling order takes it once.  q is scaled up so the logits span a
+    wide range (softmax weights from 1 down to far below fp32's epsilon)."""
+    Hkv, G, n, k = 1, 4, 6000, 1500
+    inp = make(2, n=n, Hkv=Hkv, Hq=Hkv * G, d=d, values=True)
+    q = (inp["q"] * 12.0).astype(np.float32)
+    Kf = synth.bf16_bits_to_f32(inp["K_rows"]).astype(np.float64)
+    rng = np.random.default_rng(d)
+    idx = np.empty((G, k), dtype=np.int32)
+    for h in range(G):
+        sel = rng.choice(n, k, replace=False)
+        s = Kf[0][sel] @ q[h].astype(np.float64)
+        sel = sel[np.argsort(s, kind="stable")]
+        idx[h] = sel if order == "rising" else sel[::-1]
+    out = host(F.sparse_attend(dev(q), bf16(inp["K_rows"]), bf16(inp["V_rows"]), dev(idx)))
+    want = ref.attend(q, inp["K_rows"], inp["V_rows"], idx)
+    for h in range(G):
+        assert np.linalg.norm(out[h] - want[h]) <= 1e-4 * np.linalg.norm(want[h]), (h, order)
+    assert F.last_device_status() == 0
+
+
 def test_sparse_attend_rejects_bad_row_stride():
     inp = make(2, n=300, Hkv=1, Hq=4, d=128, values=True)
     Kr, Vr = bf16(inp["K_rows"]), bf16(inp["V_rows"])

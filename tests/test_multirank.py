@@ -79,6 +79,35 @@ def test_single_process_needs_no_group():
     assert ms == 5.0 and v == pytest.approx((1 << 20) / 5e-3 / 1e9)
 
 
+def _one_rank_group_main(outdir):
+    os.environ.pop("MASTER_PORT", None)
+    os.environ.pop("WORLD_SIZE", None)
+    os.environ.pop("RANK", None)
+    sys.path.insert(0, ROOT)
+    import torch
+    from bit_plane_key_b200.ranks import Ranks
+    from bit_plane_key_b200.shard import gather_candidates
+    r = Ranks("gloo", device=torch.device("cpu"), timeout_s=60, always_group=True)
+    s, i = gather_candidates(torch.tensor([[3.0, 1.0]]), torch.tensor([[7, 2]], dtype=torch.int32))
+    res = {"world": r.world, "group": r.dist is not None, "s": s.tolist(), "i": i.tolist(), "max": r.max(2.5)}
+    r.close()
+    with open(os.path.join(outdir, "one.json"), "w") as f:
+        json.dump(res, f)
+
+
+def test_single_process_group_on_request(tmp_path):
+    """always_group makes a one-rank group, so a path that calls collectives
+    (the key-range sharded step) runs unchanged without a launcher."""
+    ctx = mp.get_context("spawn")
+    p = ctx.Process(target=_one_rank_group_main, args=(str(tmp_path),))
+    p.start()
+    p.join(120)
+    assert p.exitcode == 0
+    with open(tmp_path / "one.json") as f:
+        r = json.load(f)
+    assert r == {"world": 1, "group": True, "s": [[3.0, 1.0]], "i": [[7, 2]], "max": 2.5}
+
+
 def _shard_rank_main(rank, world, port, outdir, scores_path):
     """Key-range sharding on CPU: local top-k of the rank's range (the oracle),
     the gloo all-gather of (score, global index) lists, then a merge."""
