@@ -556,7 +556,7 @@ def _graph_of(torch, fn, warmup=3):
     return g
 
 
-def config12_cases(F, torch, dev, config, steps, warmup, flush, with_oracle=True):
+def config12_cases(F, torch, dev, config, steps, warmup, flush, with_oracle=True, groups=1):
     """Configs 1 and 2 (HBM-resident): one record per budget case (config 2
     adds fixed68 / fixed136), each timed through the one-call decode step: L2
     flushed, warm, and replayed from a CUDA graph; the scan alone; and (with
@@ -568,7 +568,7 @@ def config12_cases(F, torch, dev, config, steps, warmup, flush, with_oracle=True
     Hkv, Hq, n, k = cfg["n_kv_heads"], cfg["n_q_heads"], cfg["n"], cfg["k"]
     st = F.pack_bitplanes(inp["K"])
     Kr, Vr = inp["K_rows"], inp["V_rows"]
-    ws = torch.empty(F.decode_workspace_bytes(st, Hq, k, 1), dtype=torch.uint8, device=dev)
+    ws = torch.empty(F.decode_workspace_bytes(st, Hq, k, groups), dtype=torch.uint8, device=dev)
     bufs = dict(depths=torch.empty((Hq, 128), dtype=torch.uint8, device=dev),
                 idx=torch.empty((Hq, k), dtype=torch.int32, device=dev),
                 top_scores=torch.empty((Hq, k), dtype=torch.float32, device=dev),
@@ -578,7 +578,8 @@ def config12_cases(F, torch, dev, config, steps, warmup, flush, with_oracle=True
         cases += [("fixed68_r16", 0, 16), ("fixed136_r32", 0, 32)]
     out = []
     for name, b, fr in cases:
-        step = lambda: F.decode_step(st, inp["q_dev"], inp["sigma2_dev"], b, k, Kr, Vr, fixed_r=fr, **bufs)
+        step = lambda: F.decode_step(st, inp["q_dev"], inp["sigma2_dev"], b, k, Kr, Vr, fixed_r=fr, kv_groups=groups,
+                                     **bufs)
         t_flush = _events_ms(torch, step, steps, warmup, flush)
         t_warm = _events_ms(torch, step, steps, warmup)
         graph = _graph_of(torch, step)   # the same call replayed from a CUDA graph: no host launch cost
@@ -609,7 +610,7 @@ def config12_cases(F, torch, dev, config, steps, warmup, flush, with_oracle=True
         med = np.median(np.array(parts), axis=0)
         U = dep.view(Hkv, Hq // Hkv, 128).amax(dim=1)
         nbytes = st.plane_bytes_read(U)
-        rec = {"config": config, "case": name, "workload": cfg["name"], "n": n, "n_kv_heads": Hkv,
+        rec = {"config": config, "case": name, "workload": cfg["name"], "kv_groups": groups, "n": n, "n_kv_heads": Hkv,
                "n_q_heads": Hq, "k": k, "step_us_l2_flushed": float(np.median(t_flush)) * 1e3,
                "step_us_warm": float(np.median(t_warm)) * 1e3,
                "step_us_cuda_graph_l2_flushed": float(np.median(t_graph)) * 1e3,
@@ -705,7 +706,7 @@ def config_bench(args):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     out = []
     if args.config in (1, 2):
-        out = config12_cases(F, torch, dev, args.config, args.steps, args.warmup, flush)
+        out = config12_cases(F, torch, dev, args.config, args.steps, args.warmup, flush, groups=args.kv_groups)
     elif args.config == 4:
         out = [config4_step(F, torch, dev, args.steps, args.warmup, flush)]
     elif args.config == 5:
@@ -935,7 +936,7 @@ def matched_bench(args):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     refs = fidelity_refs(torch, layer.q, layer.inp["K_rows"], layer.inp["V_rows"], k, G)
     rows = []
-    budgets = (36, 40, 46, 52, 56, 60, 68, 80, 92)
+    budgets = (36, 46, 56, 68, 80, 92, 104, 116, 128, 136)
     for name, b, fr in [("B=%d" % b, b, 0) for b in budgets] + [("fixed68_r16", 0, 16), ("fixed136_r32", 0, 32)]:
         t = timed_pipelined(torch, layer, b, args.steps, args.warmup, fr, flush, 1)["step_ms"]
         nbytes, _ = layer.union_bytes()

@@ -276,7 +276,7 @@ int fathom_scan_topk(const fathom_store* store, const void* q, int q_dtype, cons
                                 depths, n_q_heads, scores, s, bmax, store->host_resident != 0);
     if (e != cudaSuccess) return FATHOM_ECUDA;
     e = launch_topk_blocks(scores, bmax, store->n, ld, n_q_heads, k, idx, top_scores,
-                           static_cast<char*>(workspace) + lay.topk_off, s);
+                           static_cast<char*>(workspace) + lay.topk_off, s, true);
     return to_status(e);
 }
 
@@ -359,7 +359,7 @@ int fathom_scan_topk_batched(const fathom_store* stores, int n_sessions, const v
                                         cs, bmax, any_host);
     if (e != cudaSuccess) return FATHOM_ECUDA;
     return to_status(launch_topk_blocks_map(scores, bmax, rm, n_sessions * n_q_heads, k, idx, top_scores,
-                                            static_cast<char*>(workspace) + off + a256(off / kBlock), cs));
+                                            static_cast<char*>(workspace) + off + a256(off / kBlock), cs, true));
 }
 
 int fathom_sparse_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,

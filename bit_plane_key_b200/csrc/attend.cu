@@ -76,6 +76,7 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
               const uint16_t* __restrict__ Vr, int64_t row_stride, const int32_t* __restrict__ idx, int Hq, int Hkv,
               int64_t n, int64_t key0, int k, int sort_rows, float* __restrict__ out, float* __restrict__ parts,
               unsigned int* status) {
+    pdl_wait();
     using Ln = Lanes<D>;
     constexpr int d = D;
     __shared__ int32_t s_idx[kSortCap];
@@ -294,6 +295,7 @@ attend_kernel(const void* __restrict__ q, int q_dtype, const uint16_t* __restric
 // ranges summed in order r = 0, 1, ...  One CTA per head.
 __global__ void __launch_bounds__(128)
 attend_merge_kernel(const float* __restrict__ parts, int world, int Hq, int d, float* __restrict__ out) {
+    pdl_wait();
     const int h = blockIdx.x;
     const int64_t rs = (int64_t)Hq * (d + 2);   // one range's partials
     const float* p = parts + (int64_t)h * (d + 2);
@@ -323,14 +325,13 @@ cudaError_t launch_attend_merge(const float* parts, int world, int Hq, int d, fl
 
 cudaError_t launch_attend(const void* q, int q_dtype, const uint16_t* K_rows, const uint16_t* V_rows,
                           int64_t row_stride, const int32_t* idx, int Hq, int Hkv, int64_t n, int d, int k,
-                          int sort_rows, float* out, cudaStream_t stream, int64_t key0, float* parts) {
+                          int sort_rows, float* out, cudaStream_t stream, int64_t key0, float* parts, bool pdl) {
     dim3 grid((unsigned)(Hq * kSplit));
     unsigned int* st = device_status_ptr();
     const int sr = (sort_rows && k <= kSortCap) ? 1 : 0;
     auto go = [&](auto kern) {
-        kern<<<grid, kThreads, 0, stream>>>(q, q_dtype, K_rows, V_rows, row_stride, idx, Hq, Hkv, n, key0, k, sr, out,
-                                            parts, st);
-        return cudaGetLastError();
+        return launch_ex(kern, grid, dim3(kThreads), 0, stream, pdl, 1, q, q_dtype, K_rows, V_rows, row_stride, idx, Hq,
+                         Hkv, n, key0, k, sr, out, parts, st);
     };
     switch (d) {
         case 32: return go(attend_kernel<32>);

@@ -9,7 +9,10 @@
 // The auxiliary stream is forked from and joined back to the caller's stream
 // with events, so the whole step is ordered on the caller's stream and can be
 // captured into a CUDA graph.  With one group the step is the plain sequence
-// depths -> scan -> top-k -> attention.
+// depths -> scan -> top-k -> attention on the caller's stream, each launch
+// made with programmatic serialization, so that it is scheduled while the
+// kernel before it finishes (every kernel waits for its predecessor's
+// results before it reads anything).
 //
 // Every kernel is one of the separate entry points' kernels, launched on a
 // slice of the same arrays, so the results equal fathom_alloc_depths +
@@ -71,8 +74,6 @@ cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int st
                           const uint16_t* K_rows, const uint16_t* V_rows, int64_t row_stride, int64_t rows_n,
                           int rows_host, int groups, uint8_t* depths, int32_t* idx, float* top_scores, float* out,
                           void* workspace, cudaStream_t stream) {
-    Aux* aux = aux_for_device();
-    if (!aux) return cudaErrorUnknown;
     const int hkv_g = Hkv / groups, hq_g = Hq / groups;
     const size_t q_elt = (q_dtype == FATHOM_BF16) ? 2 : 4;
     float* scores = static_cast<float*>(workspace);
@@ -83,6 +84,18 @@ cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int st
 
     cudaError_t e = launch_depths(q, q_dtype, sigma2, Hq, Hkv, d, budget, fixed_r, depths, stream);
     if (e != cudaSuccess) return e;
+    if (groups == 1) {
+        e = launch_scan(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, Hq, scores, stream, bmax,
+                        store_host != 0, true);
+        if (e == cudaSuccess)
+            e = launch_topk_blocks(scores, bmax, n, ld, Hq, k, idx, top_scores, topk_ws, stream, true);
+        if (e == cudaSuccess)
+            e = launch_attend(q, q_dtype, K_rows, V_rows, row_stride, idx, Hq, Hkv, rows_n, d, k, rows_host, out,
+                              stream, 0, nullptr, true);
+        return e;
+    }
+    Aux* aux = aux_for_device();
+    if (!aux) return cudaErrorUnknown;
     cudaError_t first = cudaSuccess;
     for (int i = 0; i < groups; ++i) {
         const int g0 = i * hkv_g, h0 = i * hq_g;
@@ -100,7 +113,7 @@ cudaError_t launch_decode(const uint32_t* planes, const uint16_t* scales, int st
         if (e == cudaSuccess) e = launch_topk_blocks(si, bi, n, ld, hq_g, k, ii, ti, topk_ws, aux->stream);
         if (e == cudaSuccess)
             e = launch_attend(qi, q_dtype, K_rows + rows_off, V_rows + rows_off, row_stride, ii, hq_g, hkv_g, rows_n,
-                              d, k, rows_host, out + (size_t)h0 * d, aux->stream);
+                              d, k, rows_host, out + (size_t)h0 * d, aux->stream, 0, nullptr, true);
         if (e != cudaSuccess) {
             first = e;
             break;

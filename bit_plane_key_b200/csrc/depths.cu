@@ -47,6 +47,7 @@ __device__ __forceinline__ uint32_t cand_key(float w, int t) {
 __global__ void __launch_bounds__(4 * kMaxD)
 depths_kernel(const void* __restrict__ q, int q_dtype, const float* __restrict__ sigma2, int Hq, int Hkv,
               int d, int budget, int fixed_r, int pooled, uint8_t* __restrict__ depths) {
+    pdl_wait();
     __shared__ int s_ties[4 * kMaxD / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.x;

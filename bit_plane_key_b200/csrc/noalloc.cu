@@ -86,7 +86,7 @@ int fathom_scan_topk_noalloc(const fathom_store* store, const void* q, int q_dty
                                 depths, n_q_heads, scores, s, bmax, store->host_resident != 0);
     if (e != cudaSuccess) return FATHOM_ECUDA;
     return to_status(launch_topk_blocks(scores, bmax, store->n, ld, n_q_heads, k, idx, top_scores,
-                                        scratch + lay.topk_off, s));
+                                        scratch + lay.topk_off, s, true));
 }
 
 }  // extern "C"

@@ -486,6 +486,7 @@ __global__ void __launch_bounds__(Geo<G>::T, Geo<G>::template min_blocks<HOST>()
 scan_kernel(const uint32_t* __restrict__ planes, const uint16_t* __restrict__ scales, int d, int64_t n,
             int64_t n_pad, const void* __restrict__ q, int q_dtype, const uint8_t* __restrict__ depths,
             float* __restrict__ scores, uint32_t* __restrict__ bmax, unsigned int* status) {
+    pdl_wait();
     const int b = (int)blockIdx.x, tiles = (int)scan_tiles(n);
     scan_head_tiles<G, HOST>(planes, scales, d, n, n_pad, b % tiles, tiles, b / tiles, q, q_dtype, depths, scores,
                              bmax, status);
@@ -497,6 +498,7 @@ __global__ void __launch_bounds__(Geo<G>::T, Geo<G>::template min_blocks<HOST>()
 scan_batched_kernel(const __grid_constant__ SessionMap map, int d, int Hq, const void* __restrict__ q, int q_dtype,
                     const uint8_t* __restrict__ depths, float* __restrict__ scores, uint32_t* __restrict__ bmax,
                     unsigned int* status) {
+    pdl_wait();
     const int t = (int)blockIdx.x;
     int lo = 0, hi = map.nsess - 1;   // last session with tile0 <= t
     while (lo < hi) {
@@ -518,7 +520,7 @@ scan_batched_kernel(const __grid_constant__ SessionMap map, int d, int Hq, const
 template <int G, bool HOST>
 cudaError_t launch_scan_g(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n,
                           int64_t n_pad, const void* q, int q_dtype, const uint8_t* depths, float* scores,
-                          uint32_t* bmax, cudaStream_t stream) {
+                          uint32_t* bmax, cudaStream_t stream, bool pdl) {
     const size_t smem = ScanSmem{d, G}.bytes();
     auto kern = scan_kernel<G, HOST>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -530,9 +532,8 @@ cudaError_t launch_scan_g(const uint32_t* planes, const uint16_t* scales, int Hk
     // too: 0.40 against 0.35 ms at n = 2^20, its CTAs ending unevenly.)
     const int64_t ctas = scan_tiles(n) * Hkv;
     if (ctas > INT32_MAX) return cudaErrorInvalidValue;
-    kern<<<(unsigned)ctas, Geo<G>::T, smem, stream>>>(planes, scales, d, n, n_pad, q, q_dtype, depths, scores, bmax,
-                                                      device_status_ptr());
-    return cudaGetLastError();
+    return launch_ex(kern, dim3((unsigned)ctas), dim3(Geo<G>::T), smem, stream, pdl, 1, planes, scales, d, n, n_pad, q,
+                     q_dtype, depths, scores, bmax, device_status_ptr());
 }
 
 template <int G, bool HOST>
@@ -550,9 +551,10 @@ cudaError_t launch_scan_batched_g(const SessionMap& map, int Hkv, int d, const v
 template <int G>
 cudaError_t launch_scan_r(bool host, const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n,
                           int64_t n_pad, const void* q, int q_dtype, const uint8_t* depths, float* scores,
-                          uint32_t* bmax, cudaStream_t stream) {
-    return host ? launch_scan_g<G, true>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream)
-                : launch_scan_g<G, false>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
+                          uint32_t* bmax, cudaStream_t stream, bool pdl) {
+    return host ? launch_scan_g<G, true>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream, pdl)
+                : launch_scan_g<G, false>(planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream,
+                                          pdl);
 }
 
 template <int G>
@@ -568,12 +570,12 @@ size_t scan_smem_bytes(int d, int G) { return ScanSmem{d, G}.bytes(); }
 
 cudaError_t launch_scan(const uint32_t* planes, const uint16_t* scales, int Hkv, int d, int64_t n, int64_t n_pad,
                         const void* q, int q_dtype, const uint8_t* depths, int Hq, float* scores,
-                        cudaStream_t stream, uint32_t* bmax, bool host) {
+                        cudaStream_t stream, uint32_t* bmax, bool host, bool pdl) {
     switch (Hq / Hkv) {
-        case 1: return launch_scan_r<1>(host, planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
-        case 2: return launch_scan_r<2>(host, planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
-        case 4: return launch_scan_r<4>(host, planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
-        case 8: return launch_scan_r<8>(host, planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream);
+        case 1: return launch_scan_r<1>(host, planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream, pdl);
+        case 2: return launch_scan_r<2>(host, planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream, pdl);
+        case 4: return launch_scan_r<4>(host, planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream, pdl);
+        case 8: return launch_scan_r<8>(host, planes, scales, Hkv, d, n, n_pad, q, q_dtype, depths, scores, bmax, stream, pdl);
         default: return cudaErrorInvalidValue;
     }
 }

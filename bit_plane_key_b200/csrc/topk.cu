@@ -381,6 +381,51 @@ __device__ void bitonic_desc(uint64_t* buf, int S) {
     }
 }
 
+// Descending bitonic sort of buf[0..S) (S a power of two, 32 <= S <=
+// blockDim.x) with one element per thread: thread e holds element e in a
+// register; stages whose partner lies in the same warp (stride < 32) exchange
+// by shuffles, the others through buf between two block barriers.  Called by
+// every thread of the block.
+__device__ void bitonic_desc_reg(uint64_t* buf, int S) {
+    const int e = threadIdx.x;
+    uint64_t v = (e < S) ? buf[e] : 0ull;
+    for (int size = 2; size <= S; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            uint64_t w;
+            if (stride >= 32) {
+                __syncthreads();
+                if (e < S) buf[e] = v;
+                __syncthreads();
+                w = (e < S) ? buf[e ^ stride] : 0ull;
+            } else {
+                const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, stride);
+                const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), stride);
+                w = ((uint64_t)hi << 32) | lo;
+            }
+            // in a descending run the lower index of a pair keeps the larger
+            const bool keep_max = ((e & stride) == 0) == ((e & size) == 0);
+            v = keep_max ? (v > w ? v : w) : (v < w ? v : w);
+        }
+    }
+    __syncthreads();
+    if (e < S) buf[e] = v;
+    __syncthreads();
+}
+
+// Number of entries of the descending list ly[0..n) greater than v: a binary
+// search whose steps depend only on n (the same for every thread that
+// searches a list of that length).
+__device__ __forceinline__ int count_above(const uint64_t* ly, int n, uint64_t v) {
+    if (n == 0) return 0;
+    const uint64_t* base = ly;
+    while (n > 1) {
+        const int half = n >> 1;
+        base = (base[half - 1] > v) ? base + half : base;
+        n -= half;
+    }
+    return (int)(base - ly) + (base[0] > v ? 1 : 0);
+}
+
 // With hist[0..nb) filled, finds the bin b holding the need-th largest key
 // (bins ordered high to low): *above = keys in bins above b, *cnt = keys in b.
 // Called by every thread of the block (a multiple of 32 threads, at most
@@ -572,6 +617,7 @@ __device__ uint32_t block_kth_key(KeyAt key_at, int64_t cnt, uint32_t need, uint
 
 __global__ void __launch_bounds__(kFinishThreads)
 topk_blk_threshold(const uint32_t* __restrict__ bmax, const __grid_constant__ RowMap m, int k, BlkWs w) {
+    pdl_wait();
     __shared__ uint32_t hist[kBins];
     __shared__ uint32_t warp_tot[32];
     __shared__ int s_bin;
@@ -606,6 +652,7 @@ topk_blk_threshold(const uint32_t* __restrict__ bmax, const __grid_constant__ Ro
 __global__ void __launch_bounds__(kPassThreads)
 topk_blk_compact(const float* __restrict__ scores, const uint32_t* __restrict__ bmax, const __grid_constant__ RowMap m,
                  BlkWs w) {
+    pdl_wait();
     const int row = blockIdx.y;
     int64_t off, n;
     row_span(m, row, &off, &n);
@@ -646,6 +693,7 @@ topk_blk_compact(const float* __restrict__ scores, const uint32_t* __restrict__ 
 __global__ void __launch_bounds__(kFinishThreads)
 topk_blk_finish(const float* __restrict__ scores, const __grid_constant__ RowMap m, int k, BlkWs w,
                 int32_t* __restrict__ idx, float* __restrict__ top_scores) {
+    pdl_wait();
     extern __shared__ uint64_t buf[];
     __shared__ uint32_t hist[kBins];
     __shared__ uint32_t warp_tot[32];
@@ -716,18 +764,31 @@ topk_blk_finish(const float* __restrict__ scores, const __grid_constant__ RowMap
 
 // ---------------------------------------------------------------------------
 // Short rows (n <= kRowsMax keys): one kernel, no workspace.  A cluster of CL
-// CTAs takes a row; CTA x holds the ordered keys of its slice of the row in
-// shared memory.  Three radix steps (12, 12 and 8 bits) each combine the CTAs'
-// histograms through distributed shared memory (cluster_pick), so every CTA
-// finds the same exact k-th key T.  Each CTA then writes its keys above T, and its keys equal
-// to T whose rank among the row's ties (CTA order, then index order) is below
-// k - #{keys > T}, into CTA 0's shared memory; CTA 0 sorts the k entries as
-// 64-bit composites (key << 32 | ~index).
+// CTAs takes a row; CTA x holds the ordered keys of its slice of the row, 32
+// per thread in registers (thread t: keys 4 (t + 512 u) .. + 3, u < 8) and a
+// copy in shared memory.  The first histogram (bits 31..20) is built while the
+// keys load.  Given the scan's 64-key block maxima and a row of at least k
+// blocks, the smallest block maximum lb bounds the k-th key from below (every
+// block holds a key >= lb), so keys below lb are left out of the histogram:
+// the bins from the top down to lb's stay exact.  The CTAs' histograms are
+// combined through distributed shared memory (cluster_pick).  When at most
+// kMaxTopK keys lie at or above max(lb, the k-th key's 12-bit bin) - the
+// usual case - those are the candidates: each CTA compacts its own (a block
+// scan of per-thread counts), sorts them, copies the other CTAs' sorted lists
+// into its shared memory, and ranks each of its candidates by binary searches
+// in them.  Otherwise two more radix steps (12 and 8 bits) find the exact k-th
+// key T; each CTA writes its keys above T, and its keys equal to T whose rank
+// among the row's ties (CTA order, then index order) is below k - #{keys > T},
+// into CTA 0's shared memory; CTA 0 sorts the k entries as 64-bit composites
+// (key << 32 | ~index).
 // ---------------------------------------------------------------------------
 constexpr int kSliceKeys = 16384;   // keys per CTA
 constexpr int kRowThreads = 512;
+constexpr int kRowVec = kSliceKeys / (4 * kRowThreads);   // 4-key groups per thread
 constexpr int kMaxCluster = 8;
 constexpr int64_t kRowsMax = (int64_t)kMaxCluster * kSliceKeys;
+// keys, histogram, candidate buffer (which also holds the cluster's range
+// sums while a pick runs): 112 KB, so two CTAs share an SM
 constexpr size_t kRowSmem = sizeof(uint32_t) * (kSliceKeys + kBins) + sizeof(uint64_t) * kMaxTopK;
 
 __device__ __forceinline__ int block_sum_int(int v, int* warp_cnt) {
@@ -741,6 +802,29 @@ __device__ __forceinline__ int block_sum_int(int v, int* warp_cnt) {
     return t;
 }
 
+// Exclusive prefix of v over the block's threads in thread order; *total gets
+// the sum.  Called by every thread.
+__device__ __forceinline__ int block_prefix_int(int v, int* warp_cnt, int* total) {
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_cnt[wp] = incl;
+    __syncthreads();
+    int before = 0, all = 0;
+    for (int x = 0; x < (int)(blockDim.x >> 5); ++x) {
+        const int c = warp_cnt[x];
+        before += (x < wp) ? c : 0;
+        all += c;
+    }
+    __syncthreads();
+    *total = all;
+    return before + incl - v;
+}
+
 template <int CL>
 __device__ __forceinline__ void cluster_barrier() {
     if constexpr (CL > 1) cg::this_cluster().sync();
@@ -750,10 +834,12 @@ __device__ __forceinline__ void cluster_barrier() {
 // With this CTA's keys added to hist[0..nb), picks the bin of the need-th
 // largest key of the whole cluster, as block_pick_bin (every CTA gets the
 // result).  The summed histogram is split: CTA x sums bins [x nb/CL,
-// (x+1) nb/CL) over the cluster and publishes their total; every CTA then
-// finds the range holding the need-th key from the totals and picks inside it
-// from that range's sums.  Each CTA reads about nb + nb/CL remote words.
-// hsum holds nb/CL words; hist is reused as scratch.
+// (x+1) nb/CL) over the cluster into hsum and publishes their total; every
+// CTA then finds the range holding the need-th key from the totals and picks
+// inside it from that range's sums.  Cluster barriers: after the first every
+// histogram is complete, after the second every range sum (hist is read by
+// other CTAs only between the two), after the third every CTA has read the
+// range it needed (hsum shares memory with the candidate buffer, written next).
 template <int CL>
 __device__ __forceinline__ void cluster_pick(uint32_t* hist, uint32_t* hsum, int nb, uint32_t need, int* s_bin,
                                              uint32_t* s_above, uint32_t* s_cnt, uint32_t* warp_tot, int* warp_cnt,
@@ -773,15 +859,17 @@ __device__ __forceinline__ void cluster_pick(uint32_t* hist, uint32_t* hsum, int
         mine = block_sum_int(mine, warp_cnt);
         if (tid == 0) *s_tot = (uint32_t)mine;
         cluster.sync();   // range sums and totals are published; nobody reads hist any more
+        uint32_t tot[CL];
+#pragma unroll
+        for (int y = 0; y < CL; ++y) tot[y] = *cluster.map_shared_rank(s_tot, y);
         uint32_t acc = 0;
         int ys = 0;
         for (int y = CL - 1; y >= 0; --y) {   // ranges from the highest bins down
-            const uint32_t t = *cluster.map_shared_rank(s_tot, y);
-            if (acc + t >= need) {
+            if (acc + tot[y] >= need) {
                 ys = y;
                 break;
             }
-            acc += t;
+            acc += tot[y];
         }
         const uint32_t* hy = cluster.map_shared_rank(hsum, ys);
         for (int j = tid; j < per; j += kRowThreads) hist[j] = hy[j];
@@ -798,67 +886,78 @@ __device__ __forceinline__ void cluster_pick(uint32_t* hist, uint32_t* hsum, int
     }
 }
 
-// The top k of a row whose candidates (keys with (key >> 20) >= b12, at most
-// kMaxTopK of them over the cluster, at least k) are known: each CTA sorts its
-// own candidates (composites, descending) in its shared buffer; the rank of a
-// candidate in the row is its position in its CTA's list plus, for every
-// other CTA, the number of that CTA's candidates above it (a binary search in
-// that CTA's sorted list through distributed shared memory); ranks below k
-// are written out.  Composites are distinct (the index is part of them), so
-// the ranks are a permutation and ties order by index.
+// The candidates of a row (its keys at or above a threshold below the k-th
+// key, at most kMaxTopK over the cluster) are sorted per CTA: buf[0..c) holds
+// this CTA's, descending, and *s_fill their count.  Each CTA copies the other
+// CTAs' lists into its own shared memory (the key slice is free by then); the
+// rank of a candidate in the row is its position in its CTA's list plus, for
+// every other CTA, the number of that CTA's candidates above it (a binary
+// search in the copy); ranks below k are written out.  Composites are
+// distinct (the index is part of them), so the ranks are a permutation and
+// ties order by index.
 template <int CL>
-__device__ void topk_rows_candidates(const uint32_t* keys, int cnt, int64_t start, uint32_t b12, int k, uint64_t* buf,
-                                     int* s_fill, int row, int32_t* __restrict__ idx,
-                                     float* __restrict__ top_scores) {
+__device__ void rank_candidates(uint32_t* keys, const uint64_t* buf, int c, int* s_fill, int row, int k,
+                                int32_t* __restrict__ idx, float* __restrict__ top_scores) {
     const int tid = threadIdx.x;
-    if (tid == 0) *s_fill = 0;
-    __syncthreads();
-    for (int e = tid; e < cnt; e += kRowThreads)
-        if ((keys[e] >> 20) >= b12) buf[atomicAdd(s_fill, 1)] = composite(keys[e], start + e);
-    __syncthreads();
-    const int c = *s_fill;
-    int S = 1;
-    while (S < c) S <<= 1;
-    for (int e = c + tid; e < S; e += kRowThreads) buf[e] = 0ull;   // below every composite of the row
-    __syncthreads();
-    if (S > 1) bitonic_desc(buf, S);
     cluster_barrier<CL>();   // every CTA's list is sorted and its count published
+    int lo_of[CL], n_of[CL];
+    uint64_t* lists = reinterpret_cast<uint64_t*>(keys);   // at most kMaxTopK composites, the slice holds kSliceKeys / 2
+    if constexpr (CL > 1) {
+        cg::cluster_group cluster = cg::this_cluster();
+        const int x = (int)cluster.block_rank();
+        int at = 0;
+#pragma unroll
+        for (int y = 0; y < CL; ++y) {
+            n_of[y] = (y == x) ? 0 : *cluster.map_shared_rank(s_fill, y);
+            lo_of[y] = at;
+            at += n_of[y];
+        }
+        // one pass over all the lists, four loads in flight per thread
+        for (int e0 = tid; e0 < at; e0 += 4 * kRowThreads) {
+            uint64_t v[4];
+            int dst[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int e = e0 + j * kRowThreads;
+                dst[j] = -1;
+                if (e < at) {
+                    int y = 0;
+#pragma unroll
+                    for (int z = 1; z < CL; ++z) y += (e >= lo_of[z]) ? 1 : 0;
+                    v[j] = cluster.map_shared_rank(buf, y)[e - lo_of[y]];
+                    dst[j] = e;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (dst[j] >= 0) lists[dst[j]] = v[j];
+        }
+        cluster_barrier<CL>();   // every CTA has its copies: no remote reads after this
+    }
     for (int j = tid; j < c; j += kRowThreads) {
         const uint64_t v = buf[j];
         int r = j;
         if constexpr (CL > 1) {
-            cg::cluster_group cluster = cg::this_cluster();
-            const int x = (int)cluster.block_rank();
 #pragma unroll
-            for (int y = 0; y < CL; ++y) {
-                if (y == x) continue;
-                const uint64_t* ly = cluster.map_shared_rank(buf, y);
-                int lo = 0, hi = *cluster.map_shared_rank(s_fill, y);   // first position below v
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (ly[mid] > v) lo = mid + 1;
-                    else hi = mid;
-                }
-                r += lo;
-            }
+            for (int y = 0; y < CL; ++y) r += count_above(lists + lo_of[y], n_of[y], v);
         }
         if (r < k) {
             idx[(int64_t)row * k + r] = (int32_t)(0xFFFFFFFFu - (uint32_t)v);
             if (top_scores) top_scores[(int64_t)row * k + r] = ordered_to_float((uint32_t)(v >> 32));
         }
     }
-    cluster_barrier<CL>();   // keep every CTA's list alive until all searches are done
 }
 
 template <int CL>
-__global__ void __launch_bounds__(kRowThreads)
-topk_rows(const float* __restrict__ scores, const __grid_constant__ RowMap m, int k, int32_t* __restrict__ idx,
-          float* __restrict__ top_scores) {
-    extern __shared__ __align__(16) unsigned char row_smem[];
-    uint32_t* keys = reinterpret_cast<uint32_t*>(row_smem);                      // [kSliceKeys]
+__global__ void __launch_bounds__(kRowThreads, 2)
+topk_rows(const float* __restrict__ scores, const uint32_t* __restrict__ bmax, const __grid_constant__ RowMap m,
+          int k, int32_t* __restrict__ idx, float* __restrict__ top_scores) {
+    pdl_wait();
+    extern __shared__ __align__(16) unsigned char row_sm[];
+    uint32_t* keys = reinterpret_cast<uint32_t*>(row_sm);                        // [kSliceKeys]
     uint32_t* hist = keys + kSliceKeys;                                           // [kBins]
-    uint64_t* buf = reinterpret_cast<uint64_t*>(hist + kBins);                    // [kMaxTopK], CTA 0
-    uint32_t* hsum = (CL > 1) ? reinterpret_cast<uint32_t*>(buf) : hist;          // cluster histogram
+    uint64_t* buf = reinterpret_cast<uint64_t*>(hist + kBins);                    // [kMaxTopK]
+    uint32_t* hsum = reinterpret_cast<uint32_t*>(buf);                            // [kBins / CL], CL > 1
     __shared__ uint32_t warp_tot[32];
     __shared__ int warp_cnt[32];
     __shared__ int s_bin, s_fill, s_gt, s_eq;
@@ -874,53 +973,105 @@ topk_rows(const float* __restrict__ scores, const __grid_constant__ RowMap m, in
     const int cnt = (int)(n - start < 0 ? 0 : (n - start < L ? n - start : L));
     const float* s = scores + off + start;
 
-    // the slice as ordered keys
-    if ((reinterpret_cast<uintptr_t>(s) & 15u) == 0) {
-        const int nv = cnt >> 2;
-        const float4* s4 = reinterpret_cast<const float4*>(s);
-        for (int v0 = tid; v0 < nv; v0 += 8 * kRowThreads) {
-            float4 x[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (v0 + u * kRowThreads < nv) x[u] = __ldg(s4 + v0 + u * kRowThreads);
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (v0 + u * kRowThreads < nv) {
-                    uint32_t* dk = keys + 4 * (v0 + u * kRowThreads);
-                    dk[0] = float_to_ordered(x[u].x);
-                    dk[1] = float_to_ordered(x[u].y);
-                    dk[2] = float_to_ordered(x[u].z);
-                    dk[3] = float_to_ordered(x[u].w);
-                }
-        }
-        for (int e = 4 * nv + tid; e < cnt; e += kRowThreads) keys[e] = float_to_ordered(s[e]);
-    } else {
-        for (int e = tid; e < cnt; e += kRowThreads) keys[e] = float_to_ordered(__ldg(s + e));
+    // the lower bound lb of the k-th key: the smallest block maximum of the
+    // row, when the row has at least k blocks (0 = no bound)
+    const int64_t nbk = (n + kBlock - 1) / kBlock;
+    const bool use_lb = bmax != nullptr && nbk >= k;
+    if (use_lb) {
+        const uint32_t* bm = bmax + off / kBlock;
+        uint32_t mn = 0xFFFFFFFFu;
+        for (int64_t b = tid; b < nbk; b += kRowThreads) mn = min(mn, __ldg(bm + b));
+        mn = __reduce_min_sync(0xffffffffu, mn);
+        if (lane == 0) warp_tot[wp] = mn;
     }
+    for (int b = tid; b < kBins; b += kRowThreads) hist[b] = 0;
     __syncthreads();
+    uint32_t lb = 0;
+    if (use_lb) {
+        lb = 0xFFFFFFFFu;
+        for (int x = 0; x < kRowThreads / 32; ++x) lb = min(lb, warp_tot[x]);
+    }
 
-    // the exact k-th largest key T of the row
+    // the slice as ordered keys in shared memory (thread t: 4-key groups
+    // t + 512 u), counted into the first histogram as they arrive
+    const bool vec = (reinterpret_cast<uintptr_t>(s) & 15u) == 0;
+#pragma unroll 4
+    for (int u = 0; u < kRowVec; ++u) {
+        const int e = 4 * (tid + kRowThreads * u);
+        uint32_t v[4];
+        if (vec && e + 3 < cnt) {
+            const float4 x = __ldg(reinterpret_cast<const float4*>(s + e));
+            v[0] = float_to_ordered(x.x);
+            v[1] = float_to_ordered(x.y);
+            v[2] = float_to_ordered(x.z);
+            v[3] = float_to_ordered(x.w);
+            *reinterpret_cast<uint4*>(keys + e) = make_uint4(v[0], v[1], v[2], v[3]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                v[c] = (e + c < cnt) ? float_to_ordered(__ldg(s + e + c)) : 0u;
+                if (e + c < cnt) keys[e + c] = v[c];
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if (e + c < cnt && v[c] >= lb) atomicAdd(&hist[v[c] >> 20], 1u);
+    }
+
+    // the exact k-th largest key T of the row (the first step's histogram is built)
     uint32_t need = (uint32_t)k, prefix = 0, above = 0;
     int shift = 32;
     while (shift > 0) {
         const int nbits = shift >= 12 ? 12 : shift, sh = shift - nbits, nb = 1 << nbits;
-        for (int b = tid; b < nb; b += kRowThreads) hist[b] = 0;
-        __syncthreads();
-        for (int e = tid; e < cnt; e += kRowThreads) {
-            const uint32_t key = keys[e];
-            if (shift == 32 || (key >> shift) == prefix) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1u);
+        if (shift != 32) {
+            for (int b = tid; b < nb; b += kRowThreads) hist[b] = 0;
+            __syncthreads();
+            for (int e = tid; e < cnt; e += kRowThreads) {
+                const uint32_t key = keys[e];
+                if ((key >> shift) == prefix) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1u);
+            }
         }
         cluster_pick<CL>(hist, hsum, nb, need, &s_bin, &s_above, &s_cnt, warp_tot, warp_cnt, &s_tot);
         need -= s_above;
         above += s_above;
         prefix = (shift == 32 ? 0u : (prefix << nbits)) | (uint32_t)s_bin;
-        const uint32_t in_bin = s_cnt;   // keys of the row in the picked bin (the same in every CTA)
+        const uint32_t in_bin = s_cnt;   // keys of the row in the picked bin (>= lb in the first step)
         shift = sh;
         __syncthreads();   // s_bin / s_above are rewritten by the next step
         if (shift == 20 && above + in_bin <= (uint32_t)kMaxTopK) {
-            // few keys at or above the k-th key's top-12-bit bin: they are the
-            // candidates, and an exact sort of them gives the top k
-            topk_rows_candidates<CL>(keys, cnt, start, prefix, k, buf, &s_fill, row, idx, top_scores);
+            // few keys at or above thr: they are the candidates, and an exact
+            // sort of them gives the top k
+            const uint32_t thr = max(lb, prefix << 20);
+            int mine = 0;
+            for (int u = 0; u < kRowVec; ++u) {
+                const int e = 4 * (tid + kRowThreads * u);
+                if (e >= cnt) break;
+                const uint4 v = *reinterpret_cast<const uint4*>(keys + e);   // past cnt: never counted
+                mine += (v.x >= thr) + (e + 1 < cnt && v.y >= thr) + (e + 2 < cnt && v.z >= thr) +
+                        (e + 3 < cnt && v.w >= thr);
+            }
+            int c_all = 0;
+            int at = block_prefix_int(mine, warp_cnt, &c_all);
+            for (int u = 0; u < kRowVec && mine > 0; ++u) {
+                const int e = 4 * (tid + kRowThreads * u);
+                if (e >= cnt) break;
+                const uint4 v = *reinterpret_cast<const uint4*>(keys + e);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (e + c < cnt && w[c] >= thr) {
+                        buf[at++] = composite(w[c], start + e + c);
+                        --mine;
+                    }
+            }
+            int S = 32;
+            while (S < c_all) S <<= 1;
+            for (int e = c_all + tid; e < S; e += kRowThreads) buf[e] = 0ull;   // below every composite of the row
+            __syncthreads();
+            if (S <= kRowThreads) bitonic_desc_reg(buf, S);
+            else bitonic_desc(buf, S);
+            if (tid == 0) s_fill = c_all;
+            rank_candidates<CL>(keys, buf, c_all, &s_fill, row, k, idx, top_scores);
             return;
         }
     }
@@ -997,36 +1148,26 @@ topk_rows(const float* __restrict__ scores, const __grid_constant__ RowMap m, in
 }
 
 template <int CL>
-cudaError_t launch_topk_rows_cl(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
-                                float* top_scores, cudaStream_t stream) {
+cudaError_t launch_topk_rows_cl(const float* scores, const uint32_t* bmax, const RowMap& map, int rows, int k,
+                                int32_t* idx, float* top_scores, cudaStream_t stream, bool pdl) {
     auto kern = topk_rows<CL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRowSmem);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(rows * CL));
-    cfg.blockDim = dim3(kRowThreads);
-    cfg.dynamicSmemBytes = kRowSmem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CL;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = CL > 1 ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, scores, map, k, idx, top_scores);
+    return launch_ex(kern, dim3((unsigned)(rows * CL)), dim3(kRowThreads), kRowSmem, stream, pdl, CL, scores, bmax,
+                     map, k, idx, top_scores);
 }
 
-// rows of at most kRowsMax keys and k <= kMaxTopK
-cudaError_t launch_topk_rows(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
-                             float* top_scores, cudaStream_t stream) {
+// rows of at most kRowsMax keys and k <= kMaxTopK; bmax: the rows' block
+// maxima, or null
+cudaError_t launch_topk_rows(const float* scores, const uint32_t* bmax, const RowMap& map, int rows, int k,
+                             int32_t* idx, float* top_scores, cudaStream_t stream, bool pdl = false) {
     int cl = 1;
     while ((int64_t)cl * kSliceKeys < map.max_n) cl <<= 1;
     switch (cl) {
-        case 1: return launch_topk_rows_cl<1>(scores, map, rows, k, idx, top_scores, stream);
-        case 2: return launch_topk_rows_cl<2>(scores, map, rows, k, idx, top_scores, stream);
-        case 4: return launch_topk_rows_cl<4>(scores, map, rows, k, idx, top_scores, stream);
-        case 8: return launch_topk_rows_cl<8>(scores, map, rows, k, idx, top_scores, stream);
+        case 1: return launch_topk_rows_cl<1>(scores, bmax, map, rows, k, idx, top_scores, stream, pdl);
+        case 2: return launch_topk_rows_cl<2>(scores, bmax, map, rows, k, idx, top_scores, stream, pdl);
+        case 4: return launch_topk_rows_cl<4>(scores, bmax, map, rows, k, idx, top_scores, stream, pdl);
+        case 8: return launch_topk_rows_cl<8>(scores, bmax, map, rows, k, idx, top_scores, stream, pdl);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -1056,28 +1197,33 @@ size_t topk_blocks_workspace_bytes(int rows) {
 }
 
 cudaError_t launch_topk_blocks_map(const float* scores, const uint32_t* bmax, const RowMap& map, int rows, int k,
-                                   int32_t* idx, float* top_scores, void* ws, cudaStream_t stream) {
+                                   int32_t* idx, float* top_scores, void* ws, cudaStream_t stream, bool pdl) {
     // The bound m is tight only when a row has many more blocks than k: with
     // at least 8k blocks, m lies in the top eighth of the block maxima and the
     // surviving blocks hold about k candidates.  Shorter rows take the
     // histogram path over the whole row.
+    if (map.max_n <= kRowsMax && k <= kMaxTopK)
+        return launch_topk_rows(scores, bmax, map, rows, k, idx, top_scores, stream, pdl);
     int64_t min_n = map.max_n;
     for (int s = 0; s < map.nsets; ++s) min_n = map.n[s] < min_n ? map.n[s] : min_n;
     if (min_n / kBlock < 8 * (int64_t)k) return launch_topk_map(scores, map, rows, k, idx, top_scores, ws, stream);
     BlkWs w = carve_blk(ws, rows);
-    topk_blk_threshold<<<rows, kFinishThreads, 0, stream>>>(bmax, map, k, w);
-    const int64_t nbk = (map.max_n + kBlock - 1) / kBlock;
-    topk_blk_compact<<<dim3((unsigned)((nbk + kPassThreads - 1) / kPassThreads), rows), kPassThreads, 0, stream>>>(
-        scores, bmax, map, w);
     const size_t smem = sizeof(uint64_t) * kSortMax;
     cudaError_t e = cudaFuncSetAttribute(topk_blk_finish, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    topk_blk_finish<<<rows, kFinishThreads, smem, stream>>>(scores, map, k, w, idx, top_scores);
-    return cudaGetLastError();
+    // the second and third launches follow the path's own kernels
+    e = launch_ex(topk_blk_threshold, dim3((unsigned)rows), dim3(kFinishThreads), 0, stream, pdl, 1, bmax, map, k, w);
+    if (e != cudaSuccess) return e;
+    const int64_t nbk = (map.max_n + kBlock - 1) / kBlock;
+    e = launch_ex(topk_blk_compact, dim3((unsigned)((nbk + kPassThreads - 1) / kPassThreads), (unsigned)rows),
+                  dim3(kPassThreads), 0, stream, true, 1, scores, bmax, map, w);
+    if (e != cudaSuccess) return e;
+    return launch_ex(topk_blk_finish, dim3((unsigned)rows), dim3(kFinishThreads), smem, stream, true, 1, scores, map, k,
+                     w, idx, top_scores);
 }
 
 cudaError_t launch_topk_blocks(const float* scores, const uint32_t* bmax, int64_t n, int64_t ld, int rows, int k,
-                               int32_t* idx, float* top_scores, void* ws, cudaStream_t stream) {
+                               int32_t* idx, float* top_scores, void* ws, cudaStream_t stream, bool pdl) {
     RowMap m;
     m.rows_per_set = rows;
     m.nsets = 1;
@@ -1085,7 +1231,7 @@ cudaError_t launch_topk_blocks(const float* scores, const uint32_t* bmax, int64_
     m.base[0] = 0;
     m.ld[0] = ld;
     m.n[0] = n;
-    return launch_topk_blocks_map(scores, bmax, m, rows, k, idx, top_scores, ws, stream);
+    return launch_topk_blocks_map(scores, bmax, m, rows, k, idx, top_scores, ws, stream, pdl);
 }
 
 size_t topk_workspace_bytes(int64_t n, int rows, int k) {
@@ -1097,7 +1243,8 @@ size_t topk_workspace_bytes(int64_t n, int rows, int k) {
 
 cudaError_t launch_topk_map(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
                             float* top_scores, void* ws, cudaStream_t stream) {
-    if (map.max_n <= kRowsMax && k <= kMaxTopK) return launch_topk_rows(scores, map, rows, k, idx, top_scores, stream);
+    if (map.max_n <= kRowsMax && k <= kMaxTopK)
+        return launch_topk_rows(scores, nullptr, map, rows, k, idx, top_scores, stream);
     Workspace w = carve(ws, rows, k);
     unsigned int* status = device_status_ptr();
     const unsigned chunks = (unsigned)((map.max_n + kChunk - 1) / kChunk);

@@ -22,8 +22,8 @@
  *   - The caller owns all memory it passes; no call allocates device
  *     memory for it.  The library keeps this state of its own, per device:
  *       . one status word (see below), a __device__ variable;
- *       . for fathom_decode_step, one auxiliary stream and 65 events, made on
- *         the first call in a context;
+ *       . for fathom_decode_step with kv_groups > 1, one auxiliary stream
+ *         and 65 events, made on the first such call in a context;
  *       . for fathom_scan_topk_noalloc, a fixed scratch array of
  *         fathom_noalloc_scratch_bytes(), a __device__ variable that every GPU
  *         which loads the library holds until the process exits.
@@ -378,9 +378,11 @@ int fathom_attend_merge(const float* parts, int world, int n_q_heads, int d, flo
  * run on an auxiliary stream that the library creates per device on first
  * use; the two are forked and joined with events, so all work is ordered on
  * `stream` and the call may be captured into a CUDA graph.  kv_groups = 1
- * runs the plain sequence.  Steps issued at the same time from several host
- * threads on one device share the auxiliary stream (they stay correct; their
- * top-k and attention serialise).
+ * runs the plain sequence on `stream` alone, each kernel launched with
+ * programmatic serialization (scheduled while the one before it finishes; it
+ * waits for that kernel's results before reading them).  Steps issued at the
+ * same time from several host threads on one device share the auxiliary
+ * stream (they stay correct; their top-k and attention serialise).
  *   store        device- or host-resident store, as fathom_scan_topk.
  *   q, q_dtype, sigma2, budget_bits, fixed_r  as fathom_alloc_depths.
  *   k            as fathom_scan_topk (1 <= k <= min(n, 4096)).

@@ -297,7 +297,8 @@ def test_topk_bit_exact(ref, n, rows, k, kind):
 
 
 @pytest.mark.parametrize("n,B,k", [(20000, 92, 2048), (5000, 46, 700), (70000, 0, 1024), (131072, 136, 4096),
-                                    (3000, 92, 3000)])
+                                    (3000, 92, 3000), (131072, 92, 2048), (100000, 68, 1500), (4096, 92, 64),
+                                    (65536, 46, 512)])
 def test_topk_from_block_maxima_equals_full_selection(n, B, k):
     """The scan's block maxima let top-k read only the blocks that can hold a
     selected key; the result must equal the selection over the whole rows bit
@@ -315,6 +316,54 @@ def test_topk_from_block_maxima_equals_full_selection(n, B, k):
     assert torch.equal(i_st, i_all) and torch.equal(t_st, t_all)
     if B == 0:
         assert np.array_equal(host(i_blk), np.tile(np.arange(k, dtype=np.int32), (8, 1)))
+    assert F.last_device_status() == 0
+
+
+def _ordered_keys(s):
+    """Order-preserving u32 keys of fp32 scores (the block-maximum format)."""
+    u = np.ascontiguousarray(s, dtype=np.float32).view(np.uint32).copy()
+    u[u == 0x80000000] = 0
+    neg = (u & 0x80000000) != 0
+    return np.where(neg, ~u, u | np.uint32(0x80000000)).astype(np.uint32)
+
+
+@pytest.mark.parametrize("case", ["ties_at_bound", "k_equals_blocks", "top_in_one_block", "ragged_tail"])
+def test_topk_block_maxima_bound_edge_cases(ref, case):
+    """Short rows with at least k blocks: keys below the smallest block maximum
+    are left out of the first histogram.  Scores built so that the k-th key is
+    that bound itself (all selected keys tie at it), sits just above it, or
+    comes from one block; checked against the oracle bit for bit."""
+    rng = np.random.default_rng(11)
+    rows, n = 2, 131072
+    if case == "ragged_tail":
+        n = 100003
+    nbk = -(-n // 64)
+    s = rng.uniform(-1.0, 1.0, (rows, n)).astype(np.float32)
+    if case == "ties_at_bound":
+        k = nbk
+        s[:, ::64] = 5.0                     # every block's maximum is 5.0: the top k all tie there
+    elif case == "k_equals_blocks":
+        k = nbk
+        s[:, ::64] = rng.uniform(2.0, 3.0, (rows, nbk)).astype(np.float32)
+    elif case == "top_in_one_block":
+        k = 1000
+        s[:, 64:128] = 10.0 + np.arange(64, dtype=np.float32)
+    else:
+        k = 1563
+        s[:, -3:] = 7.0                      # the partial last block holds the largest keys
+    ld = ((n + 1023) // 1024) * 1024
+    sd = torch.full((rows, ld), float("-inf"), device=DEV)
+    sd[:, :n] = dev(s)
+    pad = np.full((rows, nbk * 64), -np.inf, np.float32)
+    pad[:, :n] = s
+    bm = np.zeros((rows, ld // 64), np.uint32)
+    bm[:, :nbk] = _ordered_keys(pad.reshape(rows, nbk, 64).max(axis=2))
+    idx, top = F.topk(sd, n, k, block_max=dev(bm))
+    idx, top = host(idx), host(top)
+    for r in range(rows):
+        want = ref.topk(s[r], k)
+        assert np.array_equal(idx[r], want), (case, r)
+        assert np.array_equal(top[r], s[r][want])
     assert F.last_device_status() == 0
 
 
