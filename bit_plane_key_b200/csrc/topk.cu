@@ -384,12 +384,16 @@ __device__ void bitonic_desc(uint64_t* buf, int S) {
 // Descending bitonic sort of buf[0..S) (S a power of two, 32 <= S <=
 // blockDim.x) with one element per thread: thread e holds element e in a
 // register; stages whose partner lies in the same warp (stride < 32) exchange
-// by shuffles, the others through buf between two block barriers.  Called by
-// every thread of the block.
-__device__ void bitonic_desc_reg(uint64_t* buf, int S) {
+// by shuffles, the others through buf between two block barriers.  S is a
+// template argument, so every stage is unrolled with its size and stride
+// fixed.  Called by every thread of the block.
+template <int S>
+__device__ __forceinline__ void bitonic_desc_reg_t(uint64_t* buf) {
     const int e = threadIdx.x;
     uint64_t v = (e < S) ? buf[e] : 0ull;
+#pragma unroll
     for (int size = 2; size <= S; size <<= 1) {
+#pragma unroll
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
             uint64_t w;
             if (stride >= 32) {
@@ -403,8 +407,9 @@ __device__ void bitonic_desc_reg(uint64_t* buf, int S) {
                 w = ((uint64_t)hi << 32) | lo;
             }
             // in a descending run the lower index of a pair keeps the larger
-            const bool keep_max = ((e & stride) == 0) == ((e & size) == 0);
-            v = keep_max ? (v > w ? v : w) : (v < w ? v : w);
+            const bool keep_max = (((e & stride) != 0) == ((e & size) != 0));
+            const bool gt = v > w;
+            v = (keep_max == gt) ? v : w;
         }
     }
     __syncthreads();
@@ -412,18 +417,32 @@ __device__ void bitonic_desc_reg(uint64_t* buf, int S) {
     __syncthreads();
 }
 
+// bitonic_desc_reg_t for a run-time S in [32, 512]
+__device__ void bitonic_desc_reg(uint64_t* buf, int S) {
+    switch (S) {
+        case 32: bitonic_desc_reg_t<32>(buf); break;
+        case 64: bitonic_desc_reg_t<64>(buf); break;
+        case 128: bitonic_desc_reg_t<128>(buf); break;
+        case 256: bitonic_desc_reg_t<256>(buf); break;
+        default: bitonic_desc_reg_t<512>(buf); break;
+    }
+}
+
 // Number of entries of the descending list ly[0..n) greater than v: a binary
 // search whose steps depend only on n (the same for every thread that
 // searches a list of that length).
 __device__ __forceinline__ int count_above(const uint64_t* ly, int n, uint64_t v) {
     if (n == 0) return 0;
-    const uint64_t* base = ly;
-    while (n > 1) {
-        const int half = n >> 1;
-        base = (base[half - 1] > v) ? base + half : base;
-        n -= half;
+    int base = 0;
+#pragma unroll
+    for (int it = 0; it < 13; ++it) {   // n <= kMaxTopK = 2^12: at most 12 halvings
+        if (n > 1) {
+            const int half = n >> 1;
+            base += (ly[base + half - 1] > v) ? half : 0;
+            n -= half;
+        }
     }
-    return (int)(base - ly) + (base[0] > v ? 1 : 0);
+    return base + (ly[base] > v ? 1 : 0);
 }
 
 // With hist[0..nb) filled, finds the bin b holding the need-th largest key
@@ -764,16 +783,12 @@ topk_blk_finish(const float* __restrict__ scores, const __grid_constant__ RowMap
 
 // ---------------------------------------------------------------------------
 // Short rows (n <= kRowsMax keys): one kernel, no workspace.  A cluster of CL
-// CTAs takes a row; CTA x holds the ordered keys of its slice of the row, 32
-// per thread in registers (thread t: keys 4 (t + 512 u) .. + 3, u < 8) and a
-// copy in shared memory.  The first histogram (bits 31..20) is built while the
-// keys load.  Given the scan's 64-key block maxima and a row of at least k
-// blocks, the smallest block maximum lb bounds the k-th key from below (every
-// block holds a key >= lb), so keys below lb are left out of the histogram:
-// the bins from the top down to lb's stay exact.  The CTAs' histograms are
-// combined through distributed shared memory (cluster_pick).  When at most
-// kMaxTopK keys lie at or above max(lb, the k-th key's 12-bit bin) - the
-// usual case - those are the candidates: each CTA compacts its own (a block
+// CTAs takes a row; CTA x holds the ordered keys of its slice of the row
+// in shared memory (thread t: keys 4 (t + 512 u) .. + 3, u < 8).  The first
+// histogram (bits 31..20) is built while the keys load.  The CTAs' histograms
+// are combined through distributed shared memory (cluster_pick).  When at
+// most kMaxTopK keys lie at or above the k-th key's 12-bit bin - the usual
+// case - those are the candidates: each CTA compacts its own (a block
 // scan of per-thread counts), sorts them, copies the other CTAs' sorted lists
 // into its shared memory, and ranks each of its candidates by binary searches
 // in them.  Otherwise two more radix steps (12 and 8 bits) find the exact k-th
@@ -912,25 +927,20 @@ __device__ void rank_candidates(uint32_t* keys, const uint64_t* buf, int c, int*
             lo_of[y] = at;
             at += n_of[y];
         }
-        // one pass over all the lists, four loads in flight per thread
-        for (int e0 = tid; e0 < at; e0 += 4 * kRowThreads) {
-            uint64_t v[4];
-            int dst[4];
+        // the lists in rounds of kRowThreads entries, each round's remote
+        // loads all issued before its stores
+        int most = 0;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int e = e0 + j * kRowThreads;
-                dst[j] = -1;
-                if (e < at) {
-                    int y = 0;
+        for (int y = 0; y < CL; ++y) most = max(most, n_of[y]);
+        for (int base = 0; base < most; base += kRowThreads) {
+            const int e = base + tid;
+            uint64_t v[CL];
 #pragma unroll
-                    for (int z = 1; z < CL; ++z) y += (e >= lo_of[z]) ? 1 : 0;
-                    v[j] = cluster.map_shared_rank(buf, y)[e - lo_of[y]];
-                    dst[j] = e;
-                }
-            }
+            for (int y = 0; y < CL; ++y)
+                if (e < n_of[y]) v[y] = cluster.map_shared_rank(buf, y)[e];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (dst[j] >= 0) lists[dst[j]] = v[j];
+            for (int y = 0; y < CL; ++y)
+                if (e < n_of[y]) lists[lo_of[y] + e] = v[y];
         }
         cluster_barrier<CL>();   // every CTA has its copies: no remote reads after this
     }
@@ -950,8 +960,8 @@ __device__ void rank_candidates(uint32_t* keys, const uint64_t* buf, int c, int*
 
 template <int CL>
 __global__ void __launch_bounds__(kRowThreads, 2)
-topk_rows(const float* __restrict__ scores, const uint32_t* __restrict__ bmax, const __grid_constant__ RowMap m,
-          int k, int32_t* __restrict__ idx, float* __restrict__ top_scores) {
+topk_rows(const float* __restrict__ scores, const __grid_constant__ RowMap m, int k, int32_t* __restrict__ idx,
+          float* __restrict__ top_scores) {
     pdl_wait();
     extern __shared__ __align__(16) unsigned char row_sm[];
     uint32_t* keys = reinterpret_cast<uint32_t*>(row_sm);                        // [kSliceKeys]
@@ -973,49 +983,49 @@ topk_rows(const float* __restrict__ scores, const uint32_t* __restrict__ bmax, c
     const int cnt = (int)(n - start < 0 ? 0 : (n - start < L ? n - start : L));
     const float* s = scores + off + start;
 
-    // the lower bound lb of the k-th key: the smallest block maximum of the
-    // row, when the row has at least k blocks (0 = no bound)
-    const int64_t nbk = (n + kBlock - 1) / kBlock;
-    const bool use_lb = bmax != nullptr && nbk >= k;
-    if (use_lb) {
-        const uint32_t* bm = bmax + off / kBlock;
-        uint32_t mn = 0xFFFFFFFFu;
-        for (int64_t b = tid; b < nbk; b += kRowThreads) mn = min(mn, __ldg(bm + b));
-        mn = __reduce_min_sync(0xffffffffu, mn);
-        if (lane == 0) warp_tot[wp] = mn;
-    }
     for (int b = tid; b < kBins; b += kRowThreads) hist[b] = 0;
     __syncthreads();
-    uint32_t lb = 0;
-    if (use_lb) {
-        lb = 0xFFFFFFFFu;
-        for (int x = 0; x < kRowThreads / 32; ++x) lb = min(lb, warp_tot[x]);
-    }
 
     // the slice as ordered keys in shared memory (thread t: 4-key groups
     // t + 512 u), counted into the first histogram as they arrive
     const bool vec = (reinterpret_cast<uintptr_t>(s) & 15u) == 0;
+    // a whole aligned slice (every CTA of a 131072-key row) takes the loop
+    // without bounds checks
+    const bool full = vec && cnt == kSliceKeys;
+    if (full) {
 #pragma unroll 4
-    for (int u = 0; u < kRowVec; ++u) {
-        const int e = 4 * (tid + kRowThreads * u);
-        uint32_t v[4];
-        if (vec && e + 3 < cnt) {
+        for (int u = 0; u < kRowVec; ++u) {
+            const int e = 4 * (tid + kRowThreads * u);
             const float4 x = __ldg(reinterpret_cast<const float4*>(s + e));
-            v[0] = float_to_ordered(x.x);
-            v[1] = float_to_ordered(x.y);
-            v[2] = float_to_ordered(x.z);
-            v[3] = float_to_ordered(x.w);
+            const uint32_t v[4] = {float_to_ordered(x.x), float_to_ordered(x.y), float_to_ordered(x.z),
+                                   float_to_ordered(x.w)};
             *reinterpret_cast<uint4*>(keys + e) = make_uint4(v[0], v[1], v[2], v[3]);
-        } else {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                v[c] = (e + c < cnt) ? float_to_ordered(__ldg(s + e + c)) : 0u;
-                if (e + c < cnt) keys[e + c] = v[c];
-            }
+            for (int c = 0; c < 4; ++c) atomicAdd(&hist[v[c] >> 20], 1u);
         }
+    } else {
+#pragma unroll 4
+        for (int u = 0; u < kRowVec; ++u) {
+            const int e = 4 * (tid + kRowThreads * u);
+            uint32_t v[4];
+            if (vec && e + 3 < cnt) {
+                const float4 x = __ldg(reinterpret_cast<const float4*>(s + e));
+                v[0] = float_to_ordered(x.x);
+                v[1] = float_to_ordered(x.y);
+                v[2] = float_to_ordered(x.z);
+                v[3] = float_to_ordered(x.w);
+                *reinterpret_cast<uint4*>(keys + e) = make_uint4(v[0], v[1], v[2], v[3]);
+            } else {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-            if (e + c < cnt && v[c] >= lb) atomicAdd(&hist[v[c] >> 20], 1u);
+                for (int c = 0; c < 4; ++c) {
+                    v[c] = (e + c < cnt) ? float_to_ordered(__ldg(s + e + c)) : 0u;
+                    if (e + c < cnt) keys[e + c] = v[c];
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (e + c < cnt) atomicAdd(&hist[v[c] >> 20], 1u);
+        }
     }
 
     // the exact k-th largest key T of the row (the first step's histogram is built)
@@ -1035,20 +1045,28 @@ topk_rows(const float* __restrict__ scores, const uint32_t* __restrict__ bmax, c
         need -= s_above;
         above += s_above;
         prefix = (shift == 32 ? 0u : (prefix << nbits)) | (uint32_t)s_bin;
-        const uint32_t in_bin = s_cnt;   // keys of the row in the picked bin (>= lb in the first step)
+        const uint32_t in_bin = s_cnt;   // keys of the row in the picked bin
         shift = sh;
         __syncthreads();   // s_bin / s_above are rewritten by the next step
         if (shift == 20 && above + in_bin <= (uint32_t)kMaxTopK) {
             // few keys at or above thr: they are the candidates, and an exact
             // sort of them gives the top k
-            const uint32_t thr = max(lb, prefix << 20);
+            const uint32_t thr = prefix << 20;
             int mine = 0;
-            for (int u = 0; u < kRowVec; ++u) {
-                const int e = 4 * (tid + kRowThreads * u);
-                if (e >= cnt) break;
-                const uint4 v = *reinterpret_cast<const uint4*>(keys + e);   // past cnt: never counted
-                mine += (v.x >= thr) + (e + 1 < cnt && v.y >= thr) + (e + 2 < cnt && v.z >= thr) +
-                        (e + 3 < cnt && v.w >= thr);
+            if (full) {
+#pragma unroll
+                for (int u = 0; u < kRowVec; ++u) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(keys + 4 * (tid + kRowThreads * u));
+                    mine += (v.x >= thr) + (v.y >= thr) + (v.z >= thr) + (v.w >= thr);
+                }
+            } else {
+                for (int u = 0; u < kRowVec; ++u) {
+                    const int e = 4 * (tid + kRowThreads * u);
+                    if (e >= cnt) break;
+                    const uint4 v = *reinterpret_cast<const uint4*>(keys + e);   // past cnt: never counted
+                    mine += (v.x >= thr) + (e + 1 < cnt && v.y >= thr) + (e + 2 < cnt && v.z >= thr) +
+                            (e + 3 < cnt && v.w >= thr);
+                }
             }
             int c_all = 0;
             int at = block_prefix_int(mine, warp_cnt, &c_all);
@@ -1148,26 +1166,25 @@ topk_rows(const float* __restrict__ scores, const uint32_t* __restrict__ bmax, c
 }
 
 template <int CL>
-cudaError_t launch_topk_rows_cl(const float* scores, const uint32_t* bmax, const RowMap& map, int rows, int k,
-                                int32_t* idx, float* top_scores, cudaStream_t stream, bool pdl) {
+cudaError_t launch_topk_rows_cl(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
+                                float* top_scores, cudaStream_t stream, bool pdl) {
     auto kern = topk_rows<CL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRowSmem);
     if (e != cudaSuccess) return e;
-    return launch_ex(kern, dim3((unsigned)(rows * CL)), dim3(kRowThreads), kRowSmem, stream, pdl, CL, scores, bmax,
-                     map, k, idx, top_scores);
+    return launch_ex(kern, dim3((unsigned)(rows * CL)), dim3(kRowThreads), kRowSmem, stream, pdl, CL, scores, map, k,
+                     idx, top_scores);
 }
 
-// rows of at most kRowsMax keys and k <= kMaxTopK; bmax: the rows' block
-// maxima, or null
-cudaError_t launch_topk_rows(const float* scores, const uint32_t* bmax, const RowMap& map, int rows, int k,
-                             int32_t* idx, float* top_scores, cudaStream_t stream, bool pdl = false) {
+// rows of at most kRowsMax keys and k <= kMaxTopK
+cudaError_t launch_topk_rows(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
+                             float* top_scores, cudaStream_t stream, bool pdl = false) {
     int cl = 1;
     while ((int64_t)cl * kSliceKeys < map.max_n) cl <<= 1;
     switch (cl) {
-        case 1: return launch_topk_rows_cl<1>(scores, bmax, map, rows, k, idx, top_scores, stream, pdl);
-        case 2: return launch_topk_rows_cl<2>(scores, bmax, map, rows, k, idx, top_scores, stream, pdl);
-        case 4: return launch_topk_rows_cl<4>(scores, bmax, map, rows, k, idx, top_scores, stream, pdl);
-        case 8: return launch_topk_rows_cl<8>(scores, bmax, map, rows, k, idx, top_scores, stream, pdl);
+        case 1: return launch_topk_rows_cl<1>(scores, map, rows, k, idx, top_scores, stream, pdl);
+        case 2: return launch_topk_rows_cl<2>(scores, map, rows, k, idx, top_scores, stream, pdl);
+        case 4: return launch_topk_rows_cl<4>(scores, map, rows, k, idx, top_scores, stream, pdl);
+        case 8: return launch_topk_rows_cl<8>(scores, map, rows, k, idx, top_scores, stream, pdl);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -1203,7 +1220,7 @@ cudaError_t launch_topk_blocks_map(const float* scores, const uint32_t* bmax, co
     // surviving blocks hold about k candidates.  Shorter rows take the
     // histogram path over the whole row.
     if (map.max_n <= kRowsMax && k <= kMaxTopK)
-        return launch_topk_rows(scores, bmax, map, rows, k, idx, top_scores, stream, pdl);
+        return launch_topk_rows(scores, map, rows, k, idx, top_scores, stream, pdl);
     int64_t min_n = map.max_n;
     for (int s = 0; s < map.nsets; ++s) min_n = map.n[s] < min_n ? map.n[s] : min_n;
     if (min_n / kBlock < 8 * (int64_t)k) return launch_topk_map(scores, map, rows, k, idx, top_scores, ws, stream);
@@ -1244,7 +1261,7 @@ size_t topk_workspace_bytes(int64_t n, int rows, int k) {
 cudaError_t launch_topk_map(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
                             float* top_scores, void* ws, cudaStream_t stream) {
     if (map.max_n <= kRowsMax && k <= kMaxTopK)
-        return launch_topk_rows(scores, nullptr, map, rows, k, idx, top_scores, stream);
+        return launch_topk_rows(scores, map, rows, k, idx, top_scores, stream);
     Workspace w = carve(ws, rows, k);
     unsigned int* status = device_status_ptr();
     const unsigned chunks = (unsigned)((map.max_n + kChunk - 1) / kChunk);
