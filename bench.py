@@ -303,16 +303,18 @@ class Layer:
 def topk_launches(n, k, n_max=None):
     """Launches of one top-k call after the scan (the path fathom_scan_topk
     takes) on rows of n keys (the shortest row, for ragged batches; n_max the
-    longest): rows with at least 8k blocks of 64 keys take the block-maxima
-    path (threshold, compaction, final sort); rows of at most 131072 keys one
-    cluster kernel; other rows the histogram path (init, level-0 histogram and
-    select, two refine levels of histogram and select, compaction, final
-    sort)."""
+    longest): rows of at most 131072 keys, and longer rows of at least k and at
+    most 2^17 blocks of 64 keys, one cluster kernel; rows of at least 8k blocks
+    beyond that the block-maxima path (threshold, compaction, final sort);
+    other rows the histogram path (init, level-0 histogram and select, two
+    refine levels of histogram and select, compaction, final sort)."""
     n_max = n if n_max is None else n_max
-    if n // 64 >= 8 * k:
-        return 3
     if n_max <= 131072:
         return 1
+    if k <= 4096 and -(-n // 64) >= k and -(-n_max // 64) <= 1 << 17:
+        return 1
+    if n // 64 >= 8 * k:
+        return 3
     return 9
 
 

@@ -1175,6 +1175,258 @@ cudaError_t launch_topk_rows_cl(const float* scores, const RowMap& map, int rows
                      idx, top_scores);
 }
 
+// ---------------------------------------------------------------------------
+// Long rows with block maxima (at least k blocks of 64 keys, at most
+// kMaxCluster * kSliceKeys blocks): one cluster kernel, no workspace.  A
+// cluster of CL CTAs takes a row; CTA x holds the block maxima of its share of
+// the row's blocks in shared memory.  Two radix steps over the maxima (12 and
+// 12 bits, combined through distributed shared memory) give thr = the lower
+// edge of the 24-bit bin of the k-th largest block maximum m.  Every block
+// holds its maximum, so at least k keys are >= m >= thr, the row's k-th key is
+// >= thr, and every key at or above it lies in a block whose maximum is >= thr:
+// the keys >= thr of those blocks are the candidates (about k of them).  Each
+// CTA reads its surviving blocks' scores, keeps the candidates, sorts them and
+// ranks them across the cluster as the short-row kernel does.  A row with more
+// than kMaxTopK candidates (many keys tied near the threshold) is selected
+// exactly from all its keys instead (exact_topk_cluster).
+// ---------------------------------------------------------------------------
+struct RowShared {
+    uint32_t warp_tot[32];
+    int warp_cnt[32];
+    int bin, fill, gt, eq;
+    uint32_t above, cnt, tot;
+};
+
+// The exact top k of a row whose keys key_at(0..cnt) (global indices start +
+// e) are split over the CL CTAs of a cluster, with no bound on the ties:
+// radix steps (12, 12 and 8 bits) find the k-th largest key T; keys above T
+// and the first ties at T (CTA order, then index order) go to CTA 0's buffer,
+// which sorts the k entries as composites and writes them.  hist (kBins
+// words) and buf (kMaxTopK composites; also the range sums) are this CTA's.
+template <int CL, class KeyAt>
+__device__ void exact_topk_cluster(KeyAt key_at, int cnt, int64_t start, int k, uint32_t* hist, uint64_t* buf,
+                                   RowShared* sh, int row, int32_t* __restrict__ idx,
+                                   float* __restrict__ top_scores) {
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    int rank = 0;
+    if constexpr (CL > 1) rank = (int)cg::this_cluster().block_rank();
+    uint32_t* hsum = reinterpret_cast<uint32_t*>(buf);
+    uint32_t need = (uint32_t)k, prefix = 0, above = 0;
+    for (int shift = 32; shift > 0;) {
+        const int nbits = shift >= 12 ? 12 : shift, sh_ = shift - nbits, nb = 1 << nbits;
+        cluster_barrier<CL>();   // nobody reads this CTA's histogram or range sums any more
+        for (int b = tid; b < nb; b += kRowThreads) hist[b] = 0;
+        __syncthreads();
+        for (int e = tid; e < cnt; e += kRowThreads) {
+            const uint32_t key = key_at(e);
+            if (shift == 32 || (key >> shift) == prefix) atomicAdd(&hist[(key >> sh_) & (nb - 1)], 1u);
+        }
+        cluster_pick<CL>(hist, hsum, nb, need, &sh->bin, &sh->above, &sh->cnt, sh->warp_tot, sh->warp_cnt, &sh->tot);
+        need -= sh->above;
+        above += sh->above;
+        prefix = (shift == 32 ? 0u : (prefix << nbits)) | (uint32_t)sh->bin;
+        shift = sh_;
+        __syncthreads();   // bin / above are rewritten by the next step
+    }
+    const uint32_t T = prefix;
+    const int gt_row = (int)above, take_eq = k - gt_row;   // keys above T; ties to take (>= 1)
+    int my_gt = 0, my_eq = 0;
+    for (int e = tid; e < cnt; e += kRowThreads) {
+        const uint32_t key = key_at(e);
+        my_gt += key > T;
+        my_eq += key == T;
+    }
+    my_gt = block_sum_int(my_gt, sh->warp_cnt);
+    my_eq = block_sum_int(my_eq, sh->warp_cnt);
+    if (tid == 0) {
+        sh->gt = my_gt;
+        sh->eq = my_eq;
+        sh->fill = 0;
+    }
+    cluster_barrier<CL>();
+    int gt_before = 0, eq_before = 0;
+    uint64_t* dst = buf;
+    if constexpr (CL > 1) {
+        cg::cluster_group cluster = cg::this_cluster();
+        for (int x = 0; x < rank; ++x) {
+            gt_before += cluster.map_shared_rank(sh, x)->gt;
+            eq_before += cluster.map_shared_rank(sh, x)->eq;
+        }
+        dst = cluster.map_shared_rank(buf, 0);
+    }
+    for (int e = tid; e < cnt; e += kRowThreads) {
+        const uint32_t key = key_at(e);
+        if (key > T) dst[gt_before + atomicAdd(&sh->fill, 1)] = composite(key, start + e);
+    }
+    if (my_eq > 0 && eq_before < take_eq) {
+        if (eq_before + my_eq <= take_eq) {   // all of this CTA's ties are taken: any order
+            __syncthreads();
+            if (tid == 0) sh->fill = 0;
+            __syncthreads();
+            for (int e = tid; e < cnt; e += kRowThreads)
+                if (key_at(e) == T) dst[gt_row + eq_before + atomicAdd(&sh->fill, 1)] = composite(T, start + e);
+        } else {   // the cut falls inside this CTA: ordered scan
+            int got = eq_before;
+            for (int base = 0; base < cnt && got < take_eq; base += kRowThreads) {
+                const int e = base + tid;
+                const bool f = e < cnt && key_at(e) == T;
+                const unsigned msk = __ballot_sync(0xffffffffu, f);
+                if (lane == 0) sh->warp_cnt[wp] = __popc(msk);
+                __syncthreads();
+                int before = 0, all = 0;
+                for (int x = 0; x < kRowThreads / 32; ++x) {
+                    before += (x < wp) ? sh->warp_cnt[x] : 0;
+                    all += sh->warp_cnt[x];
+                }
+                const int r = got + before + __popc(msk & ((1u << lane) - 1u));
+                if (f && r < take_eq) dst[gt_row + r] = composite(T, start + e);
+                got += all;
+                __syncthreads();   // warp_cnt is rewritten by the next window
+            }
+        }
+    }
+    cluster_barrier<CL>();   // CTA 0 holds the row's k entries
+    if (rank != 0) return;
+    int S = 1;
+    while (S < k) S <<= 1;
+    for (int e = k + tid; e < S; e += kRowThreads) buf[e] = 0ull;
+    __syncthreads();
+    bitonic_desc(buf, S);
+    for (int e = tid; e < k; e += kRowThreads) {
+        const uint64_t c = buf[e];
+        idx[(int64_t)row * k + e] = (int32_t)(0xFFFFFFFFu - (uint32_t)c);
+        if (top_scores) top_scores[(int64_t)row * k + e] = ordered_to_float((uint32_t)(c >> 32));
+    }
+}
+
+constexpr int kGatherBlocks = 8;   // surviving blocks a warp reads at once
+
+template <int CL>
+__global__ void __launch_bounds__(kRowThreads, 2)
+topk_bmax_rows(const float* __restrict__ scores, const uint32_t* __restrict__ bmax, const __grid_constant__ RowMap m,
+               int k, int32_t* __restrict__ idx, float* __restrict__ top_scores) {
+    pdl_wait();
+    extern __shared__ __align__(16) unsigned char row_smem[];
+    uint32_t* maxima = reinterpret_cast<uint32_t*>(row_smem);                    // [kSliceKeys]
+    uint32_t* hist = maxima + kSliceKeys;                                         // [kBins]
+    uint64_t* buf = reinterpret_cast<uint64_t*>(hist + kBins);                    // [kMaxTopK]
+    uint32_t* hsum = reinterpret_cast<uint32_t*>(buf);                            // range sums, CL > 1
+    __shared__ RowShared sh;
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    int rank = 0;
+    if constexpr (CL > 1) rank = (int)cg::this_cluster().block_rank();
+    const int row = blockIdx.x / CL;
+    int64_t off, n;
+    row_span(m, row, &off, &n);
+    const int64_t nbk = (n + kBlock - 1) / kBlock;
+    const int64_t Lb = (nbk + CL - 1) / CL;   // blocks per CTA, <= kSliceKeys
+    const int64_t b0 = rank * Lb;
+    const int cntb = (int)(nbk - b0 < 0 ? 0 : (nbk - b0 < Lb ? nbk - b0 : Lb));
+    const uint32_t* bm = bmax + off / kBlock + b0;
+    const float* srow = scores + off;
+
+    // this CTA's block maxima, counted into the first histogram as they load
+    for (int b = tid; b < kBins; b += kRowThreads) hist[b] = 0;
+    __syncthreads();
+    for (int b = tid; b < cntb; b += kRowThreads) {
+        const uint32_t v = __ldg(bm + b);
+        maxima[b] = v;
+        atomicAdd(&hist[v >> 20], 1u);
+    }
+    cluster_pick<CL>(hist, hsum, kBins, (uint32_t)k, &sh.bin, &sh.above, &sh.cnt, sh.warp_tot, sh.warp_cnt, &sh.tot);
+    const uint32_t p1 = (uint32_t)sh.bin, need2 = (uint32_t)k - sh.above;
+    __syncthreads();
+    for (int b = tid; b < kBins; b += kRowThreads) hist[b] = 0;   // the pick ended with a cluster barrier
+    __syncthreads();
+    for (int b = tid; b < cntb; b += kRowThreads) {
+        const uint32_t v = maxima[b];
+        if ((v >> 20) == p1) atomicAdd(&hist[(v >> 8) & (kBins - 1)], 1u);
+    }
+    cluster_pick<CL>(hist, hsum, kBins, need2, &sh.bin, &sh.above, &sh.cnt, sh.warp_tot, sh.warp_cnt, &sh.tot);
+    const uint32_t thr = ((p1 << 12) | (uint32_t)sh.bin) << 8;   // <= the k-th largest block maximum
+    if (tid == 0) sh.fill = 0;
+    __syncthreads();
+
+    // the keys >= thr of the blocks whose maximum is >= thr, kGatherBlocks
+    // blocks per warp in flight
+    const unsigned lower = (1u << lane) - 1u;
+    for (int bb = wp * 32; bb < cntb; bb += kRowThreads) {
+        const int b = bb + lane;
+        unsigned msk = __ballot_sync(0xffffffffu, b < cntb && maxima[b] >= thr);
+        while (msk) {   // warp-uniform
+            int src[kGatherBlocks];
+            float x[kGatherBlocks][2];
+#pragma unroll
+            for (int j = 0; j < kGatherBlocks; ++j) {
+                src[j] = msk ? __ffs(msk) - 1 : -1;
+                msk &= msk ? msk - 1 : 0u;
+                if (src[j] >= 0) {
+                    const int64_t i0 = (b0 + bb + src[j]) * kBlock;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int64_t i = i0 + half * 32 + lane;
+                        x[j][half] = (i < n) ? __ldg(srow + i) : 0.0f;
+                    }
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kGatherBlocks; ++j) {
+                if (src[j] < 0) break;   // warp-uniform
+                const int64_t i0 = (b0 + bb + src[j]) * kBlock;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int64_t i = i0 + half * 32 + lane;
+                    const uint32_t key = float_to_ordered(x[j][half]);
+                    const bool keep = i < n && key >= thr;
+                    const unsigned km = __ballot_sync(0xffffffffu, keep);
+                    if (!km) continue;
+                    int base = 0;
+                    if (lane == 0) base = atomicAdd(&sh.fill, __popc(km));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    const int slot = base + __popc(km & lower);
+                    if (keep && slot < kMaxTopK) buf[slot] = composite(key, i);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    const int c_all = sh.fill;   // may exceed kMaxTopK (then only the first kMaxTopK were kept)
+    cluster_barrier<CL>();       // every CTA's count is published
+    int total = 0;
+    if constexpr (CL > 1) {
+        cg::cluster_group cluster = cg::this_cluster();
+#pragma unroll
+        for (int y = 0; y < CL; ++y) total += cluster.map_shared_rank(&sh, y)->fill;
+    } else {
+        total = c_all;
+    }
+    if (total > kMaxTopK) {   // the same decision in every CTA of the row
+        const int64_t L = (n + CL - 1) / CL;
+        const int64_t start = rank * L;
+        const int cnt = (int)(n - start < 0 ? 0 : (n - start < L ? n - start : L));
+        exact_topk_cluster<CL>([&](int e) { return float_to_ordered(srow[start + e]); }, cnt, start, k, hist, buf, &sh,
+                               row, idx, top_scores);
+        return;
+    }
+    int S = 32;
+    while (S < c_all) S <<= 1;
+    for (int e = c_all + tid; e < S; e += kRowThreads) buf[e] = 0ull;   // below every composite of the row
+    __syncthreads();
+    if (S <= kRowThreads) bitonic_desc_reg(buf, S);
+    else bitonic_desc(buf, S);
+    rank_candidates<CL>(maxima, buf, c_all, &sh.fill, row, k, idx, top_scores);
+}
+
+template <int CL>
+cudaError_t launch_topk_bmax_rows_cl(const float* scores, const uint32_t* bmax, const RowMap& map, int rows, int k,
+                                     int32_t* idx, float* top_scores, cudaStream_t stream, bool pdl) {
+    auto kern = topk_bmax_rows<CL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRowSmem);
+    if (e != cudaSuccess) return e;
+    return launch_ex(kern, dim3((unsigned)(rows * CL)), dim3(kRowThreads), kRowSmem, stream, pdl, CL, scores, bmax,
+                     map, k, idx, top_scores);
+}
+
 // rows of at most kRowsMax keys and k <= kMaxTopK
 cudaError_t launch_topk_rows(const float* scores, const RowMap& map, int rows, int k, int32_t* idx,
                              float* top_scores, cudaStream_t stream, bool pdl = false) {
@@ -1223,6 +1475,11 @@ cudaError_t launch_topk_blocks_map(const float* scores, const uint32_t* bmax, co
         return launch_topk_rows(scores, map, rows, k, idx, top_scores, stream, pdl);
     int64_t min_n = map.max_n;
     for (int s = 0; s < map.nsets; ++s) min_n = map.n[s] < min_n ? map.n[s] : min_n;
+    // rows of at least k blocks and at most kMaxCluster * kSliceKeys blocks:
+    // the one-kernel cluster path over the block maxima
+    if (k <= kMaxTopK && (min_n + kBlock - 1) / kBlock >= k &&
+        (map.max_n + kBlock - 1) / kBlock <= (int64_t)kMaxCluster * kSliceKeys)
+        return launch_topk_bmax_rows_cl<kMaxCluster>(scores, bmax, map, rows, k, idx, top_scores, stream, pdl);
     if (min_n / kBlock < 8 * (int64_t)k) return launch_topk_map(scores, map, rows, k, idx, top_scores, ws, stream);
     BlkWs w = carve_blk(ws, rows);
     const size_t smem = sizeof(uint64_t) * kSortMax;

@@ -220,10 +220,12 @@ int fathom_scan_scores(const fathom_store* store, const void* q, int q_dtype, co
  *               that fathom_scan_scores wrote with these scores (ld a
  *               multiple of 64): with m = the k-th largest block maximum of a
  *               row, k keys score at least m, so only the blocks whose
- *               maximum is >= m are read.  The bound is used for rows of at
- *               least 8k blocks; rows of at most 131072 keys are selected in
- *               on-chip memory by one kernel, longer ones by histogram passes
- *               over the whole row.  The result is the same on every path.
+ *               maximum is >= m are read.  Rows of at most 131072 keys are
+ *               selected in on-chip memory by one kernel; longer rows with
+ *               block maxima and at least k blocks (up to 2^23 keys) by one
+ *               cluster kernel over the maxima and the surviving blocks; the
+ *               rest by histogram passes over the whole row.  The result is
+ *               the same on every path.
  *   idx         device, i32 [n_rows][k].
  *   top_scores  device, f32 [n_rows][k], or NULL.
  *   workspace   device, at least fathom_topk_workspace_bytes(n, n_rows, k) bytes,

@@ -298,7 +298,8 @@ def test_topk_bit_exact(ref, n, rows, k, kind):
 
 @pytest.mark.parametrize("n,B,k", [(20000, 92, 2048), (5000, 46, 700), (70000, 0, 1024), (131072, 136, 4096),
                                     (3000, 92, 3000), (131072, 92, 2048), (100000, 68, 1500), (4096, 92, 64),
-                                    (65536, 46, 512)])
+                                    (65536, 46, 512), (300000, 92, 2048), (150001, 46, 777), (1 << 20, 68, 4096),
+                                    (200000, 0, 1000), (524288, 136, 64)])
 def test_topk_from_block_maxima_equals_full_selection(n, B, k):
     """The scan's block maxima let top-k read only the blocks that can hold a
     selected key; the result must equal the selection over the whole rows bit
@@ -327,27 +328,41 @@ def _ordered_keys(s):
     return np.where(neg, ~u, u | np.uint32(0x80000000)).astype(np.uint32)
 
 
-@pytest.mark.parametrize("case", ["ties_at_bound", "k_equals_blocks", "top_in_one_block", "ragged_tail"])
-def test_topk_block_maxima_bound_edge_cases(ref, case):
-    """Short rows with at least k blocks: keys below the smallest block maximum
-    are left out of the first histogram.  Scores built so that the k-th key is
-    that bound itself (all selected keys tie at it), sits just above it, or
-    comes from one block; checked against the oracle bit for bit."""
+@pytest.mark.parametrize("long_rows", [False, True])
+@pytest.mark.parametrize("case", ["ties_at_bound", "k_equals_blocks", "top_in_one_block", "ragged_tail",
+                                  "all_equal", "rounded_ties"])
+def test_topk_block_maxima_bound_edge_cases(ref, case, long_rows):
+    """Rows with at least k blocks, given block maxima computed here.  Short
+    rows (<= 131072 keys) take the one-kernel cluster path over the scores;
+    long rows the cluster path over the block maxima, which keeps the keys at
+    or above the 24-bit bin of the k-th largest block maximum.  Scores built so
+    that all selected keys tie at the k-th block maximum, the top keys sit in
+    one block or in a ragged last block, every score is equal (the candidates
+    overflow and the row is selected exactly from all its keys), or scores are
+    rounded so that ties pile up; checked against the oracle bit for bit."""
     rng = np.random.default_rng(11)
     rows, n = 2, 131072
     if case == "ragged_tail":
         n = 100003
+    if long_rows:
+        n = 4 * n + 17
     nbk = -(-n // 64)
     s = rng.uniform(-1.0, 1.0, (rows, n)).astype(np.float32)
     if case == "ties_at_bound":
-        k = nbk
+        k = min(nbk, 4096)
         s[:, ::64] = 5.0                     # every block's maximum is 5.0: the top k all tie there
     elif case == "k_equals_blocks":
-        k = nbk
+        k = min(nbk, 4096)
         s[:, ::64] = rng.uniform(2.0, 3.0, (rows, nbk)).astype(np.float32)
     elif case == "top_in_one_block":
         k = 1000
         s[:, 64:128] = 10.0 + np.arange(64, dtype=np.float32)
+    elif case == "all_equal":
+        k = 1000
+        s[:] = 1.5
+    elif case == "rounded_ties":
+        k = 2048
+        s = np.round(rng.standard_normal((rows, n)), 1).astype(np.float32)
     else:
         k = 1563
         s[:, -3:] = 7.0                      # the partial last block holds the largest keys
