@@ -1299,7 +1299,7 @@ __device__ void exact_topk_cluster(KeyAt key_at, int cnt, int64_t start, int k, 
     }
 }
 
-constexpr int kGatherBlocks = 8;   // surviving blocks a warp reads at once
+constexpr int kGatherBlocks = 8;   // surviving blocks a half-warp reads at once
 
 template <int CL>
 __global__ void __launch_bounds__(kRowThreads, 2)
@@ -1347,48 +1347,71 @@ topk_bmax_rows(const float* __restrict__ scores, const uint32_t* __restrict__ bm
     if (tid == 0) sh.fill = 0;
     __syncthreads();
 
-    // the keys >= thr of the blocks whose maximum is >= thr, kGatherBlocks
-    // blocks per warp in flight
+    // the numbers of the blocks whose maximum is >= thr (any order) in hist,
+    // which the picks no longer need; each of them holds at least one
+    // candidate, so more than kBins of them means a candidate overflow
     const unsigned lower = (1u << lane) - 1u;
-    for (int bb = wp * 32; bb < cntb; bb += kRowThreads) {
-        const int b = bb + lane;
-        unsigned msk = __ballot_sync(0xffffffffu, b < cntb && maxima[b] >= thr);
-        while (msk) {   // warp-uniform
-            int src[kGatherBlocks];
-            float x[kGatherBlocks][2];
+    if (tid == 0) sh.tot = 0;
+    __syncthreads();
+    for (int b0w = wp * 32; b0w < cntb; b0w += kRowThreads) {
+        const int b = b0w + lane;
+        const bool surv = b < cntb && maxima[b] >= thr;
+        const unsigned sm = __ballot_sync(0xffffffffu, surv);
+        if (!sm) continue;
+        int base = 0;
+        if (lane == 0) base = (int)atomicAdd(&sh.tot, (uint32_t)__popc(sm));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        const int slot = base + __popc(sm & lower);
+        if (surv && slot < kBins) hist[slot] = (uint32_t)b;
+    }
+    __syncthreads();
+    const int nsurv = (int)sh.tot;
+    // the keys >= thr of those blocks: a half-warp reads a block (16 lanes x 4
+    // keys), a warp 2 * kGatherBlocks blocks at once
+    const int hw = lane >> 4, hl = lane & 15;
+    const bool vec = (reinterpret_cast<uintptr_t>(srow) & 15u) == 0;
+    const int nlist = min(nsurv, kBins);
+    for (int q0 = wp * 2 * kGatherBlocks; q0 < nlist; q0 += (kRowThreads / 32) * 2 * kGatherBlocks) {
+        float4 x[kGatherBlocks];
+        int i0[kGatherBlocks];   // a row on this path has at most 2^23 keys
 #pragma unroll
-            for (int j = 0; j < kGatherBlocks; ++j) {
-                src[j] = msk ? __ffs(msk) - 1 : -1;
-                msk &= msk ? msk - 1 : 0u;
-                if (src[j] >= 0) {
-                    const int64_t i0 = (b0 + bb + src[j]) * kBlock;
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int64_t i = i0 + half * 32 + lane;
-                        x[j][half] = (i < n) ? __ldg(srow + i) : 0.0f;
-                    }
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < kGatherBlocks; ++j) {
-                if (src[j] < 0) break;   // warp-uniform
-                const int64_t i0 = (b0 + bb + src[j]) * kBlock;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int64_t i = i0 + half * 32 + lane;
-                    const uint32_t key = float_to_ordered(x[j][half]);
-                    const bool keep = i < n && key >= thr;
-                    const unsigned km = __ballot_sync(0xffffffffu, keep);
-                    if (!km) continue;
-                    int base = 0;
-                    if (lane == 0) base = atomicAdd(&sh.fill, __popc(km));
-                    base = __shfl_sync(0xffffffffu, base, 0);
-                    const int slot = base + __popc(km & lower);
-                    if (keep && slot < kMaxTopK) buf[slot] = composite(key, i);
+        for (int j = 0; j < kGatherBlocks; ++j) {
+            const int q = q0 + 2 * j + hw;
+            i0[j] = -1;
+            x[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (q < nlist) {
+                const int i = (int)((b0 + (int64_t)hist[q]) * kBlock) + 4 * hl;
+                i0[j] = i;
+                if (vec && i + 3 < n) {
+                    x[j] = __ldg(reinterpret_cast<const float4*>(srow + i));
+                } else {
+                    x[j].x = (i < n) ? __ldg(srow + i) : 0.0f;
+                    x[j].y = (i + 1 < n) ? __ldg(srow + i + 1) : 0.0f;
+                    x[j].z = (i + 2 < n) ? __ldg(srow + i + 2) : 0.0f;
+                    x[j].w = (i + 3 < n) ? __ldg(srow + i + 3) : 0.0f;
                 }
             }
         }
+#pragma unroll
+        for (int j = 0; j < kGatherBlocks; ++j) {
+            const float v4[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int i = i0[j] + c;
+                const uint32_t key = float_to_ordered(v4[c]);
+                const bool keep = i0[j] >= 0 && i < n && key >= thr;
+                const unsigned km = __ballot_sync(0xffffffffu, keep);
+                if (!km) continue;
+                int base = 0;
+                if (lane == 0) base = atomicAdd(&sh.fill, __popc(km));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                const int slot = base + __popc(km & lower);
+                if (keep && slot < kMaxTopK) buf[slot] = composite(key, i);
+            }
+        }
     }
+    __syncthreads();
+    if (nsurv > kBins && tid == 0) sh.fill = kMaxTopK + 1;   // too many blocks: the exact selection below
     __syncthreads();
     const int c_all = sh.fill;   // may exceed kMaxTopK (then only the first kMaxTopK were kept)
     cluster_barrier<CL>();       // every CTA's count is published
