@@ -1180,8 +1180,8 @@ cudaError_t launch_topk_rows_cl(const float* scores, const RowMap& map, int rows
 // kMaxCluster * kSliceKeys blocks): one cluster kernel, no workspace.  A
 // cluster of CL CTAs takes a row; CTA x holds the block maxima of its share of
 // the row's blocks in shared memory.  Two radix steps over the maxima (12 and
-// 12 bits, combined through distributed shared memory) give thr = the lower
-// edge of the 24-bit bin of the k-th largest block maximum m.  Every block
+// 8 bits, combined through distributed shared memory) give thr = the lower
+// edge of the 20-bit bin of the k-th largest block maximum m.  Every block
 // holds its maximum, so at least k keys are >= m >= thr, the row's k-th key is
 // >= thr, and every key at or above it lies in a block whose maximum is >= thr:
 // the keys >= thr of those blocks are the candidates (about k of them).  Each
@@ -1340,10 +1340,10 @@ topk_bmax_rows(const float* __restrict__ scores, const uint32_t* __restrict__ bm
     __syncthreads();
     for (int b = tid; b < cntb; b += kRowThreads) {
         const uint32_t v = maxima[b];
-        if ((v >> 20) == p1) atomicAdd(&hist[(v >> 8) & (kBins - 1)], 1u);
+        if ((v >> 20) == p1) atomicAdd(&hist[(v >> 12) & 255u], 1u);
     }
-    cluster_pick<CL>(hist, hsum, kBins, need2, &sh.bin, &sh.above, &sh.cnt, sh.warp_tot, sh.warp_cnt, &sh.tot);
-    const uint32_t thr = ((p1 << 12) | (uint32_t)sh.bin) << 8;   // <= the k-th largest block maximum
+    cluster_pick<CL>(hist, hsum, 256, need2, &sh.bin, &sh.above, &sh.cnt, sh.warp_tot, sh.warp_cnt, &sh.tot);
+    const uint32_t thr = ((p1 << 8) | (uint32_t)sh.bin) << 12;   // <= the k-th largest block maximum
     if (tid == 0) sh.fill = 0;
     __syncthreads();
 
@@ -1372,41 +1372,56 @@ topk_bmax_rows(const float* __restrict__ scores, const uint32_t* __restrict__ bm
     const bool vec = (reinterpret_cast<uintptr_t>(srow) & 15u) == 0;
     const int nlist = min(nsurv, kBins);
     for (int q0 = wp * 2 * kGatherBlocks; q0 < nlist; q0 += (kRowThreads / 32) * 2 * kGatherBlocks) {
-        float4 x[kGatherBlocks];
-        int i0[kGatherBlocks];   // a row on this path has at most 2^23 keys
+        // the keys as ordered u32; a key past the row's end or past the list
+        // reads as 0, below every threshold (thr > 0: the k-th block maximum
+        // is a real score)
+        uint4 x[kGatherBlocks];
 #pragma unroll
         for (int j = 0; j < kGatherBlocks; ++j) {
             const int q = q0 + 2 * j + hw;
-            i0[j] = -1;
-            x[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            x[j] = make_uint4(0u, 0u, 0u, 0u);
             if (q < nlist) {
                 const int i = (int)((b0 + (int64_t)hist[q]) * kBlock) + 4 * hl;
-                i0[j] = i;
                 if (vec && i + 3 < n) {
-                    x[j] = __ldg(reinterpret_cast<const float4*>(srow + i));
+                    const float4 f = __ldg(reinterpret_cast<const float4*>(srow + i));
+                    x[j] = make_uint4(float_to_ordered(f.x), float_to_ordered(f.y), float_to_ordered(f.z),
+                                      float_to_ordered(f.w));
                 } else {
-                    x[j].x = (i < n) ? __ldg(srow + i) : 0.0f;
-                    x[j].y = (i + 1 < n) ? __ldg(srow + i + 1) : 0.0f;
-                    x[j].z = (i + 2 < n) ? __ldg(srow + i + 2) : 0.0f;
-                    x[j].w = (i + 3 < n) ? __ldg(srow + i + 3) : 0.0f;
+                    x[j].x = (i < n) ? float_to_ordered(__ldg(srow + i)) : 0u;
+                    x[j].y = (i + 1 < n) ? float_to_ordered(__ldg(srow + i + 1)) : 0u;
+                    x[j].z = (i + 2 < n) ? float_to_ordered(__ldg(srow + i + 2)) : 0u;
+                    x[j].w = (i + 3 < n) ? float_to_ordered(__ldg(srow + i + 3)) : 0u;
                 }
             }
         }
+        // this lane's candidates, one reservation per warp
+        int mine = 0;
 #pragma unroll
-        for (int j = 0; j < kGatherBlocks; ++j) {
-            const float v4[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
+        for (int j = 0; j < kGatherBlocks; ++j)
+            mine += (x[j].x >= thr) + (x[j].y >= thr) + (x[j].z >= thr) + (x[j].w >= thr);
+        int incl = mine;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int i = i0[j] + c;
-                const uint32_t key = float_to_ordered(v4[c]);
-                const bool keep = i0[j] >= 0 && i < n && key >= thr;
-                const unsigned km = __ballot_sync(0xffffffffu, keep);
-                if (!km) continue;
-                int base = 0;
-                if (lane == 0) base = atomicAdd(&sh.fill, __popc(km));
-                base = __shfl_sync(0xffffffffu, base, 0);
-                const int slot = base + __popc(km & lower);
-                if (keep && slot < kMaxTopK) buf[slot] = composite(key, i);
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const int wtot = __shfl_sync(0xffffffffu, incl, 31);
+        int base = 0;
+        if (lane == 0 && wtot > 0) base = atomicAdd(&sh.fill, wtot);
+        base = __shfl_sync(0xffffffffu, base, 0);
+        int pos = base + incl - mine;
+        if (mine > 0) {
+#pragma unroll
+            for (int j = 0; j < kGatherBlocks; ++j) {
+                const int q = q0 + 2 * j + hw;
+                const uint32_t w4[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (w4[c] >= thr) {
+                        const int i = (int)((b0 + (int64_t)hist[q]) * kBlock) + 4 * hl + c;
+                        if (pos < kMaxTopK) buf[pos] = composite(w4[c], i);
+                        ++pos;
+                    }
             }
         }
     }
