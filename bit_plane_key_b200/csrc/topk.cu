@@ -1179,8 +1179,8 @@ cudaError_t launch_topk_rows_cl(const float* scores, const RowMap& map, int rows
 // Long rows with block maxima (at least k blocks of 64 keys, at most
 // kMaxCluster * kSliceKeys blocks): one cluster kernel, no workspace.  A
 // cluster of CL CTAs takes a row; CTA x holds the block maxima of its share of
-// the row's blocks in shared memory.  Two radix steps over the maxima (12 and
-// 8 bits, combined through distributed shared memory) give thr = the lower
+// the row's blocks in shared memory.  Two radix steps over the maxima (10 and
+// 10 bits, combined through distributed shared memory) give thr = the lower
 // edge of the 20-bit bin of the k-th largest block maximum m.  Every block
 // holds its maximum, so at least k keys are >= m >= thr, the row's k-th key is
 // >= thr, and every key at or above it lies in a block whose maximum is >= thr:
@@ -1325,25 +1325,25 @@ topk_bmax_rows(const float* __restrict__ scores, const uint32_t* __restrict__ bm
     const uint32_t* bm = bmax + off / kBlock + b0;
     const float* srow = scores + off;
 
-    // this CTA's block maxima, counted into the first histogram as they load
+    // this CTA's block maxima, counted into the first (10-bit) histogram as they load
     for (int b = tid; b < kBins; b += kRowThreads) hist[b] = 0;
     __syncthreads();
     for (int b = tid; b < cntb; b += kRowThreads) {
         const uint32_t v = __ldg(bm + b);
         maxima[b] = v;
-        atomicAdd(&hist[v >> 20], 1u);
+        atomicAdd(&hist[v >> 22], 1u);
     }
-    cluster_pick<CL>(hist, hsum, kBins, (uint32_t)k, &sh.bin, &sh.above, &sh.cnt, sh.warp_tot, sh.warp_cnt, &sh.tot);
+    cluster_pick<CL>(hist, hsum, 1024, (uint32_t)k, &sh.bin, &sh.above, &sh.cnt, sh.warp_tot, sh.warp_cnt, &sh.tot);
     const uint32_t p1 = (uint32_t)sh.bin, need2 = (uint32_t)k - sh.above;
     __syncthreads();
-    for (int b = tid; b < kBins; b += kRowThreads) hist[b] = 0;   // the pick ended with a cluster barrier
+    for (int b = tid; b < 1024; b += kRowThreads) hist[b] = 0;   // the pick ended with a cluster barrier
     __syncthreads();
     for (int b = tid; b < cntb; b += kRowThreads) {
         const uint32_t v = maxima[b];
-        if ((v >> 20) == p1) atomicAdd(&hist[(v >> 12) & 255u], 1u);
+        if ((v >> 22) == p1) atomicAdd(&hist[(v >> 12) & 1023u], 1u);
     }
-    cluster_pick<CL>(hist, hsum, 256, need2, &sh.bin, &sh.above, &sh.cnt, sh.warp_tot, sh.warp_cnt, &sh.tot);
-    const uint32_t thr = ((p1 << 8) | (uint32_t)sh.bin) << 12;   // <= the k-th largest block maximum
+    cluster_pick<CL>(hist, hsum, 1024, need2, &sh.bin, &sh.above, &sh.cnt, sh.warp_tot, sh.warp_cnt, &sh.tot);
+    const uint32_t thr = ((p1 << 10) | (uint32_t)sh.bin) << 12;   // <= the k-th largest block maximum
     if (tid == 0) sh.fill = 0;
     __syncthreads();
 
