@@ -46,8 +46,11 @@ def _separate(st, q, s2, B, k, Kr, Vr):
 
 @pytest.mark.parametrize("n,Hkv,Hq,groups,host", [
     (20000, 8, 32, 1, False), (20000, 8, 32, 2, False), (20000, 8, 32, 8, False),
-    (9001, 4, 8, 4, False), (9001, 4, 8, 2, True), (40000, 8, 32, 4, True)])
+    (9001, 4, 8, 4, False), (9001, 4, 8, 2, True), (40000, 8, 32, 4, True),
+    (200001, 4, 16, 1, False), (200001, 4, 16, 2, True)])
 def test_decode_step_equals_separate_calls(n, Hkv, Hq, groups, host):
+    """Rows of up to 131072 keys take the cluster top-k over the scores, the
+    200001-key rows the cluster top-k over the block maxima."""
     inp, q, s2, st, Kr, Vr = _layer(n, Hkv, Hq)
     B, k = 92, 512
     if host:   # host-resident store and interleaved host rows
