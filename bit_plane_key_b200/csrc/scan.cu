@@ -455,7 +455,7 @@ __device__ __forceinline__ void scan_head_tiles(const uint32_t* __restrict__ pla
         for (int h = 0; h < HG; ++h) {
             const int hq = g * G + hg * HG + h;
             float* out = scores + (int64_t)hq * ld + kb;
-            uint32_t kmax = 0u;
+            float fmax_ = -INFINITY;   // the block's largest score (ordered once: the order is monotone)
 #pragma unroll
             for (int wd = 0; wd < 2; ++wd)
 #pragma unroll
@@ -470,8 +470,9 @@ __device__ __forceinline__ void scan_head_tiles(const uint32_t* __restrict__ pla
                         if (kb + o + 1 >= n) v1 = -INFINITY;
                     }
                     *reinterpret_cast<float2*>(out + o) = make_float2(v0, v1);
-                    kmax = max(kmax, max(float_to_ordered(v0), float_to_ordered(v1)));
+                    fmax_ = fmaxf(fmax_, fmaxf(v0, v1));
                 }
+            uint32_t kmax = float_to_ordered(fmax_);
             kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, 1));
             kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, 2));
             if (bmax && p == 0) bmax[(int64_t)hq * (ld / kBlock) + tile0 / kBlock + b] = kmax;
