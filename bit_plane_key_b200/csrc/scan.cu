@@ -235,8 +235,13 @@ __device__ __forceinline__ void scan_head_tiles(const uint32_t* __restrict__ pla
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     // ---- plan: depths, union list, per-(slot, head) factors, item runs ----
+    // the group's depths and queries are read together (the queries parked in
+    // the chunk staging buffer, which the first chunk's loads overwrite only
+    // after the plan)
+    float* s_qraw = reinterpret_cast<float*>(s_raw);   // [G][d]
     for (int e = tid; e < G * d; e += T) {
         int t = depths[(int64_t)g * G * d + e];
+        s_qraw[e] = load_q(q, q_dtype, (int64_t)g * G * d + e);
         if (t > 4) {
             atomicOr(status, (unsigned)FATHOM_DEV_BAD_DEPTH);
             t = 0;
@@ -268,7 +273,7 @@ __device__ __forceinline__ void scan_head_tiles(const uint32_t* __restrict__ pla
         const int a = e / G, hh = e - a * G;
         const int c = s_act[a];
         const int t = s_t[hh * d + c];
-        const float qv = load_q(q, q_dtype, ((int64_t)g * G + hh) * d + c);
+        const float qv = s_qraw[hh * d + c];
         s_qq[e] = (t > 0) ? make_float2(32.0f * qv, qv * (__uint_as_float((uint32_t)(130 - t) << 23) - 24.0f))
                           : make_float2(0.0f, 0.0f);
     }
