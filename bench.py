@@ -321,11 +321,11 @@ def topk_launches(n, k, n_max=None):
 # Link / DRAM bytes per unit (key x KV head) of the scan kernel, from one ncu
 # capture each; the sha256 is that of scan.cu when the counters were taken.
 SCAN_TRAFFIC = {
-    "host": {"kernel_src_sha256": "624b097a73dfd8d5788a0f6d4100e7e92c1f698994e902fd55c79e8c3cfe5e1a",
-             "counter": "pcie__read_bytes.sum", "bytes_per_unit": 54097920 / 2097152, "captured_units": 2097152,
+    "host": {"kernel_src_sha256": "d3377178b224c410f571dd41745b20b4d2e792ad17983a4f860186ce165b9a91",
+             "counter": "pcie__read_bytes.sum", "bytes_per_unit": 54098944 / 2097152, "captured_units": 2097152,
              "capture": "ncu of bench.py --kernel scan --resident host --n 262144"},
-    "hbm": {"kernel_src_sha256": "624b097a73dfd8d5788a0f6d4100e7e92c1f698994e902fd55c79e8c3cfe5e1a",
-            "counter": "dram__bytes_read.sum + dram__bytes_write.sum", "bytes_per_unit": (196147456 + 95932928) / 8388608,
+    "hbm": {"kernel_src_sha256": "d3377178b224c410f571dd41745b20b4d2e792ad17983a4f860186ce165b9a91",
+            "counter": "dram__bytes_read.sum + dram__bytes_write.sum", "bytes_per_unit": (196240896 + 96179200) / 8388608,
             "captured_units": 8388608,
             "capture": "ncu of bench.py --kernel scan --resident hbm --n 1048576"},
 }
