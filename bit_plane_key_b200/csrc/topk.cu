@@ -817,29 +817,6 @@ __device__ __forceinline__ int block_sum_int(int v, int* warp_cnt) {
     return t;
 }
 
-// Exclusive prefix of v over the block's threads in thread order; *total gets
-// the sum.  Called by every thread.
-__device__ __forceinline__ int block_prefix_int(int v, int* warp_cnt, int* total) {
-    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) warp_cnt[wp] = incl;
-    __syncthreads();
-    int before = 0, all = 0;
-    for (int x = 0; x < (int)(blockDim.x >> 5); ++x) {
-        const int c = warp_cnt[x];
-        before += (x < wp) ? c : 0;
-        all += c;
-    }
-    __syncthreads();
-    *total = all;
-    return before + incl - v;
-}
-
 template <int CL>
 __device__ __forceinline__ void cluster_barrier() {
     if constexpr (CL > 1) cg::this_cluster().sync();
@@ -984,6 +961,7 @@ topk_rows(const float* __restrict__ scores, const __grid_constant__ RowMap m, in
     const float* s = scores + off + start;
 
     for (int b = tid; b < kBins; b += kRowThreads) hist[b] = 0;
+    if (tid == 0) s_fill = 0;   // the candidate count (the fast path's reservations)
     __syncthreads();
 
     // the slice as ordered keys in shared memory (thread t: 4-key groups
@@ -1068,8 +1046,17 @@ topk_rows(const float* __restrict__ scores, const __grid_constant__ RowMap m, in
                             (e + 3 < cnt && v.w >= thr);
                 }
             }
-            int c_all = 0;
-            int at = block_prefix_int(mine, warp_cnt, &c_all);
+            // one reservation per warp in the candidate buffer (any order: sorted next)
+            int incl = mine;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int wtot = __shfl_sync(0xffffffffu, incl, 31);
+            int wbase = 0;
+            if (lane == 0 && wtot > 0) wbase = atomicAdd(&s_fill, wtot);
+            int at = __shfl_sync(0xffffffffu, wbase, 0) + incl - mine;
             for (int u = 0; u < kRowVec && mine > 0; ++u) {
                 const int e = 4 * (tid + kRowThreads * u);
                 if (e >= cnt) break;
@@ -1082,13 +1069,14 @@ topk_rows(const float* __restrict__ scores, const __grid_constant__ RowMap m, in
                         --mine;
                     }
             }
+            __syncthreads();
+            const int c_all = s_fill;
             int S = 32;
             while (S < c_all) S <<= 1;
             for (int e = c_all + tid; e < S; e += kRowThreads) buf[e] = 0ull;   // below every composite of the row
             __syncthreads();
             if (S <= kRowThreads) bitonic_desc_reg(buf, S);
             else bitonic_desc(buf, S);
-            if (tid == 0) s_fill = c_all;
             rank_candidates<CL>(keys, buf, c_all, &s_fill, row, k, idx, top_scores);
             return;
         }

@@ -299,7 +299,7 @@ def test_topk_bit_exact(ref, n, rows, k, kind):
 @pytest.mark.parametrize("n,B,k", [(20000, 92, 2048), (5000, 46, 700), (70000, 0, 1024), (131072, 136, 4096),
                                     (3000, 92, 3000), (131072, 92, 2048), (100000, 68, 1500), (4096, 92, 64),
                                     (65536, 46, 512), (300000, 92, 2048), (150001, 46, 777), (1 << 20, 68, 4096),
-                                    (200000, 0, 1000), (524288, 136, 64)])
+                                    (200000, 0, 1000), (524288, 136, 64), (131073, 92, 2048), (131073, 92, 3000)])
 def test_topk_from_block_maxima_equals_full_selection(n, B, k):
     """The scan's block maxima let top-k read only the blocks that can hold a
     selected key; the result must equal the selection over the whole rows bit
