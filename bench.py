@@ -1103,9 +1103,11 @@ def main():
                 "peak_source": "%d SMs x 128 lanes x %.0f MHz (sampled)" % (sms, mhz)}
             layer.store, layer.K_rows, layer.V_rows = keep
         # the pages' other workloads on the same kernels: config 2 (n = 131072,
-        # HBM, B sweep and fixed68/136) and one config-4 batched step
-        extras["config2"] = config12_cases(F, torch, dev, 2, args.steps, args.warmup, flush, with_oracle=False)
-        extras["config4"] = config4_step(F, torch, dev, args.steps, args.warmup, flush, with_oracle=False)
+        # HBM, B sweep and fixed68/136) and one config-4 batched step (one GPU
+        # runs only: they are side measurements, not part of a scaling run)
+        if world == 1:
+            extras["config2"] = config12_cases(F, torch, dev, 2, args.steps, args.warmup, flush, with_oracle=False)
+            extras["config4"] = config4_step(F, torch, dev, args.steps, args.warmup, flush, with_oracle=False)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
