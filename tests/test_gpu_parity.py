@@ -213,6 +213,23 @@ def test_scan_scores(ref, case):
     check_scores(ref, planes, scales, n, q, dep, s)
 
 
+@pytest.mark.parametrize("Hkv,Hq", [(64, 64), (52, 208)])
+def test_scan_scores_wide_grid(ref, Hkv, Hq):
+    """Many KV heads (64 heads of one query, 52 heads of four): grids of
+    1820-2240 CTAs, more than the SMs hold at once, so tiles of one head run
+    in different waves; each head's last 2048-key tile is a half tile and its
+    last block ragged, and depths 0..4 vary per channel and head.  Device- and
+    host-resident stores give the same scores."""
+    inp = make(2, n=70000, Hkv=Hkv, Hq=Hq, d=32)
+    st = F.pack_bitplanes(dev(inp["K"]))
+    planes, scales = ref.pack(inp["K"])
+    dep = np.random.default_rng(5).integers(0, 5, inp["q"].shape).astype(np.uint8)
+    s = host(F.scan_scores(st, q_dev(inp), dev(dep)))
+    assert np.all(np.isneginf(s[:, 70000:]))
+    check_scores(ref, planes, scales, 70000, inp["q"], dep, s)
+    assert np.array_equal(host(F.scan_scores(st.to_host(), q_dev(inp), dev(dep))), s)
+
+
 def test_scan_all_depths_uniform(ref):
     """t = 0..4 for every channel: full-depth and zero-depth corners."""
     inp = make(1, n=700, Hkv=1, Hq=1, d=128)
