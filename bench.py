@@ -861,7 +861,7 @@ def shard_bench(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     # the step's all-gathers run at every world size, one rank included
-    ranks = Ranks("nccl", device=dev, sync=torch.cuda.synchronize, timeout_s=300, always_group=True)
+    ranks = Ranks("nccl", device=dev, sync=torch.cuda.synchronize, timeout_s=180, always_group=True)
     world, rank = ranks.world, ranks.rank
     n, k, B = args.n, args.k, args.budget
     inp = synth.layer_inputs_cuda(3, n=n, device=dev, with_values=True, needles=0, part=rank)
@@ -996,7 +996,7 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    ranks = Ranks("nccl", device=dev, sync=torch.cuda.synchronize)
+    ranks = Ranks("nccl", device=dev, sync=torch.cuda.synchronize, timeout_s=180)
     world, rank = ranks.world, ranks.rank
     from bit_plane_key_b200 import fathom as F
     barrier, max_over_ranks = ranks.barrier, ranks.max
