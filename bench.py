@@ -1036,7 +1036,11 @@ def main():
                 "frac": achieved / link["peak_gbs"], "traffic": traffic, "traffic_source": traffic_src,
                 "algorithmic_bytes": scan_bytes,
                 "peak_source": "measured in this run: max(pinned H2D copy %.1f, SM zero-copy read %.1f) GB/s"
-                               % (link["h2d_copy_gbs"], link["zero_copy_read_gbs"])}
+                               % (link["h2d_copy_gbs"], link["zero_copy_read_gbs"]),
+                # reads issued by the SMs (the kernels' only way to follow data-dependent rows) reach
+                # less of the link than the copy engine: the scan's fraction of that ceiling
+                "sm_read_peak": link["zero_copy_read_gbs"],
+                "frac_of_sm_read": achieved / link["zero_copy_read_gbs"] if link["zero_copy_read_gbs"] > 0 else None}
     else:
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
                 "traffic": traffic, "traffic_source": traffic_src, "algorithmic_bytes": scan_bytes,
